@@ -1,0 +1,345 @@
+"""Pins of the CPU oracle against facts the mathematics fixes (no GPU).
+
+Each test is chosen so that a plausible slip in the oracle (a wrong Hadamard
+construction, a transposed operand, a dropped 1/16, a wrong tie rule, a lost
+scale, a wrong nibble order, a sign error in the epilogue) fails at least one.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import rbd_oracle as O
+from rotated_bit_dit_b200 import inputs as I
+
+H = O.hadamard_regular_kron()
+
+
+# --------------------------------------------------------------- Hadamard
+def test_hadamard_entries_and_orthogonality():
+    assert set(np.unique(H)) == {-1, 1}
+    assert np.array_equal(H @ H.T, 256 * np.eye(256, dtype=np.int64))
+
+
+def test_hadamard_symmetric_and_regular():
+    assert np.array_equal(H, H.T)
+    # regular: every row (and column) sums to sqrt(256) = 16
+    assert np.all(H.sum(axis=1) == 16) and np.all(H.sum(axis=0) == 16)
+
+
+def test_hadamard_two_constructions_agree():
+    assert np.array_equal(H, O.hadamard_regular_digits())
+
+
+def test_hadamard_order4_is_J_minus_2I():
+    h4 = O.hadamard_regular_kron(4)
+    assert np.array_equal(h4, np.array([[-1, 1, 1, 1], [1, -1, 1, 1], [1, 1, -1, 1], [1, 1, 1, -1]]))
+
+
+def test_sylvester_is_a_different_reading():
+    s = O.hadamard_sylvester()
+    assert np.array_equal(s @ s.T, 256 * np.eye(256, dtype=np.int64))
+    assert not np.array_equal(s, H)
+    # Sylvester is not regular: its row sums are 256, 0, 0, ...
+    assert s.sum(axis=1)[0] == 256 and s.sum(axis=1)[1] == 0
+
+
+# --------------------------------------------------------------- rotation
+def _rand_bf16(seed, shape, std=1.0, frac=0.0, scale=1.0):
+    return O.bf16_to_f64(I.gaussian_bf16(seed, shape, std, frac, scale))
+
+
+def test_rotation_constant_block_is_fixed_point():
+    # regularity: R (c 1) = c 1 (each column of H sums to 16)
+    for c in (1.0, -3.5, 0.015625):
+        x = np.full((1, 256), c)
+        assert np.array_equal(O.rotate(x), np.full((1, 256), c, dtype=np.float32))
+    # the Sylvester reading maps a constant block to (16c, 0, 0, ...)
+    s = O.hadamard_sylvester().astype(np.float64) / 16
+    y = np.full((1, 256), 2.0) @ s
+    assert y[0, 0] == 32.0 and np.all(y[0, 1:] == 0)
+
+
+def test_rotation_unit_vector_is_a_column_over_16():
+    for j in (0, 5, 255):
+        x = np.zeros((1, 256))
+        x[0, j] = 1.0
+        y = O.rotate(x)[0]
+        assert np.array_equal(y, (H[:, j] / 16.0).astype(np.float32))
+        assert set(np.abs(y)) == {np.float32(1 / 16)}
+
+
+def test_rotation_is_an_involution_in_float64():
+    # R = R^T and R R^T = I, so rotating twice returns the input exactly
+    x = _rand_bf16(11, (4, 512))
+    r = O.rotation_matrix()
+    xg = x.reshape(4, 2, 256)
+    assert np.array_equal(np.matmul(np.matmul(xg, r), r), xg)
+
+
+def test_rotation_groups_are_independent_blocks():
+    x = _rand_bf16(12, (3, 768))
+    y = O.rotate(x)
+    for g in range(3):
+        assert np.array_equal(y[:, 256 * g:256 * (g + 1)], O.rotate(x[:, 256 * g:256 * (g + 1)]))
+
+
+def test_rotation_matches_exact_rationals():
+    # brute force: exact rational sum, rounded once to float32
+    x = _rand_bf16(13, (2, 256), 1.0, 0.05, 30.0)
+    got = O.rotate(x)
+    for r in range(2):
+        assert np.array_equal(got[r], O.rotate_exact_fraction(x[r]))
+
+
+def test_rotation_wide_exponent_span_uses_exact_path():
+    # a group whose exponent span exceeds the float64 exactness bound
+    x = np.zeros((1, 256))
+    x[0, 0] = 2.0 ** 60
+    x[0, 1] = 2.0 ** -40 * 1.5
+    x[0, 2] = 3.0
+    assert not O._group_span_ok(x.reshape(1, 1, 256)).all()
+    assert np.array_equal(O.rotate(x)[0], O.rotate_exact_fraction(x[0]))
+
+
+def test_rotation_preserves_products_before_quantisation():
+    # X W^T = (X R)(W R)^T per block, float64, to 1e-12 relative
+    x = _rand_bf16(14, (8, 512), 1.0, 0.01, 20.0)
+    w = _rand_bf16(15, (16, 512), 0.02)
+    r = O.rotation_matrix()
+    xr = np.matmul(x.reshape(8, 2, 256), r).reshape(8, 512)
+    wr = np.matmul(w.reshape(16, 2, 256), r).reshape(16, 512)
+    ref = x @ w.T
+    assert np.max(np.abs(xr @ wr.T - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_no_rotation_mode_is_identity():
+    x = _rand_bf16(16, (2, 256))
+    assert np.array_equal(O.rotate(x, 0), x.astype(np.float32))
+
+
+# --------------------------------------------------------------- quantiser
+@pytest.mark.parametrize("bits", [4, 8])
+def test_quantiser_is_nearest_code_with_even_ties(bits):
+    qmax = O.qmax_of(bits)
+    xr = O.rotate(_rand_bf16(17, (16, 256), 1.0, 0.02, 20.0))
+    q, s = O.quantize(xr, bits)
+    codes = np.arange(-qmax - 1, qmax + 1)
+    for m in range(xr.shape[0]):
+        amax = np.float32(np.abs(xr[m]).max())
+        inv = np.float32(np.float32(qmax) / amax)
+        assert s[m] == np.float32(amax / np.float32(qmax))
+        t = (xr[m] * inv).astype(np.float32).astype(np.float64)
+        d = np.abs(t[:, None] - codes[None, :])
+        best = d.min(axis=1, keepdims=True)
+        cand = np.where(d == best, codes[None, :], 10 ** 6)
+        # ties: prefer the even code
+        even = np.where((cand % 2 == 0) & (cand != 10 ** 6), cand, 10 ** 6).min(axis=1)
+        first = cand.min(axis=1)
+        expect = np.where((d == best).sum(axis=1) > 1, even, first)
+        assert np.array_equal(q[m].astype(np.int64), expect)
+
+
+def test_quantiser_error_bound():
+    for bits in (4, 8):
+        xr = O.rotate(_rand_bf16(18, (32, 512), 1.0, 0.01, 30.0))
+        q, s = O.quantize(xr, bits)
+        err = np.abs(xr.astype(np.float64) - q.astype(np.float64) * s[:, None].astype(np.float64))
+        assert np.all(err <= s[:, None] / 2 * (1 + 2.0 ** -20))
+
+
+def test_quantiser_range_and_extremes():
+    xr = O.rotate(_rand_bf16(19, (8, 256)))
+    q, s = O.quantize(xr, 4)
+    assert q.min() >= -7 and q.max() <= 7          # -8 is never produced by symmetric scaling
+    amax_idx = np.abs(xr).argmax(axis=1)
+    assert np.all(np.abs(q[np.arange(8), amax_idx]) == 7)
+
+
+def test_quantiser_half_way_ties():
+    # amax = 7 -> inv = 1: values k + 0.5 must go to the even neighbour
+    xr = np.zeros((1, 256), dtype=np.float32)
+    xr[0, :8] = [7.0, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.5]
+    q, s = O.quantize(xr, 4)
+    assert s[0] == 1.0
+    assert list(q[0, :8]) == [7, 0, 2, 2, 0, -2, -2, 4]
+
+
+def test_zero_row_and_zero_group():
+    xr = np.zeros((2, 128), dtype=np.float32)
+    xr[1, 64:] = 1.0
+    q, s = O.quantize(xr, 4, scale_group=64)
+    assert np.all(q[0] == 0) and np.all(s[0] == 0)
+    assert s[1, 0] == 0 and np.all(q[1, :64] == 0)
+    assert s[1, 1] == np.float32(1 / np.float32(7)) and np.all(q[1, 64:] == 7)
+
+
+def test_group_scales_equal_row_scale_when_groups_share_amax():
+    xr = np.tile(np.linspace(-1, 1, 64, dtype=np.float32), (3, 4))
+    q_row, s_row = O.quantize(xr, 4)
+    q_g, s_g = O.quantize(xr, 4, scale_group=64)
+    assert np.array_equal(q_row, q_g)
+    assert np.all(s_g == s_row[:, None])
+
+
+# --------------------------------------------------------------- packing
+def test_pack_nibble_order_and_twos_complement():
+    q = np.array([[1, -1, 7, -8, 0, 3]], dtype=np.int8)
+    p = O.pack_int4(q)
+    # byte 0: low nibble k=0 (1), high nibble k=1 (-1 -> 0xF) -> 0xF1
+    assert list(p[0]) == [0xF1, 0x87, 0x30]
+    assert np.array_equal(O.unpack_int4(p), q)
+
+
+def test_pack_roundtrip_all_codes():
+    q = np.array([np.arange(-8, 8)] * 2, dtype=np.int8)
+    assert np.array_equal(O.unpack_int4(O.pack_int4(q)), q)
+
+
+# --------------------------------------------------------------- GEMM
+def test_gemm_matches_loops_on_tiny_shapes():
+    rng = np.random.default_rng(0)
+    qx = rng.integers(-8, 8, (3, 256)).astype(np.int8)
+    qw = rng.integers(-8, 8, (4, 256)).astype(np.int8)
+    assert np.array_equal(O.gemm_acc(qx, qw), O.gemm_acc_loops(qx, qw))
+
+
+def test_gemm_hand_expanded():
+    qx = np.array([[1, 2, 3, 4]], dtype=np.int8)
+    qw = np.array([[1, 0, -1, 2], [7, 7, 7, 7]], dtype=np.int8)
+    assert O.gemm_acc(qx, qw).tolist() == [[1 - 3 + 8, 70]]
+
+
+def test_unrotated_integer_inputs_reduce_to_integer_matmul():
+    # rot_group=0, integer inputs in [-7,7] whose row amax is 7: scales are 1, codes = inputs
+    rng = np.random.default_rng(1)
+    xi = rng.integers(-7, 8, (5, 64)).astype(np.float64)
+    wi = rng.integers(-7, 8, (6, 64)).astype(np.float64)
+    xi[:, 0] = 7
+    wi[:, 0] = 7
+    xb = I.f32_to_bf16_bits(xi.astype(np.float32))
+    wb = I.f32_to_bf16_bits(wi.astype(np.float32))
+    out = O.linear_reference(xb, wb, 4, rot_group=0)
+    assert np.all(out["sx"] == 1) and np.all(out["sw"] == 1)
+    assert np.array_equal(out["y64"], xi @ wi.T)
+
+
+def test_group_partials_sum_to_row_accumulator():
+    rng = np.random.default_rng(2)
+    qx = rng.integers(-7, 8, (4, 256)).astype(np.int8)
+    qw = rng.integers(-7, 8, (5, 256)).astype(np.int8)
+    assert np.array_equal(O.gemm_acc_grouped(qx, qw, 64).sum(axis=0), O.gemm_acc(qx, qw))
+    ones_x = np.ones((4, 4), np.float32)
+    ones_w = np.ones((5, 4), np.float32)
+    assert np.allclose(O.dequant(qx, ones_x, qw, ones_w, 64), O.gemm_acc(qx, qw))
+
+
+def test_dequant_scales_each_operand_once():
+    rng = np.random.default_rng(3)
+    qx = rng.integers(-7, 8, (2, 64)).astype(np.int8)
+    qw = rng.integers(-7, 8, (3, 64)).astype(np.int8)
+    sx = np.array([2.0, 0.5], np.float32)
+    sw = np.array([1.0, 4.0, 0.25], np.float32)
+    acc = O.gemm_acc(qx, qw)
+    assert np.array_equal(O.dequant(qx, sx, qw, sw), acc * np.outer(sx, sw))
+
+
+# --------------------------------------------------------------- epilogue
+def test_epilogue_special_cases():
+    rng = np.random.default_rng(4)
+    y = rng.standard_normal((4, 8))
+    res = I.gaussian_bf16(5, (4, 8))
+    zero_g = np.zeros(8, dtype=np.uint16)
+    # g = 0: out = residual
+    assert np.array_equal(O.epilogue(y, gate_mode=2, gate_bits=zero_g, residual_bits=res), O.bf16_to_f64(res))
+    # g = 1, residual = 0: out = y
+    one_g = I.f32_to_bf16_bits(np.ones(8, np.float32))
+    zres = np.zeros((4, 8), np.uint16)
+    assert np.array_equal(O.epilogue(y, gate_mode=2, gate_bits=one_g, residual_bits=zres), y)
+    # L2 = 0 leaves y unchanged; bias adds per column
+    ld = rng.standard_normal((4, 2))
+    assert np.array_equal(O.epilogue(y, ld=ld, l2_bits=np.zeros((2, 8), np.uint16)), y)
+    b = I.f32_to_bf16_bits(np.arange(8, dtype=np.float32))
+    assert np.array_equal(O.epilogue(y, bias=b), y + np.arange(8)[None, :])
+    # sigmoid on the gate columns only; sigmoid(0) = 1/2 exactly
+    z = np.zeros((2, 8))
+    out = O.epilogue(z, gate_mode=1, gate_cols=(4, 8))
+    assert np.all(out[:, 4:] == 0.5) and np.all(out[:, :4] == 0.0)
+
+
+def test_lowrank_branch_is_parallel_linear():
+    # (W + L1 L2)-style branch: X L1 L2 added once, on the unrotated input
+    x = I.gaussian_bf16(6, (3, 256))
+    l1 = I.gaussian_bf16(7, (256, 4), 0.1)
+    l2 = I.gaussian_bf16(8, (4, 5), 0.1)
+    ld = O.lowrank_down(x, l1)
+    xd, l1d, l2d = O.bf16_to_f64(x), O.bf16_to_f64(l1), O.bf16_to_f64(l2)
+    assert np.allclose(O.epilogue(np.zeros((3, 5)), ld=ld, l2_bits=l2), xd @ (l1d @ l2d), rtol=1e-12, atol=1e-15)
+
+
+def test_bf16_rounding_ties_and_against_torch():
+    # direct float64 -> bf16, nearest even; compare with torch on float32-exact values
+    rng = np.random.default_rng(5)
+    v = rng.standard_normal(20000).astype(np.float32).astype(np.float64)
+    ref = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.f64_to_bf16(v), ref)
+    # exact ties: 1 + 2^-8 lies half-way between 1 and 1 + 2^-7 -> 1 (even)
+    assert O.f64_to_bf16(np.array([1 + 2.0 ** -8]))[0] == 0x3F80
+    assert O.f64_to_bf16(np.array([1 + 3 * 2.0 ** -8]))[0] == 0x3F82
+    # a value just above the tie in float64 (not representable in float32) rounds up
+    assert O.f64_to_bf16(np.array([1 + 2.0 ** -8 + 2.0 ** -40]))[0] == 0x3F81
+
+
+def test_end_to_end_tiny_layer_matches_float_reference():
+    # at 4 bits the quantised layer stays close to the float layer (sanity of scale placement)
+    cfg = I.CONFIGS["tiny_w4a4"]
+    t = I.make_layer_inputs(cfg, seed=0)
+    out = O.linear_reference(t["x"], t["w"], 4)
+    ref = O.bf16_to_f64(t["x"]) @ O.bf16_to_f64(t["w"]).T
+    rel = np.linalg.norm(out["y64"] - ref) / np.linalg.norm(ref)
+    assert rel < 0.25
+    # and reconstructing from codes reproduces y64
+    qw = O.unpack_int4(out["wq"])
+    xd = out["codes"].astype(np.float64) * out["sx"].astype(np.float64)[:, None]
+    wd = qw.astype(np.float64) * out["sw"].astype(np.float64)[:, None]
+    assert np.allclose(out["y64"], xd @ wd.T, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------- NVFP4
+def test_e2m1_rounding_brute_force():
+    grid = np.concatenate([-O.E2M1_GRID[::-1], O.E2M1_GRID])
+    enc = {0.0: 0, 0.5: 1, 1.0: 2, 1.5: 3, 2.0: 4, 3.0: 5, 4.0: 6, 6.0: 7}
+    vals = np.concatenate([np.linspace(-7, 7, 2801), [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]])
+    got = O.round_e2m1(vals)
+    for v, g in zip(vals, got):
+        a = min(abs(v), 6.0)
+        d = np.abs(np.abs(grid) - a)
+        best = d.min()
+        cands = sorted({abs(float(x)) for x in grid[d == best]})
+        pick = cands[0] if len(cands) == 1 else [c for c in cands if enc[c] % 2 == 0][0]
+        assert abs(g) == pick and (g == 0 or np.sign(g) == np.sign(v))
+
+
+def test_e4m3_rounding_against_torch():
+    rng = np.random.default_rng(6)
+    v = np.concatenate([rng.standard_normal(20000) * 50, rng.standard_normal(2000) * 1e-2,
+                        [448.0, -448.0, 0.0, 2.0 ** -9, 3 * 2.0 ** -10]]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    sel = np.abs(v) <= 448
+    assert np.array_equal(O.round_e4m3(v.astype(np.float64))[sel], ref[sel])
+    assert np.all(O.round_e4m3(np.array([1000.0, -500.0])) == [448.0, -448.0])
+
+
+def test_nvfp4_block_error_bound_and_scale_range():
+    xr = O.rotate(_rand_bf16(20, (8, 512), 1.0, 0.01, 30.0))
+    q, bs, gs = O.nvfp4_quantize(xr)
+    deq = q * np.repeat(bs, 16, axis=1) * float(gs)
+    assert np.all(bs <= 448) and np.all(bs >= 0)
+    # the block holding the tensor amax has scale 448 (up to E4M3 rounding of the ratio)
+    assert bs.max() == 448.0
+    # error within half a grid step at the largest step (2 * bs * gs) per element, plus scale rounding
+    step = 2.0 * np.repeat(bs, 16, axis=1) * float(gs)
+    assert np.all(np.abs(xr - deq) <= step / 2 * 1.0001 + 1e-30)
+    rel = np.linalg.norm(xr - deq) / np.linalg.norm(xr)
+    assert rel < 0.12
