@@ -1,0 +1,175 @@
+/*
+ * rbd.h -- C ABI of the rotated low-bit quantized linear layer (B200, sm_100a).
+ *
+ * The layer (as described on the Krea-2 model cards):
+ *   - bf16 activations are rotated online, group-wise, by a 256-wide regular
+ *     Hadamard matrix and quantised per token inside the kernel
+ *     ("Krea-2 Turbo -- INT4 tensorwise W4A4 (+ConvRot, mixed int8 fallback)",
+ *     header paragraph);
+ *   - weights are rotated the same way and packed offline to signed INT4, or
+ *     kept as per-row INT8 for the protected ff.down layers
+ *     ("Krea 2 Turbo OrbitQuant W4A4", sections "Fused transformer" and
+ *     "What is quantized");
+ *   - the low-bit GEMM accumulates in int32; scales, bias, an optional
+ *     SVDQuant-style low-rank branch and a sigmoid gate or gated residual are
+ *     applied in the epilogue ("Fused transformer"; "Krea-2-SVDQuant-ComfyUI",
+ *     sections "Why this exists" and "LoRA");
+ *   - group-64 scales follow "Krea 2 Turbo Nunchaku Lite INT4 r32", header.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named x, w, codes, scales, y, ... are DEVICE pointers owned by
+ *     the caller; the library allocates no device memory and never frees.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     enqueued asynchronously on it; no call synchronises the host except
+ *     rbd_check().
+ *   - bf16 tensors are passed as `const void*` holding IEEE bfloat16 bits.
+ *   - All matrices are row-major.  ld* arguments are row strides in elements.
+ *   - Arguments are validated on the host before anything is launched.  An
+ *     invalid call returns a non-zero rbd_status and launches nothing.  There
+ *     is no fallback path: an unsupported shape or mode is an error.
+ *   - A kernel whose bounded wait expires records RBD_ERR_DEVICE_TIMEOUT in a
+ *     device status word; rbd_check() reports (and clears) it.
+ */
+#ifndef RBD_H_
+#define RBD_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum rbd_status {
+  RBD_OK = 0,
+  RBD_ERR_INVALID_ARG = 1,    /* null pointer, bad size or inconsistent arguments */
+  RBD_ERR_UNSUPPORTED = 2,    /* valid request this library does not implement   */
+  RBD_ERR_ALIGNMENT = 3,      /* pointer or stride not 16-byte aligned           */
+  RBD_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed               */
+  RBD_ERR_DEVICE_TIMEOUT = 5  /* a device-side bounded wait expired              */
+} rbd_status;
+
+/* Quantisation configuration.
+ *   bits        4 (signed INT4, codes in [-8,7], produced range [-7,7]) or
+ *               8 (signed INT8, produced range [-127,127]).
+ *   rot_group   256: rotate every 256-wide K block by R = H/16, H the regular
+ *               Hadamard matrix (J4 - 2 I4) Kronecker-powered four times;
+ *               0: no rotation.
+ *   scale_group 0: one scale per row (per token for activations, per output
+ *               channel for weights); 64: one scale per 64-wide K block of a
+ *               row (group-64 scales).                                        */
+typedef struct rbd_qcfg {
+  int32_t bits;
+  int32_t rot_group;
+  int32_t scale_group;
+} rbd_qcfg;
+
+/* Online activation rotate + dynamic quantise (INT4 tensorwise card, header:
+ * "activations rotated online and dynamically quantized inside the kernel").
+ *   x       bf16 [M, ldx], first K columns used.  ldx >= K, ldx % 8 == 0,
+ *           x 16-byte aligned.
+ *   M       >= 0 (M == 0 is a no-op).   K: multiple of 256 (rotation) or of 64,
+ *           K <= 16384.
+ *   codes   int8 [M, K] (one code per byte), 16-byte aligned.
+ *   scales  float32 [M] (scale_group 0) or [M, K/64] (scale_group 64);
+ *           dequantised value = code * scale.
+ * Per row (or per 64 block): amax = max |xr|, scale = amax/qmax,
+ * code = clamp(rint_even(xr * (qmax/amax))), all float32 IEEE operations, xr the
+ * exact rotated value rounded once to float32.  An all-zero row or block gets
+ * scale 0 and codes 0.                                                         */
+rbd_status rbd_rot_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, rbd_qcfg cfg,
+                             int8_t* codes, float* scales, void* stream);
+
+/* rbd_rot_quant_act plus the first factor of the low-rank branch on the
+ * UNROTATED input: ld = X L1 (Krea-2-SVDQuant-ComfyUI, "LoRA": the branch is a
+ * parallel linear, (W + L2 L1) x = W x + L2 (L1 x)).
+ *   l1      bf16 [K, r] row-major.     r in {16, 32, 64}.
+ *   ld      bf16 [M, r] row-major (float32 accumulation, rounded once).       */
+rbd_status rbd_lowrank_fused(const void* x, int64_t M, int64_t K, int64_t ldx, rbd_qcfg cfg,
+                             int8_t* codes, float* scales, const void* l1, int32_t r, void* ld,
+                             void* stream);
+
+/* Offline weight rotate + quantise + pack to signed INT4 (INT4 tensorwise card,
+ * header: "packed signed INT4 weights with group-256 ... rotation").
+ * Each output row of W is rotated and quantised exactly like a token.
+ *   w       bf16 [N, K] row-major, 16-byte aligned.    cfg.bits must be 4.
+ *   packed  uint8 [N, K/2]: byte k/2 of row n holds code k (even k) in the low
+ *           nibble and code k+1 in the high nibble, two's complement.
+ *   scales  float32 [N] or [N, K/64].                                          */
+rbd_status rbd_pack_weights_int4(const void* w, int64_t N, int64_t K, rbd_qcfg cfg,
+                                 uint8_t* packed, float* scales, void* stream);
+
+/* Offline per-row INT8 weights for the protected ff.down layers (OrbitQuant
+ * card, "What is quantized": per-row INT8 weights for a W8A8 GEMM).
+ *   w8      int8 [N, K].  cfg.bits must be 8.                                  */
+rbd_status rbd_pack_weights_int8(const void* w, int64_t N, int64_t K, rbd_qcfg cfg,
+                                 int8_t* w8, float* scales, void* stream);
+
+/* Epilogue options of the linear calls ("Fused transformer": sigmoid gate in
+ * the Q|K|V|gate GEMM epilogue, gated residual updates in the GEMM epilogues;
+ * "What is quantized": biases are not 4-bit tensors).
+ *   bias      bf16 [N] or NULL.
+ *   ld, l2t   low-rank branch: ld bf16 [M, r] (from rbd_lowrank_fused) and the
+ *             second factor stored output-major, l2t bf16 [N, r] (the
+ *             nn.Linear layout of the up projection; the branch adds
+ *             ld @ l2t^T).  r in {16, 32, 64}; r = 0 disables the branch.
+ *   gate_mode 0: none.  1: sigmoid on output columns [gate_col0, gate_col1).
+ *             2: out = residual + gate[n] * y (gated residual).
+ *   gate      bf16 [N] (gate_mode 2).   residual bf16 [M, ldr] (gate_mode 2).
+ *   acc_debug NULL, or int32 receiving the exact integer accumulators:
+ *             [M, N] with scale_group 0, [K/64, M, N] with scale_group 64.
+ *             Meant for small checks; it adds a full int32 write per output.
+ * Order: y = dequant(acc) + bias + ld l2t^T, then the gate, one round to bf16. */
+typedef struct rbd_epilogue {
+  const void* bias;
+  const void* ld;
+  const void* l2t;
+  int32_t r;
+  int32_t gate_mode;
+  int64_t gate_col0;
+  int64_t gate_col1;
+  const void* gate;
+  const void* residual;
+  int64_t ldr;
+  int32_t* acc_debug;
+} rbd_epilogue;
+
+/* W4A4 linear: INT4 activation codes (int8 containers, from rbd_rot_quant_act
+ * with bits 4) times packed INT4 weights (rbd_pack_weights_int4), int32
+ * accumulation on the tcgen05 INT8 tensor path, then the epilogue.
+ *   codes   int8 [M, K], sx float32 [M] or [M, K/64].
+ *   w_packed uint8 [N, K/2], sw float32 [N] or [N, K/64].
+ *   K % 128 == 0, N % 128 == 0, M >= 1 (ragged M is handled).
+ *   epi     may be NULL (no bias, branch or gate).
+ *   y       bf16 [M, ldy], ldy >= N, ldy % 8 == 0.                           */
+rbd_status rbd_w4a4_linear(const int8_t* codes, const float* sx, const uint8_t* w_packed,
+                           const float* sw, int64_t M, int64_t N, int64_t K, rbd_qcfg cfg,
+                           const rbd_epilogue* epi, void* y, int64_t ldy, void* stream);
+
+/* W8A8 linear (per-row INT8 ff.down): INT8 codes times INT8 weights.
+ * Same contract as rbd_w4a4_linear with w8 int8 [N, K] and cfg.bits == 8.   */
+rbd_status rbd_w8a8_linear(const int8_t* codes, const float* sx, const int8_t* w8,
+                           const float* sw, int64_t M, int64_t N, int64_t K, rbd_qcfg cfg,
+                           const rbd_epilogue* epi, void* y, int64_t ldy, void* stream);
+
+/* Synchronises `stream`, then reports the first device-side error recorded
+ * since the last rbd_check (RBD_ERR_DEVICE_TIMEOUT) or a CUDA error, and
+ * clears the device status word.                                              */
+rbd_status rbd_check(void* stream);
+
+/* Launches a single-thread kernel that waits on an mbarrier nobody signals,
+ * bounded by timeout_ns, then records RBD_ERR_DEVICE_TIMEOUT.  It exercises
+ * the device-side timeout path without hanging or faulting the GPU; follow it
+ * with rbd_check().                                                           */
+rbd_status rbd_debug_timeout_probe(int64_t timeout_ns, void* stream);
+
+/* Human-readable name of a status code (static storage).                     */
+const char* rbd_status_string(rbd_status s);
+
+/* Library version string (static storage).                                  */
+const char* rbd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RBD_H_ */

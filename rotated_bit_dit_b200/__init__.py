@@ -1,0 +1,26 @@
+"""rotated_bit_dit_b200: the rotated low-bit quantized linear layer on B200 (sm_100a).
+
+The compute runs in librbd.so (hand-written CUDA for sm_100a behind a C ABI,
+include/rbd.h); this package is the ctypes binding plus a small layer object.
+Importing the package does not load the library; the first call does, and it
+raises if the library cannot be loaded (there is no CPU fallback).
+"""
+from ._binding import (  # noqa: F401
+    EXPORTED,
+    Epilogue,
+    QCfg,
+    RbdError,
+    load,
+    make_epilogue,
+    rbd_check,
+    rbd_debug_timeout_probe,
+    rbd_lowrank_fused,
+    rbd_pack_weights_int4,
+    rbd_pack_weights_int8,
+    rbd_rot_quant_act,
+    rbd_status_string,
+    rbd_version,
+    rbd_w4a4_linear,
+    rbd_w8a8_linear,
+)
+from .layer import RotatedLowBitLinear  # noqa: F401

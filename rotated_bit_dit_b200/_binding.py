@@ -1,0 +1,205 @@
+"""ctypes binding of librbd.so: the same entry points as include/rbd.h.
+
+Argument marshalling only.  Every computation runs in the library's CUDA
+kernels; there is no Python or CPU fallback.  Tensors must be CUDA tensors on
+the current device; the current torch stream is used unless `stream` is given.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+RBD_OK = 0
+STATUS_NAMES = {0: "RBD_OK", 1: "RBD_ERR_INVALID_ARG", 2: "RBD_ERR_UNSUPPORTED", 3: "RBD_ERR_ALIGNMENT",
+                4: "RBD_ERR_CUDA", 5: "RBD_ERR_DEVICE_TIMEOUT"}
+
+EXPORTED = ("rbd_rot_quant_act", "rbd_lowrank_fused", "rbd_pack_weights_int4", "rbd_pack_weights_int8",
+            "rbd_w4a4_linear", "rbd_w8a8_linear", "rbd_check", "rbd_debug_timeout_probe",
+            "rbd_status_string", "rbd_version")
+
+
+class RbdError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class QCfg(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int32), ("rot_group", ctypes.c_int32), ("scale_group", ctypes.c_int32)]
+
+
+class Epilogue(ctypes.Structure):
+    _fields_ = [("bias", ctypes.c_void_p), ("ld", ctypes.c_void_p), ("l2t", ctypes.c_void_p),
+                ("r", ctypes.c_int32), ("gate_mode", ctypes.c_int32), ("gate_col0", ctypes.c_int64),
+                ("gate_col1", ctypes.c_int64), ("gate", ctypes.c_void_p), ("residual", ctypes.c_void_p),
+                ("ldr", ctypes.c_int64), ("acc_debug", ctypes.c_void_p)]
+
+
+_LIB = None
+
+
+def lib_path() -> str:
+    return _build.LIB_PATH
+
+
+def load(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load librbd.so (building it first when absent).  Raises if it cannot be loaded."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = lib_path()
+    if not os.path.exists(path):
+        if not build_if_missing:
+            raise RuntimeError(f"librbd.so not built: {path}")
+        _build.build()
+    lib = ctypes.CDLL(path)
+    i64, i32, vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p
+    sigs = {
+        "rbd_rot_quant_act": [vp, i64, i64, i64, QCfg, vp, vp, vp],
+        "rbd_lowrank_fused": [vp, i64, i64, i64, QCfg, vp, vp, vp, i32, vp, vp],
+        "rbd_pack_weights_int4": [vp, i64, i64, QCfg, vp, vp, vp],
+        "rbd_pack_weights_int8": [vp, i64, i64, QCfg, vp, vp, vp],
+        "rbd_w4a4_linear": [vp, vp, vp, vp, i64, i64, i64, QCfg, ctypes.POINTER(Epilogue), vp, i64, vp],
+        "rbd_w8a8_linear": [vp, vp, vp, vp, i64, i64, i64, QCfg, ctypes.POINTER(Epilogue), vp, i64, vp],
+        "rbd_check": [vp],
+        "rbd_debug_timeout_probe": [i64, vp],
+    }
+    for name, args in sigs.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.rbd_status_string.argtypes = [ctypes.c_int]
+    lib.rbd_status_string.restype = ctypes.c_char_p
+    lib.rbd_version.argtypes = []
+    lib.rbd_version.restype = ctypes.c_char_p
+    _LIB = lib
+    return lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ok(status: int, where: str):
+    if status != RBD_OK:
+        raise RbdError(status, where)
+
+
+def _qcfg(bits: int, rot_group: int, scale_group: int) -> QCfg:
+    return QCfg(bits, rot_group, scale_group)
+
+
+def _rowstride(t: torch.Tensor) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D row-major tensor")
+    return t.stride(0)
+
+
+# ---------------------------------------------------------------- entry points
+def rbd_rot_quant_act(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, bits: int = 4,
+                      rot_group: int = 256, scale_group: int = 0, stream=None) -> None:
+    """x bf16 [M, K] -> codes int8 [M, K], scales float32 [M] or [M, K/64]."""
+    M, K = x.shape
+    _ok(load().rbd_rot_quant_act(_ptr(x), M, K, _rowstride(x), _qcfg(bits, rot_group, scale_group),
+                                 _ptr(codes), _ptr(scales), _stream(stream)), "rbd_rot_quant_act")
+
+
+def rbd_lowrank_fused(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, l1: torch.Tensor,
+                      ld: torch.Tensor, bits: int = 4, rot_group: int = 256, scale_group: int = 0,
+                      stream=None) -> None:
+    """rbd_rot_quant_act plus ld = X @ L1 (l1 bf16 [K, r], ld bf16 [M, r])."""
+    M, K = x.shape
+    r = l1.shape[1]
+    _ok(load().rbd_lowrank_fused(_ptr(x), M, K, _rowstride(x), _qcfg(bits, rot_group, scale_group),
+                                 _ptr(codes), _ptr(scales), _ptr(l1), r, _ptr(ld), _stream(stream)),
+        "rbd_lowrank_fused")
+
+
+def rbd_pack_weights_int4(w: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, rot_group: int = 256,
+                          scale_group: int = 0, stream=None) -> None:
+    """w bf16 [N, K] -> packed uint8 [N, K/2], scales float32 [N] or [N, K/64]."""
+    N, K = w.shape
+    _ok(load().rbd_pack_weights_int4(_ptr(w), N, K, _qcfg(4, rot_group, scale_group), _ptr(packed),
+                                     _ptr(scales), _stream(stream)), "rbd_pack_weights_int4")
+
+
+def rbd_pack_weights_int8(w: torch.Tensor, w8: torch.Tensor, scales: torch.Tensor, rot_group: int = 256,
+                          scale_group: int = 0, stream=None) -> None:
+    """w bf16 [N, K] -> w8 int8 [N, K], scales float32 [N] or [N, K/64]."""
+    N, K = w.shape
+    _ok(load().rbd_pack_weights_int8(_ptr(w), N, K, _qcfg(8, rot_group, scale_group), _ptr(w8),
+                                     _ptr(scales), _stream(stream)), "rbd_pack_weights_int8")
+
+
+def make_epilogue(bias=None, ld=None, l2t=None, gate_mode: int = 0, gate_cols=(0, 0), gate=None,
+                  residual=None, acc_debug=None) -> Epilogue:
+    e = Epilogue()
+    e.bias = _ptr(bias)
+    e.ld = _ptr(ld)
+    e.l2t = _ptr(l2t)
+    e.r = 0 if ld is None else int(ld.shape[1])
+    e.gate_mode = gate_mode
+    e.gate_col0, e.gate_col1 = int(gate_cols[0]), int(gate_cols[1])
+    e.gate = _ptr(gate)
+    e.residual = _ptr(residual)
+    e.ldr = 0 if residual is None else _rowstride(residual)
+    e.acc_debug = _ptr(acc_debug)
+    return e
+
+
+def _linear(fn, where, codes, sx, w, sw, y, bits, rot_group, scale_group, epi, stream):
+    M, K = codes.shape
+    N = y.shape[1]
+    e = epi if epi is not None else Epilogue()
+    _ok(fn(_ptr(codes), _ptr(sx), _ptr(w), _ptr(sw), M, N, K, _qcfg(bits, rot_group, scale_group),
+           ctypes.byref(e), _ptr(y), _rowstride(y), _stream(stream)), where)
+
+
+def rbd_w4a4_linear(codes: torch.Tensor, sx: torch.Tensor, w_packed: torch.Tensor, sw: torch.Tensor,
+                    y: torch.Tensor, scale_group: int = 0, epi: Optional[Epilogue] = None,
+                    rot_group: int = 256, stream=None) -> None:
+    """y bf16 [M, N] = epilogue(dequant(codes @ unpack(w_packed)^T))."""
+    _linear(load().rbd_w4a4_linear, "rbd_w4a4_linear", codes, sx, w_packed, sw, y, 4, rot_group,
+            scale_group, epi, stream)
+
+
+def rbd_w8a8_linear(codes: torch.Tensor, sx: torch.Tensor, w8: torch.Tensor, sw: torch.Tensor,
+                    y: torch.Tensor, scale_group: int = 0, epi: Optional[Epilogue] = None,
+                    rot_group: int = 256, stream=None) -> None:
+    """y bf16 [M, N] = epilogue(dequant(codes @ w8^T))."""
+    _linear(load().rbd_w8a8_linear, "rbd_w8a8_linear", codes, sx, w8, sw, y, 8, rot_group,
+            scale_group, epi, stream)
+
+
+def rbd_check(stream=None) -> int:
+    """Synchronise the stream and return the device status (0 = fine)."""
+    return load().rbd_check(_stream(stream))
+
+
+def rbd_debug_timeout_probe(timeout_ns: int, stream=None) -> None:
+    _ok(load().rbd_debug_timeout_probe(int(timeout_ns), _stream(stream)), "rbd_debug_timeout_probe")
+
+
+def rbd_status_string(status: int) -> str:
+    return load().rbd_status_string(status).decode()
+
+
+def rbd_version() -> str:
+    return load().rbd_version().decode()

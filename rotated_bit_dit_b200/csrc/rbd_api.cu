@@ -1,0 +1,257 @@
+// C ABI of the rotated low-bit linear library: argument validation, tensor-map
+// construction, launches, and the device status word.  Every entry point
+// validates before launching and never falls back to another implementation.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "rbd_common.cuh"
+
+#include "rbd_internal.cuh"
+
+namespace {
+
+using rbd::GemmArgs;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+rbd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RBD_OK : RBD_ERR_CUDA; }
+
+rbd_status check_qcfg(const rbd_qcfg& c, int64_t K) {
+  if (c.bits != 4 && c.bits != 8) return RBD_ERR_INVALID_ARG;
+  if (c.rot_group != 0 && c.rot_group != 256) return RBD_ERR_UNSUPPORTED;
+  if (c.scale_group != 0 && c.scale_group != 64) return RBD_ERR_UNSUPPORTED;
+  if (K <= 0 || K % 256 != 0 || K > 16384) return RBD_ERR_UNSUPPORTED;
+  return RBD_OK;
+}
+
+// --- driver entry point for tensor-map encoding (no link against libcuda)
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Row-major 2D tensor [rows, cols] with row stride `row_bytes`; box = [box_rows, box_cols].
+bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint32_t elem_bytes, uint64_t cols,
+                 uint64_t rows, uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint32_t inner_bytes = box_cols * elem_bytes;
+  CUtensorMapSwizzle sw;
+  switch (inner_bytes) {
+    case 128: sw = CU_TENSOR_MAP_SWIZZLE_128B; break;
+    case 64: sw = CU_TENSOR_MAP_SWIZZLE_64B; break;
+    case 32: sw = CU_TENSOR_MAP_SWIZZLE_32B; break;
+    default: return false;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms_current() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static std::mutex mu;
+  static int cache[64] = {0};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 64 && cache[dev]) return cache[dev];
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
+rbd_status quant_common(const void* x, int64_t M, int64_t K, int64_t ld, rbd_qcfg cfg, void* out, float* scales,
+                        bool packed, void* stream) {
+  if (M < 0) return RBD_ERR_INVALID_ARG;
+  rbd_status s = check_qcfg(cfg, K);
+  if (s != RBD_OK) return s;
+  if (M == 0) return RBD_OK;
+  if (!x || !out || !scales) return RBD_ERR_INVALID_ARG;
+  if (ld < K) return RBD_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out) || (ld % 8) != 0) return RBD_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(scales) & 3u) return RBD_ERR_ALIGNMENT;
+  return cuda_status(rbd::launch_rot_quant(static_cast<const uint16_t*>(x), M, K, ld, cfg.bits, cfg.rot_group != 0,
+                                           cfg.scale_group == 64, packed, static_cast<int8_t*>(out), scales,
+                                           as_stream(stream)));
+}
+
+template <bool W4>
+rbd_status linear_common(const int8_t* codes, const float* sx, const void* w, const float* sw, int64_t M,
+                         int64_t N, int64_t K, rbd_qcfg cfg, const rbd_epilogue* epi, void* y, int64_t ldy,
+                         void* stream) {
+  if (cfg.bits != (W4 ? 4 : 8)) return RBD_ERR_INVALID_ARG;
+  if (cfg.scale_group != 0 && cfg.scale_group != 64) return RBD_ERR_UNSUPPORTED;
+  if (M < 0 || N <= 0 || K <= 0) return RBD_ERR_INVALID_ARG;
+  if (K % 128 != 0 || N % 128 != 0) return RBD_ERR_UNSUPPORTED;
+  if (M > (int64_t)INT32_MAX / 2 || N > (1 << 24) || K > (1 << 20)) return RBD_ERR_UNSUPPORTED;
+  if (M == 0) return RBD_OK;
+  if (!codes || !sx || !w || !sw || !y) return RBD_ERR_INVALID_ARG;
+  if (ldy < N) return RBD_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(w) || !aligned16(y) || (ldy % 8) != 0) return RBD_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(sx) & 3u) || (reinterpret_cast<uintptr_t>(sw) & 3u)) return RBD_ERR_ALIGNMENT;
+  const int G = cfg.scale_group ? static_cast<int>(K / 64) : 1;
+  if (G > 256) return RBD_ERR_UNSUPPORTED;
+
+  rbd_epilogue e{};
+  if (epi) e = *epi;
+  if (e.r != 0 && e.r != 16 && e.r != 32 && e.r != 64) return RBD_ERR_UNSUPPORTED;
+  if (e.r && (!e.ld || !e.l2t)) return RBD_ERR_INVALID_ARG;
+  if (e.r && (!aligned16(e.ld) || !aligned16(e.l2t))) return RBD_ERR_ALIGNMENT;
+  if (e.gate_mode < 0 || e.gate_mode > 2) return RBD_ERR_INVALID_ARG;
+  if (e.gate_mode == 1 && (e.gate_col0 < 0 || e.gate_col1 < e.gate_col0 || e.gate_col1 > N))
+    return RBD_ERR_INVALID_ARG;
+  if (e.gate_mode == 2) {
+    if (!e.gate || !e.residual) return RBD_ERR_INVALID_ARG;
+    if (e.ldr < N) return RBD_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(e.residual) & 1u) || (reinterpret_cast<uintptr_t>(e.gate) & 1u))
+      return RBD_ERR_ALIGNMENT;
+  }
+  if (e.bias && (reinterpret_cast<uintptr_t>(e.bias) & 1u)) return RBD_ERR_ALIGNMENT;
+  if (e.acc_debug && (reinterpret_cast<uintptr_t>(e.acc_debug) & 3u)) return RBD_ERR_ALIGNMENT;
+
+  CUtensorMap tm_x{}, tm_w{}, tm_ld{}, tm_l2{};
+  if (!make_map_2d(&tm_x, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, K, 128, 128)) return RBD_ERR_CUDA;
+  if (!W4 && !make_map_2d(&tm_w, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, K, 128, 128)) return RBD_ERR_CUDA;
+  if (e.r) {
+    if (!make_map_2d(&tm_ld, e.ld, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, e.r, M, 2 * e.r, e.r, 128))
+      return RBD_ERR_CUDA;
+    if (!make_map_2d(&tm_l2, e.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, e.r, N, 2 * e.r, e.r, 128))
+      return RBD_ERR_CUDA;
+  }
+  GemmArgs a{};
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.seg = cfg.scale_group ? 64 : static_cast<int>(K);
+  a.G = G;
+  a.sx = sx;
+  a.sw = sw;
+  a.w4 = W4 ? static_cast<const uint8_t*>(w) : nullptr;
+  a.bias = static_cast<const uint16_t*>(e.bias);
+  a.r = e.r;
+  a.gate_mode = e.gate_mode;
+  a.gate_c0 = static_cast<int>(e.gate_col0);
+  a.gate_c1 = static_cast<int>(e.gate_col1);
+  a.gate = static_cast<const uint16_t*>(e.gate);
+  a.residual = static_cast<const uint16_t*>(e.residual);
+  a.ldr = e.ldr;
+  a.y = static_cast<uint16_t*>(y);
+  a.ldy = ldy;
+  a.acc_debug = e.acc_debug;
+  a.acc_scale = W4 ? 1.0f / 16.0f : 1.0f;
+  a.num_m_tiles = static_cast<int>((M + 127) / 128);
+  a.num_tiles = a.num_m_tiles * static_cast<int>(N / 128);
+  const int sms = num_sms_current();
+  if (sms <= 0) return RBD_ERR_CUDA;
+  return cuda_status(rbd::launch_lowbit_gemm(W4, cfg.scale_group == 64, tm_x, tm_w, tm_ld, tm_l2, a, sms,
+                                             as_stream(stream)));
+}
+
+__global__ void timeout_probe_kernel(int64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    rbd::mbar_init(&bar, 1);
+    rbd::fence_barrier_init();
+    // Nothing ever arrives on `bar`: the bounded wait must expire and record a timeout.
+    rbd::mbar_wait(&bar, 0, static_cast<uint64_t>(timeout_ns));
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+rbd_status rbd_rot_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, rbd_qcfg cfg, int8_t* codes,
+                             float* scales, void* stream) {
+  return quant_common(x, M, K, ldx, cfg, codes, scales, false, stream);
+}
+
+rbd_status rbd_lowrank_fused(const void* x, int64_t M, int64_t K, int64_t ldx, rbd_qcfg cfg, int8_t* codes,
+                             float* scales, const void* l1, int32_t r, void* ld, void* stream) {
+  if (r != 16 && r != 32 && r != 64) return RBD_ERR_UNSUPPORTED;
+  if (M > 0 && (!l1 || !ld)) return RBD_ERR_INVALID_ARG;
+  if (M > 0 && (!aligned16(l1) || !aligned16(ld))) return RBD_ERR_ALIGNMENT;
+  rbd_status s = quant_common(x, M, K, ldx, cfg, codes, scales, false, stream);
+  if (s != RBD_OK || M == 0) return s;
+  return cuda_status(rbd::launch_lowrank_down(static_cast<const uint16_t*>(x), M, K, ldx,
+                                              static_cast<const uint16_t*>(l1), r, static_cast<uint16_t*>(ld),
+                                              as_stream(stream)));
+}
+
+rbd_status rbd_pack_weights_int4(const void* w, int64_t N, int64_t K, rbd_qcfg cfg, uint8_t* packed, float* scales,
+                                 void* stream) {
+  if (cfg.bits != 4) return RBD_ERR_INVALID_ARG;
+  return quant_common(w, N, K, K, cfg, packed, scales, true, stream);
+}
+
+rbd_status rbd_pack_weights_int8(const void* w, int64_t N, int64_t K, rbd_qcfg cfg, int8_t* w8, float* scales,
+                                 void* stream) {
+  if (cfg.bits != 8) return RBD_ERR_INVALID_ARG;
+  return quant_common(w, N, K, K, cfg, w8, scales, false, stream);
+}
+
+rbd_status rbd_w4a4_linear(const int8_t* codes, const float* sx, const uint8_t* w_packed, const float* sw,
+                           int64_t M, int64_t N, int64_t K, rbd_qcfg cfg, const rbd_epilogue* epi, void* y,
+                           int64_t ldy, void* stream) {
+  return linear_common<true>(codes, sx, w_packed, sw, M, N, K, cfg, epi, y, ldy, stream);
+}
+
+rbd_status rbd_w8a8_linear(const int8_t* codes, const float* sx, const int8_t* w8, const float* sw, int64_t M,
+                           int64_t N, int64_t K, rbd_qcfg cfg, const rbd_epilogue* epi, void* y, int64_t ldy,
+                           void* stream) {
+  return linear_common<false>(codes, sx, w8, sw, M, N, K, cfg, epi, y, ldy, stream);
+}
+
+rbd_status rbd_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return RBD_ERR_CUDA;
+  int st = 0;
+  e = cudaMemcpyFromSymbol(&st, rbd::g_device_status, sizeof(int));
+  if (e != cudaSuccess) return RBD_ERR_CUDA;
+  if (st != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(rbd::g_device_status, &zero, sizeof(int)) != cudaSuccess) return RBD_ERR_CUDA;
+    return static_cast<rbd_status>(st);
+  }
+  return RBD_OK;
+}
+
+rbd_status rbd_debug_timeout_probe(int64_t timeout_ns, void* stream) {
+  if (timeout_ns <= 0 || timeout_ns > 10000000000ll) return RBD_ERR_INVALID_ARG;
+  timeout_probe_kernel<<<1, 32, 0, as_stream(stream)>>>(timeout_ns);
+  return cuda_status(cudaGetLastError());
+}
+
+const char* rbd_status_string(rbd_status s) {
+  switch (s) {
+    case RBD_OK: return "RBD_OK";
+    case RBD_ERR_INVALID_ARG: return "RBD_ERR_INVALID_ARG";
+    case RBD_ERR_UNSUPPORTED: return "RBD_ERR_UNSUPPORTED";
+    case RBD_ERR_ALIGNMENT: return "RBD_ERR_ALIGNMENT";
+    case RBD_ERR_CUDA: return "RBD_ERR_CUDA";
+    case RBD_ERR_DEVICE_TIMEOUT: return "RBD_ERR_DEVICE_TIMEOUT";
+  }
+  return "RBD_ERR_UNKNOWN";
+}
+
+const char* rbd_version(void) { return "rotated_bit_dit_b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

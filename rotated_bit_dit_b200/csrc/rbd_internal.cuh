@@ -1,0 +1,40 @@
+// Host-side interfaces between the C ABI layer and the kernel launchers.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace rbd {
+
+// Arguments of the low-bit GEMM kernel (one launch = one linear call).
+struct GemmArgs {
+  int M, N, K;
+  int seg;              // accumulation segment length along K (64, or K for row scales)
+  int G;                // segments per tile = K / seg
+  const float* sx;      // activation scales [M] or [M, K/64]
+  const float* sw;      // weight scales [N] or [N, K/64]
+  const uint8_t* w4;    // packed INT4 weights [N, K/2] (W4A4 only)
+  const uint16_t* bias; // bf16 [N] or null
+  int r;                // low-rank rank, 0 = no branch
+  int gate_mode;        // 0 none, 1 sigmoid on [gate_c0, gate_c1), 2 gated residual
+  int gate_c0, gate_c1;
+  const uint16_t* gate;      // bf16 [N]
+  const uint16_t* residual;  // bf16 [M, ldr]
+  int64_t ldr;
+  uint16_t* y;          // bf16 [M, ldy]
+  int64_t ldy;
+  int32_t* acc_debug;   // optional exact accumulators
+  float acc_scale;      // 1/16 for widened INT4 weights, 1 for INT8
+  int num_m_tiles, num_tiles;
+};
+
+cudaError_t launch_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot, bool g64,
+                             bool packed, int8_t* codes, float* scales, cudaStream_t st);
+cudaError_t launch_lowrank_down(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const uint16_t* l1, int r,
+                                uint16_t* ld, cudaStream_t st);
+cudaError_t launch_lowbit_gemm(bool w4, bool g64, const CUtensorMap& tm_x, const CUtensorMap& tm_w8,
+                               const CUtensorMap& tm_ld, const CUtensorMap& tm_l2, const GemmArgs& a, int num_sms,
+                               cudaStream_t st);
+
+}  // namespace rbd

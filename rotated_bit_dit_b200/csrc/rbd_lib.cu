@@ -1,0 +1,6 @@
+// Single translation unit of librbd.so: the device status word defined in
+// rbd_api.cu is referenced by kernels of the other files, so they are compiled
+// together (no relocatable device code needed).
+#include "rbd_api.cu"
+#include "rbd_prologue.cu"
+#include "rbd_gemm.cu"

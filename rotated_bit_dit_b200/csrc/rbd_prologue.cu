@@ -1,0 +1,400 @@
+// Activation / weight prologue kernels: group-wise regular-Hadamard rotation,
+// dynamic symmetric quantisation, INT4 packing, and the low-rank down product.
+//
+// Method: "Krea-2 Turbo -- INT4 tensorwise W4A4 (+ConvRot, mixed int8
+// fallback)", header paragraph (group-256 regular-Hadamard rotation of the
+// activations online, dynamic quantisation inside the kernel, packed signed
+// INT4 weights); group-64 scales per "Krea 2 Turbo Nunchaku Lite INT4 r32".
+//
+// Rotation arithmetic.  H = (J4 - 2 I4)^{(x)4} factors into four radix-4
+// stages, one per base-4 digit of the index inside the 256-block:
+// y_i = S - 2 x_i with S the sum of the four values that differ only in that
+// digit.  The stages run in float64 on values pre-scaled by 1/16 (exact).
+// Every partial sum of +-x/16 over bf16 inputs whose leading-bit exponents
+// span at most 37 binades needs at most 53 significant bits, so each stage is
+// exact and the float64 result is the exact rotated value; one
+// __double2float_rn then gives the correctly rounded float32.
+//
+// Thread layout.  16 threads ("a team") own one 256-block: thread tau holds
+// the 16 contiguous elements 16*tau .. 16*tau+15 (digits j0, j1 in registers,
+// j2 j3 = tau), transforms digits j0 and j1, swaps through shared memory so
+// that it holds positions tau + 16*i (digits j2, j3 in registers), transforms
+// those, and quantises.  Codes go back through shared memory so each thread
+// stores 16 contiguous bytes.
+#include "rbd_common.cuh"
+#include "rbd_internal.cuh"
+
+namespace rbd {
+
+namespace {
+
+constexpr int kTeam = 16;  // threads per 256-block
+
+__device__ __forceinline__ void radix4_regular(double& a, double& b, double& c, double& d) {
+  const double s = (a + b) + (c + d);
+  a = fma(-2.0, a, s);
+  b = fma(-2.0, b, s);
+  c = fma(-2.0, c, s);
+  d = fma(-2.0, d, s);
+}
+
+// 16 bf16 (two 16-byte vectors) -> 16 doubles scaled by 1/16.
+__device__ __forceinline__ void load16_scaled(const uint4& lo, const uint4& hi, double (&v)[16]) {
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float f0 = __uint_as_float(w[i] << 16);
+    const float f1 = __uint_as_float(w[i] & 0xFFFF0000u);
+    v[2 * i] = static_cast<double>(f0) * 0.0625;
+    v[2 * i + 1] = static_cast<double>(f1) * 0.0625;
+  }
+}
+
+__device__ __forceinline__ void load16_f32(const uint4& lo, const uint4& hi, float (&v)[16]) {
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// Swizzled index into a team's 256-double exchange buffer: conflict-free both
+// for "thread tau writes 16*tau + e" and "thread tau reads tau + 16*i".
+__device__ __forceinline__ int xchg_idx(int p) { return p ^ ((p >> 4) & 15); }
+
+struct QuantParams {
+  float qmax;
+};
+
+__device__ __forceinline__ int quant1(float v, float inv, float qmax) {
+  const float t = __fmul_rn(v, inv);
+  int q = __float2int_rn(t);
+  const int hi = static_cast<int>(qmax);
+  q = q > hi ? hi : q;
+  q = q < -hi - 1 ? -hi - 1 : q;
+  return q;
+}
+
+}  // namespace
+
+// One CTA handles `rows` rows; each row is handled by T = 16 * teams threads;
+// team `tm` of a row processes 256-blocks g = tm, tm + teams, ... (at most CMAX).
+// OUT_PACKED: write packed INT4 bytes instead of one code per byte.
+template <bool ROT, bool G64, bool OUT_PACKED, int CMAX>
+__global__ void __launch_bounds__(256) rot_quant_kernel(const uint16_t* __restrict__ x, int64_t M, int K,
+                                                        int64_t ldx, float qmax, int teams, int rows,
+                                                        int8_t* __restrict__ codes, float* __restrict__ scales) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* xbuf = reinterpret_cast<double*>(smem_raw);        // [teams*rows][256]
+  float* red = reinterpret_cast<float*>(smem_raw + (size_t)blockDim.x / kTeam * 256 * sizeof(double));
+
+  const int T = kTeam * teams;
+  const int tid = threadIdx.x;
+  const int rloc = tid / T;
+  const int t_in_row = tid % T;
+  const int team = t_in_row / kTeam;
+  const int tau = t_in_row % kTeam;
+  const int64_t m = (int64_t)blockIdx.x * rows + rloc;
+  const bool row_ok = (rloc < rows) && (m < M);
+  const int G = K >> 8;
+  double* tb = xbuf + (size_t)(tid / kTeam) * 256;
+
+  // ---- load all chunks of this thread (16 bf16 each)
+  uint4 raw[CMAX][2];
+#pragma unroll
+  for (int c = 0; c < CMAX; ++c) {
+    const int g = team + c * teams;
+    if (row_ok && g < G) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + m * ldx + (int64_t)g * 256 + tau * 16);
+      raw[c][0] = __ldg(src);
+      raw[c][1] = __ldg(src + 1);
+    } else {
+      raw[c][0] = make_uint4(0, 0, 0, 0);
+      raw[c][1] = make_uint4(0, 0, 0, 0);
+    }
+  }
+
+  // ---- rotate
+  float xr[CMAX][16];
+#pragma unroll
+  for (int c = 0; c < CMAX; ++c) {
+    if constexpr (ROT) {
+      double v[16];
+      load16_scaled(raw[c][0], raw[c][1], v);
+      // digit j0 (e & 3), then digit j1 (e >> 2)
+#pragma unroll
+      for (int j1 = 0; j1 < 4; ++j1) radix4_regular(v[4 * j1], v[4 * j1 + 1], v[4 * j1 + 2], v[4 * j1 + 3]);
+#pragma unroll
+      for (int j0 = 0; j0 < 4; ++j0) radix4_regular(v[j0], v[j0 + 4], v[j0 + 8], v[j0 + 12]);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) tb[xchg_idx(16 * tau + e)] = v[e];
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = tb[xchg_idx(tau + 16 * i)];
+      __syncwarp();
+      // now v[i] is position tau + 16*i: digit j2 = i & 3, j3 = i >> 2
+#pragma unroll
+      for (int j3 = 0; j3 < 4; ++j3) radix4_regular(v[4 * j3], v[4 * j3 + 1], v[4 * j3 + 2], v[4 * j3 + 3]);
+#pragma unroll
+      for (int j2 = 0; j2 < 4; ++j2) radix4_regular(v[j2], v[j2 + 4], v[j2 + 8], v[j2 + 12]);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xr[c][i] = __double2float_rn(v[i]);
+    } else {
+      load16_f32(raw[c][0], raw[c][1], xr[c]);
+    }
+  }
+
+  // ---- scales
+  // Position of register i of chunk c inside its 256-block:
+  //   ROT: tau + 16*i ; !ROT: 16*tau + i.
+  float inv_row = 0.f;
+  float inv_g[CMAX][4];
+  if constexpr (!G64) {
+    float amax = 0.f;
+#pragma unroll
+    for (int c = 0; c < CMAX; ++c)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(xr[c][i]));
+    if (T <= 32) {
+      for (int off = T / 2; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    } else {
+      for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      const int wpr = T / 32;
+      if ((tid & 31) == 0) red[tid / 32] = amax;
+      __syncthreads();
+      amax = 0.f;
+      for (int w = 0; w < wpr; ++w) amax = fmaxf(amax, red[rloc * wpr + w]);
+    }
+    inv_row = amax > 0.f ? __fdiv_rn(qmax, amax) : 0.f;
+    if (row_ok && t_in_row == 0) scales[m] = __fdiv_rn(amax, qmax);
+  } else {
+#pragma unroll
+    for (int c = 0; c < CMAX; ++c) {
+      const int g = team + c * teams;
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        float am = 0.f;
+        if constexpr (ROT) {
+#pragma unroll
+          for (int i = 4 * a; i < 4 * a + 4; ++i) am = fmaxf(am, fabsf(xr[c][i]));
+          for (int off = 8; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+        } else {
+          // 64-block a of this 256-block covers threads 4a .. 4a+3
+#pragma unroll
+          for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(xr[c][i]));
+          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+          am = __shfl_sync(0xffffffffu, am, (tid & ~15) + 4 * a);
+        }
+        inv_g[c][a] = am > 0.f ? __fdiv_rn(qmax, am) : 0.f;
+        if (row_ok && g < G && tau == a) scales[m * (K / 64) + g * 4 + a] = __fdiv_rn(am, qmax);
+      }
+    }
+  }
+
+  // ---- quantise and store
+#pragma unroll
+  for (int c = 0; c < CMAX; ++c) {
+    const int g = team + c * teams;
+    uint32_t packed_words[4];
+    if constexpr (ROT) {
+      unsigned char* cb = reinterpret_cast<unsigned char*>(tb);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float inv = G64 ? inv_g[c][i >> 2] : inv_row;
+        cb[tau + 16 * i] = static_cast<unsigned char>(static_cast<int8_t>(quant1(xr[c][i], inv, qmax)));
+      }
+      __syncwarp();
+      const uint4 q4 = *reinterpret_cast<const uint4*>(cb + 16 * tau);
+      __syncwarp();
+      packed_words[0] = q4.x; packed_words[1] = q4.y; packed_words[2] = q4.z; packed_words[3] = q4.w;
+    } else {
+#pragma unroll
+      for (int wv = 0; wv < 4; ++wv) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int i = 4 * wv + b;
+          const float inv = G64 ? inv_g[c][tau >> 2] : inv_row;
+          word |= (static_cast<uint32_t>(quant1(xr[c][i], inv, qmax)) & 0xFFu) << (8 * b);
+        }
+        packed_words[wv] = word;
+      }
+    }
+    if (row_ok && g < G) {
+      const int64_t k0 = (int64_t)g * 256 + tau * 16;
+      if constexpr (OUT_PACKED) {
+        // 16 codes -> 8 bytes, code k (even) in the low nibble, k+1 in the high nibble
+        uint32_t outw[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t acc = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t pair = (h * 2 + j / 2 < 4) ? packed_words[h * 2 + j / 2] : 0u;
+            const uint32_t lo = (pair >> (16 * (j & 1))) & 0xFu;
+            const uint32_t hi = (pair >> (16 * (j & 1) + 8)) & 0xFu;
+            acc |= (lo | (hi << 4)) << (8 * j);
+          }
+          outw[h] = acc;
+        }
+        uint8_t* dst = reinterpret_cast<uint8_t*>(codes) + m * (int64_t)(K / 2) + k0 / 2;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(outw[0], outw[1]);
+      } else {
+        *reinterpret_cast<uint4*>(codes + m * (int64_t)K + k0) =
+            make_uint4(packed_words[0], packed_words[1], packed_words[2], packed_words[3]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Low-rank down product ld[M, r] = X[M, K] @ L1[K, r] (unrotated bf16 input),
+// legacy bf16 mma.sync (m16n8k16), fp32 accumulation.  One CTA = 16 tokens,
+// 4 warps split K and reduce through shared memory.
+// ---------------------------------------------------------------------------
+template <int R>
+__global__ void __launch_bounds__(128) lowrank_down_kernel(const uint16_t* __restrict__ x, int64_t M, int K,
+                                                           int64_t ldx, const uint16_t* __restrict__ l1,
+                                                           uint16_t* __restrict__ ld) {
+  constexpr int NT = R / 8;
+  __shared__ float part[4][16][R + 1];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c4 = lane & 3;
+  const int64_t m0 = (int64_t)blockIdx.x * 16;
+  const int64_t ra = m0 + g, rb = m0 + g + 8;
+  const bool va = ra < M, vb = rb < M;
+  float acc[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  const int kper = K / 4;
+  const int kbeg = warp * kper, kend = kbeg + kper;
+  for (int k = kbeg; k < kend; k += 16) {
+    uint32_t a[4];
+    const uint32_t* xa = reinterpret_cast<const uint32_t*>(x + ra * ldx + k);
+    const uint32_t* xb = reinterpret_cast<const uint32_t*>(x + rb * ldx + k);
+    a[0] = va ? __ldg(xa + c4) : 0u;
+    a[1] = vb ? __ldg(xb + c4) : 0u;
+    a[2] = va ? __ldg(xa + c4 + 4) : 0u;
+    a[3] = vb ? __ldg(xb + c4 + 4) : 0u;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int col = n * 8 + g;
+      const uint32_t b0 = (uint32_t)__ldg(l1 + (int64_t)(k + 2 * c4) * R + col) |
+                          ((uint32_t)__ldg(l1 + (int64_t)(k + 2 * c4 + 1) * R + col) << 16);
+      const uint32_t b1 = (uint32_t)__ldg(l1 + (int64_t)(k + 2 * c4 + 8) * R + col) |
+                          ((uint32_t)__ldg(l1 + (int64_t)(k + 2 * c4 + 9) * R + col) << 16);
+      asm volatile(
+          "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+          "{%0,%1,%2,%3};"
+          : "+f"(acc[n][0]), "+f"(acc[n][1]), "+f"(acc[n][2]), "+f"(acc[n][3])
+          : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    part[warp][g][n * 8 + 2 * c4] = acc[n][0];
+    part[warp][g][n * 8 + 2 * c4 + 1] = acc[n][1];
+    part[warp][g + 8][n * 8 + 2 * c4] = acc[n][2];
+    part[warp][g + 8][n * 8 + 2 * c4 + 1] = acc[n][3];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 16 * R; i += blockDim.x) {
+    const int rr = i / R, cc = i % R;
+    const int64_t mm = m0 + rr;
+    if (mm < M) {
+      const float s = (part[0][rr][cc] + part[1][rr][cc]) + (part[2][rr][cc] + part[3][rr][cc]);
+      ld[mm * R + cc] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------
+namespace {
+struct Geometry {
+  int teams, cmax, T, rows, threads;
+  size_t smem;
+};
+
+Geometry geometry(int64_t K) {
+  Geometry gm{};
+  const int G = static_cast<int>(K / 256);
+  int teams = G < 16 ? G : 16;
+  if (teams > 1 && (teams & 1)) teams += 1;   // keep T a multiple of 32 when above 16
+  gm.teams = teams;
+  gm.cmax = (G + teams - 1) / teams;
+  gm.T = kTeam * teams;
+  gm.rows = gm.T >= 256 ? 1 : 256 / gm.T;
+  gm.threads = gm.T * gm.rows;
+  gm.smem = (size_t)(gm.threads / kTeam) * 256 * sizeof(double) + 64 * sizeof(float);
+  return gm;
+}
+
+template <bool ROT, bool G64, bool PK>
+cudaError_t launch_rq_c(int cmax, dim3 grid, int threads, size_t smem, cudaStream_t st, const uint16_t* x,
+                        int64_t M, int K, int64_t ldx, float qmax, int teams, int rows, int8_t* codes,
+                        float* scales) {
+  switch (cmax) {
+#define RBD_RQ_CASE(C)                                                                                    \
+  case C: {                                                                                               \
+    auto kern = rot_quant_kernel<ROT, G64, PK, C>;                                                        \
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    if (e != cudaSuccess) return e;                                                                       \
+    kern<<<grid, threads, smem, st>>>(x, M, K, ldx, qmax, teams, rows, codes, scales);                   \
+    return cudaGetLastError();                                                                            \
+  }
+    RBD_RQ_CASE(1)
+    RBD_RQ_CASE(2)
+    RBD_RQ_CASE(3)
+    RBD_RQ_CASE(4)
+#undef RBD_RQ_CASE
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+}  // namespace
+
+cudaError_t launch_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot, bool g64,
+                             bool packed, int8_t* codes, float* scales, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  const Geometry gm = geometry(K);
+  const float qmax = bits == 4 ? 7.f : 127.f;
+  const dim3 grid(static_cast<unsigned>((M + gm.rows - 1) / gm.rows));
+  const int Ki = static_cast<int>(K);
+#define RBD_RQ_DISPATCH(R_, G_, P_)                                                                      \
+  return launch_rq_c<R_, G_, P_>(gm.cmax, grid, gm.threads, gm.smem, st, x, M, Ki, ldx, qmax, gm.teams, \
+                                 gm.rows, codes, scales)
+  if (rot) {
+    if (g64) {
+      if (packed) RBD_RQ_DISPATCH(true, true, true); else RBD_RQ_DISPATCH(true, true, false);
+    } else {
+      if (packed) RBD_RQ_DISPATCH(true, false, true); else RBD_RQ_DISPATCH(true, false, false);
+    }
+  } else {
+    if (g64) {
+      if (packed) RBD_RQ_DISPATCH(false, true, true); else RBD_RQ_DISPATCH(false, true, false);
+    } else {
+      if (packed) RBD_RQ_DISPATCH(false, false, true); else RBD_RQ_DISPATCH(false, false, false);
+    }
+  }
+#undef RBD_RQ_DISPATCH
+}
+
+cudaError_t launch_lowrank_down(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const uint16_t* l1, int r,
+                                uint16_t* ld, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  const dim3 grid(static_cast<unsigned>((M + 15) / 16));
+  const int Ki = static_cast<int>(K);
+  switch (r) {
+    case 16: lowrank_down_kernel<16><<<grid, 128, 0, st>>>(x, M, Ki, ldx, l1, ld); break;
+    case 32: lowrank_down_kernel<32><<<grid, 128, 0, st>>>(x, M, Ki, ldx, l1, ld); break;
+    case 64: lowrank_down_kernel<64><<<grid, 128, 0, st>>>(x, M, Ki, ldx, l1, ld); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace rbd

@@ -1,0 +1,106 @@
+"""The C-ABI library on the CPU: it loads, exports every declared entry point,
+and rejects invalid calls before launching anything (no GPU needed: the
+validation paths return before the first CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import rotated_bit_dit_b200 as R
+from rotated_bit_dit_b200 import _binding as B
+
+HDR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "rbd.h")
+
+
+def declared_entry_points():
+    text = open(HDR).read()
+    return re.findall(r"^(?:rbd_status|const char\*)\s+(rbd_\w+)\(", text, re.M)
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = R.load()
+    names = declared_entry_points()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(B.EXPORTED)
+    assert R.rbd_version().startswith("rotated_bit_dit_b200")
+
+
+def test_status_strings():
+    for code, name in B.STATUS_NAMES.items():
+        assert R.rbd_status_string(code) == name
+    assert R.rbd_status_string(99) == "RBD_ERR_UNKNOWN"
+
+
+FAKE = ctypes.c_void_p(0x10000)          # 16-byte aligned, never dereferenced
+FAKE_MIS = ctypes.c_void_p(0x10001)      # misaligned
+
+
+def q(bits=4, rot=256, sg=0):
+    return B.QCfg(bits, rot, sg)
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((FAKE, 4, 100, 100, q(), FAKE, FAKE, None), 2),            # K not a multiple of 256
+    ((FAKE, 4, 256, 256, q(bits=5), FAKE, FAKE, None), 1),      # bad bits
+    ((FAKE, 4, 256, 256, q(rot=128), FAKE, FAKE, None), 2),     # unsupported rotation group
+    ((FAKE, 4, 256, 256, q(sg=32), FAKE, FAKE, None), 2),       # unsupported scale group
+    ((FAKE, -1, 256, 256, q(), FAKE, FAKE, None), 1),           # negative M
+    ((None, 4, 256, 256, q(), FAKE, FAKE, None), 1),            # null input
+    ((FAKE, 4, 256, 128, q(), FAKE, FAKE, None), 1),            # ldx < K
+    ((FAKE_MIS, 4, 256, 256, q(), FAKE, FAKE, None), 3),        # misaligned x
+    ((FAKE, 4, 256, 260, q(), FAKE, FAKE, None), 3),            # row stride not 16-byte aligned
+    ((FAKE, 4, 32768, 32768, q(), FAKE, FAKE, None), 2),        # K above the supported maximum
+])
+def test_rot_quant_rejects_before_launch(args, expect):
+    assert R.load().rbd_rot_quant_act(*args) == expect
+
+
+def test_zero_rows_is_a_noop_without_pointers():
+    assert R.load().rbd_rot_quant_act(None, 0, 256, 256, q(), None, None, None) == 0
+
+
+def _lin(lib_fn, M=128, N=128, K=256, cfg=None, epi=None, codes=FAKE, w=FAKE, y=FAKE, ldy=None):
+    cfg = cfg or q()
+    e = epi if epi is not None else B.Epilogue()
+    return lib_fn(codes, FAKE, w, FAKE, M, N, K, cfg, ctypes.byref(e), y, N if ldy is None else ldy, None)
+
+
+def test_linear_rejects_before_launch():
+    lib = R.load()
+    w4, w8 = lib.rbd_w4a4_linear, lib.rbd_w8a8_linear
+    assert _lin(w4, cfg=q(bits=8)) == 1                      # W4A4 with 8-bit config
+    assert _lin(w8, cfg=q(bits=4)) == 1
+    assert _lin(w4, K=192) == 2                              # K % 128
+    assert _lin(w4, N=96) == 2                               # N % 128
+    assert _lin(w4, codes=FAKE_MIS) == 3
+    assert _lin(w4, y=FAKE_MIS) == 3
+    assert _lin(w4, ldy=64) == 1                             # ldy < N
+    e = B.Epilogue()
+    e.r = 24
+    assert _lin(w4, epi=e) == 2                              # unsupported rank
+    e = B.Epilogue()
+    e.r = 32
+    assert _lin(w4, epi=e) == 1                              # rank without factors
+    e = B.Epilogue()
+    e.gate_mode = 2
+    assert _lin(w4, epi=e) == 1                              # gated residual without tensors
+    e = B.Epilogue()
+    e.gate_mode = 1
+    e.gate_col0, e.gate_col1 = 64, 512
+    assert _lin(w4, epi=e) == 1                              # gate columns out of range
+    e = B.Epilogue()
+    e.gate_mode = 3
+    assert _lin(w4, epi=e) == 1
+    assert _lin(w4, M=0) == 0                                # empty batch: nothing to do
+
+
+def test_lowrank_and_pack_reject_before_launch():
+    lib = R.load()
+    assert lib.rbd_lowrank_fused(FAKE, 4, 256, 256, q(), FAKE, FAKE, FAKE, 24, FAKE, None) == 2
+    assert lib.rbd_lowrank_fused(FAKE, 4, 256, 256, q(), FAKE, FAKE, None, 32, FAKE, None) == 1
+    assert lib.rbd_pack_weights_int4(FAKE, 4, 256, q(bits=8), FAKE, FAKE, None) == 1
+    assert lib.rbd_pack_weights_int8(FAKE, 4, 256, q(bits=4), FAKE, FAKE, None) == 1
+    assert lib.rbd_debug_timeout_probe(0, None) == 1
