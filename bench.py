@@ -1,0 +1,333 @@
+"""Benchmark of the rotated low-bit linear layer on B200.
+
+One step = one full layer call on one batch of synthetic tokens: the
+rotate + quantise prologue with the low-rank down product, then the tcgen05
+W4A4 GEMM with group-64 dequant, rank-32 branch and sigmoid gate epilogue
+(the grouped Q|K|V|gate projection, M=4096 tokens, K=3072, N=4*3072).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own replica on its own batch (tokens are
+independent; no collective on the data path), scaling is weak and the value
+is the whole-job throughput over the slowest rank.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "w4a4_qkvg"
+METRIC = "W4A4 rotated linear TOPS & tokens/s at M=4096, % of B200 INT8 tensor peak"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def workload_desc(cfg):
+    return (f"{WORKLOAD}: grouped Q|K|V|gate W4A4 projection, M={cfg['M']} tokens, K={cfg['K']}, "
+            f"N={cfg['N']}, group-64 scales, rank-{cfg['rank']} bf16 low-rank branch, sigmoid on columns "
+            f"[{cfg['gate_cols'][0]},{cfg['gate_cols'][1]})")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+def oracle_sample(t, cfg, wq_qw_sw, rows):
+    """The oracle's per-token path on `rows` (weights already quantised, as on the GPU side)."""
+    from oracle import rbd_oracle as O
+    qw, sw = wq_qw_sw
+    x = t["x"][rows]
+    qx, sx = O.rot_quant(x, 4, 256, 64)
+    y = O.dequant(qx, sx, qw, sw, 64)
+    ld = O.lowrank_down(x, t["l1"])
+    return O.epilogue(y, None, ld, t["l2"], 1, cfg["gate_cols"])
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(t, cfg, rows_n=1024):
+    from oracle import rbd_oracle as O
+    wq, sw = O.quantize_weights(t["w"], 4, 256, 64)
+    prep = (O.unpack_int4(wq), sw)
+    rows = np.arange(rows_n)
+    oracle_sample(t, cfg, prep, rows[:8])                       # warm
+    t0 = time.perf_counter()
+    oracle_sample(t, cfg, prep, rows)
+    dt = time.perf_counter() - t0
+    tops = 2.0 * rows_n * cfg["N"] * cfg["K"] / dt / 1e12
+    return {"value": tops, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows_n} of {cfg['M']} token rows of the same layer (per-token path: rotate, quantise, "
+                      f"group-64 dequant GEMM, low-rank branch, sigmoid; weights quantised beforehand), "
+                      f"{dt:.2f} s", "tokens_per_s": rows_n / dt, "seconds": dt}
+
+
+def run_reference(args, cfg, t):
+    """--impl reference: the CPU oracle, as it stands, on bounded samples of the workload."""
+    from oracle import rbd_oracle as O
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wq, sw = O.quantize_weights(t["w"], 4, 256, 64)
+    prep = (O.unpack_int4(wq), sw)
+    rows_n = 256
+    rows = np.arange(rows_n)
+    for _ in range(args.warmup):
+        oracle_sample(t, cfg, prep, rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample(t, cfg, prep, rows)
+    dt = (time.perf_counter() - t0) / args.steps
+    tops = 2.0 * rows_n * cfg["N"] * cfg["K"] / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "sample_rows_per_step": rows_n},
+            "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{rows_n} token rows per step of the {cfg['M']}-token layer"},
+            "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "tokens_per_s": rows_n / dt}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU leg
+def run_ours(args, cfg, t):
+    import torch
+    import torch.distributed as dist
+
+    import rotated_bit_dit_b200 as R
+    from rotated_bit_dit_b200 import _binding as B
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    R.load()
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    M, K, N, r = cfg["M"], cfg["K"], cfg["N"], cfg["rank"]
+    layer = R.RotatedLowBitLinear(up(t["w"]), bits=4, scale_group=64, l1=up(t["l1"]), l2=up(t["l2"]),
+                                  gate_mode=1, gate_cols=cfg["gate_cols"])
+    x = up(t["x"])
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    codes, sx, ld = layer.buffers(M, dev)
+    epi = B.make_epilogue(None, ld, layer.l2t, 1, cfg["gate_cols"])
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)   # > 126 MB L2
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        B.rbd_lowrank_fused(x, codes, sx, layer.l1t, ld, 4, 256, 64)
+        if ev:
+            ev[1].record()
+        B.rbd_w4a4_linear(codes, sx, layer.wq, layer.sw, out, 64, epi)
+        if ev:
+            ev[2].record()
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    assert R.rbd_check() == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    status = R.rbd_check()
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    pro = [e[0].elapsed_time(e[1]) for e in evs]
+    gemm = [e[1].elapsed_time(e[2]) for e in evs]
+    tot = [e[0].elapsed_time(e[2]) for e in evs]
+    t_rank = sum(tot) / 1e3           # seconds over K steps, this rank
+    if world > 1:
+        tt = torch.tensor([t_rank], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+    else:
+        t_max = t_rank
+    ops_step = 2.0 * M * N * K
+    value = world * args.steps * ops_step / t_max / 1e12
+    tokens_s = world * args.steps * M / t_max
+
+    # ---- end to end through the public layer call with host buffers
+    xh = torch.from_numpy(np.ascontiguousarray(t["x"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(x)
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for _ in range(2):
+        xd.copy_(xh, non_blocking=True)
+        layer(xd, out=out)
+        yh.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record()
+        xd.copy_(xh, non_blocking=True)
+        layer(xd, out=out)
+        yh.copy_(out, non_blocking=True)
+        e2e_ev[i][1].record()
+    torch.cuda.synchronize()
+    e2e_t = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / 1e3
+    if world > 1:
+        tt = torch.tensor([e2e_t], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_t = float(tt.item())
+    e2e_value = world * args.steps * ops_step / e2e_t / 1e12
+
+    if rank == 0:
+        peaks, src = load_peaks()
+        int8_peak = 2.0 * peaks["bf16_tflops"]
+        gemm_s = statistics.mean(gemm) / 1e3
+        pro_s = statistics.mean(pro) / 1e3
+        achieved = ops_step / gemm_s / 1e12
+        pro_bytes = M * K * 2 + M * K + M * (K // 64) * 4 + K * r * 2 + M * r * 2
+        traffic = _profile_traffic()
+        line = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "M": M, "K": K, "N": N, "rank": r, "scale_group": 64,
+                       "bits": 4, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed (256 MB write) before every timed step"},
+            "tokens_per_s": tokens_s,
+            "pct_int8_peak": 100.0 * value / world / int8_peak,
+            "kernels_ms": {"rot_quant+lowrank_down": statistics.mean(pro), "w4a4_gemm": statistics.mean(gemm)},
+            "roofline": {"bound": "tensor", "kernel": "lowbit_gemm_kernel<W4,G64,LR>", "achieved": achieved,
+                         "peak": int8_peak, "unit": "TOPS", "frac": achieved / int8_peak,
+                         "peak_source": f"{src} bf16 dense {peaks['bf16_tflops']} TFLOP/s x 2 (nominal "
+                                        f"INT8:BF16 ratio)", "traffic": traffic,
+                         "algorithmic": "2*M*N*K int ops per launch"},
+            "prologue_roofline": {"bound": "hbm", "achieved": pro_bytes / pro_s / 1e9, "peak": peaks["hbm_gbs"],
+                                  "unit": "GB/s", "frac": pro_bytes / pro_s / 1e9 / peaks["hbm_gbs"],
+                                  "algorithmic_bytes": pro_bytes},
+            "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": int(xh.numel() * 2),
+                    "d2h_bytes_per_step": int(yh.numel() * 2)},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(t, cfg)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _profile_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary, when present."""
+    p = os.path.join(ROOT, "profiles", "traffic_w4a4_qkvg.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f).get("dram_bytes_per_launch")
+    return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from rotated_bit_dit_b200 import inputs as I
+    cfg = I.CONFIGS[WORKLOAD]
+    t = I.make_layer_inputs(cfg, seed=0)
+    if args.impl == "reference":
+        run_reference(args, cfg, t)
+    else:
+        run_ours(args, cfg, t)
+
+
+if __name__ == "__main__":
+    main()

@@ -81,11 +81,13 @@ rbd_status rbd_rot_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, r
 
 /* rbd_rot_quant_act plus the first factor of the low-rank branch on the
  * UNROTATED input: ld = X L1 (Krea-2-SVDQuant-ComfyUI, "LoRA": the branch is a
- * parallel linear, (W + L2 L1) x = W x + L2 (L1 x)).
- *   l1      bf16 [K, r] row-major.     r in {16, 32, 64}.
- *   ld      bf16 [M, r] row-major (float32 accumulation, rounded once).       */
+ * parallel linear, (W + L1 L2)-style, W x + L2 (L1 x)).
+ *   l1t     bf16 [r, K] row-major: L1 stored output-major, which is the
+ *           nn.Linear weight layout of the down projection.  r in {16, 32, 64}.
+ *   ld      bf16 [M, r] row-major (float32 accumulation, rounded once).
+ * Enqueues two kernels (rotate/quantise, then the down product).             */
 rbd_status rbd_lowrank_fused(const void* x, int64_t M, int64_t K, int64_t ldx, rbd_qcfg cfg,
-                             int8_t* codes, float* scales, const void* l1, int32_t r, void* ld,
+                             int8_t* codes, float* scales, const void* l1t, int32_t r, void* ld,
                              void* stream);
 
 /* Offline weight rotate + quantise + pack to signed INT4 (INT4 tensorwise card,
@@ -138,7 +140,9 @@ typedef struct rbd_epilogue {
  * accumulation on the tcgen05 INT8 tensor path, then the epilogue.
  *   codes   int8 [M, K], sx float32 [M] or [M, K/64].
  *   w_packed uint8 [N, K/2], sw float32 [N] or [N, K/64].
- *   K % 128 == 0, N % 128 == 0, M >= 1 (ragged M is handled).
+ *   K % 128 == 0, N % 128 == 0, M >= 1 (ragged M is handled).  A shape whose
+ *   per-tile scale table does not fit in shared memory (group scales with a
+ *   very large K) returns RBD_ERR_UNSUPPORTED.
  *   epi     may be NULL (no bias, branch or gate).
  *   y       bf16 [M, ldy], ldy >= N, ldy % 8 == 0.                           */
 rbd_status rbd_w4a4_linear(const int8_t* codes, const float* sx, const uint8_t* w_packed,

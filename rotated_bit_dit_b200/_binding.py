@@ -121,14 +121,16 @@ def rbd_rot_quant_act(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor
                                  _ptr(codes), _ptr(scales), _stream(stream)), "rbd_rot_quant_act")
 
 
-def rbd_lowrank_fused(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, l1: torch.Tensor,
+def rbd_lowrank_fused(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, l1t: torch.Tensor,
                       ld: torch.Tensor, bits: int = 4, rot_group: int = 256, scale_group: int = 0,
                       stream=None) -> None:
-    """rbd_rot_quant_act plus ld = X @ L1 (l1 bf16 [K, r], ld bf16 [M, r])."""
+    """rbd_rot_quant_act plus ld = X @ L1 (l1t = L1^T bf16 [r, K], ld bf16 [M, r])."""
     M, K = x.shape
-    r = l1.shape[1]
+    r = l1t.shape[0]
+    if _rowstride(l1t) != K:
+        raise ValueError("l1t must be a contiguous [r, K] tensor")
     _ok(load().rbd_lowrank_fused(_ptr(x), M, K, _rowstride(x), _qcfg(bits, rot_group, scale_group),
-                                 _ptr(codes), _ptr(scales), _ptr(l1), r, _ptr(ld), _stream(stream)),
+                                 _ptr(codes), _ptr(scales), _ptr(l1t), r, _ptr(ld), _stream(stream)),
         "rbd_lowrank_fused")
 
 

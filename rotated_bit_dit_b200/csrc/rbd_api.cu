@@ -127,6 +127,8 @@ rbd_status linear_common(const int8_t* codes, const float* sx, const void* w, co
   if (e.bias && (reinterpret_cast<uintptr_t>(e.bias) & 1u)) return RBD_ERR_ALIGNMENT;
   if (e.acc_debug && (reinterpret_cast<uintptr_t>(e.acc_debug) & 3u)) return RBD_ERR_ALIGNMENT;
 
+  if (rbd::gemm_smem_bytes(W4, e.r, G) > 227u * 1024u) return RBD_ERR_UNSUPPORTED;
+
   CUtensorMap tm_x{}, tm_w{}, tm_ld{}, tm_l2{};
   if (!make_map_2d(&tm_x, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, K, 128, 128)) return RBD_ERR_CUDA;
   if (!W4 && !make_map_2d(&tm_w, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, K, 128, 128)) return RBD_ERR_CUDA;
@@ -185,14 +187,14 @@ rbd_status rbd_rot_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, r
 }
 
 rbd_status rbd_lowrank_fused(const void* x, int64_t M, int64_t K, int64_t ldx, rbd_qcfg cfg, int8_t* codes,
-                             float* scales, const void* l1, int32_t r, void* ld, void* stream) {
+                             float* scales, const void* l1t, int32_t r, void* ld, void* stream) {
   if (r != 16 && r != 32 && r != 64) return RBD_ERR_UNSUPPORTED;
-  if (M > 0 && (!l1 || !ld)) return RBD_ERR_INVALID_ARG;
-  if (M > 0 && (!aligned16(l1) || !aligned16(ld))) return RBD_ERR_ALIGNMENT;
+  if (M > 0 && (!l1t || !ld)) return RBD_ERR_INVALID_ARG;
+  if (M > 0 && (!aligned16(l1t) || !aligned16(ld))) return RBD_ERR_ALIGNMENT;
   rbd_status s = quant_common(x, M, K, ldx, cfg, codes, scales, false, stream);
   if (s != RBD_OK || M == 0) return s;
   return cuda_status(rbd::launch_lowrank_down(static_cast<const uint16_t*>(x), M, K, ldx,
-                                              static_cast<const uint16_t*>(l1), r, static_cast<uint16_t*>(ld),
+                                              static_cast<const uint16_t*>(l1t), r, static_cast<uint16_t*>(ld),
                                               as_stream(stream)));
 }
 

@@ -79,19 +79,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity to complete.  Returns false
 // (and records RBD_ERR_DEVICE_TIMEOUT) when the bound expires or another
 // thread already recorded a failure; callers then leave their loops.
+// The status word in global memory is read only after 50 us of waiting and
+// then every 50 us, so a normal hand-off never waits behind a memory load.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           uint64_t timeout_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  uint32_t spins = 0;
+  uint64_t next_check = t0 + 50000ull;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++spins & 63u) == 0) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t now = globaltimer_ns();
+    if (now >= next_check) {
       if (device_failed()) return false;
-      if (globaltimer_ns() - t0 > timeout_ns) {
+      if (now - t0 > timeout_ns) {
         record_status(RBD_ERR_DEVICE_TIMEOUT);
         return false;
       }
+      next_check = now + 50000ull;
     }
   }
 }

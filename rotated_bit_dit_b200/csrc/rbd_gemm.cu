@@ -70,9 +70,8 @@ __host__ __device__ inline SmemLayout smem_layout(bool w4, int r, int G) {
   L.sx_stride = kTileT + 4;
   L.sx_off = off;
   off += (uint32_t)G * L.sx_stride * 4;
-  L.sw_stride = G + 1;
+  L.sw_stride = 0;
   L.sw_off = off;
-  off += (uint32_t)kTileF * L.sw_stride * 4;
   off = (off + 15u) & ~15u;
   L.bar_off = off;
   off += 32 * 8 + 16;
@@ -232,6 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp < kWarpEpi0) {
     // ------------------------------------------------------------ INT4 -> INT8 converters
+    // Each thread owns one weight row of the tile (its TMEM lane).  Packed bytes
+    // are fetched two stages ahead of the stage being widened.
     if (W4) {
       const uint32_t q = warp & 3u;
       const uint32_t lane_base = (32u * q) << 16;
@@ -243,19 +244,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nt = t / args.num_m_tiles;
         const int n = nt * kTileF + 32 * q + lane;
         const uint4* wrow = reinterpret_cast<const uint4*>(args.w4 + (int64_t)n * half_k);
-        uint4 cur[4];
+        uint4 c0[4], c1[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cur[i] = __ldg(wrow + i);
+        for (int i = 0; i < 4; ++i) c0[i] = __ldg(wrow + i);
+        if (nks > 1) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) c1[i] = __ldg(wrow + 4 + i);
+        }
         for (int ks = 0; ks < nks; ++ks) {
-          uint4 nxt[4];
-          if (ks + 1 < nks) {
+          uint4 c2[4];
+          if (ks + 2 < nks) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) nxt[i] = __ldg(wrow + (ks + 1) * 4 + i);
+            for (int i = 0; i < 4; ++i) c2[i] = __ldg(wrow + (ks + 2) * 4 + i);
           }
           uint32_t outw[32];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const uint32_t pw[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+            const uint32_t pw[4] = {c0[i].x, c0[i].y, c0[i].z, c0[i].w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint32_t lo = (pw[j] << 4) & 0xF0F0F0F0u;  // even k, as 16*q
@@ -263,6 +268,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               outw[8 * i + 2 * j] = __byte_perm(lo, hi, 0x5140);
               outw[8 * i + 2 * j + 1] = __byte_perm(lo, hi, 0x7362);
             }
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            c0[i] = c1[i];
+            c1[i] = c2[i];
           }
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           tc_fence_after();
@@ -272,22 +282,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&full[stage]);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
-          if (ks + 1 < nks) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
-          }
         }
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Thread = one output feature (TMEM lane) x 64 tokens (TMEM columns).
     const uint32_t q = warp & 3u;
     const uint32_t h = (warp - kWarpEpi0) >> 2;   // token half of the tile
     const uint32_t lane_base = (32u * q) << 16;
     const int etid = threadIdx.x - kWarpEpi0 * 32;  // 0..255
     const int G = args.G;
     float* sx_s = reinterpret_cast<float*>(smem + L.sx_off);
-    float* sw_s = reinterpret_cast<float*>(smem + L.sw_off);
     const int fr = 32 * q + lane;  // feature row of this thread in the tile
 
     // partial buffers start released; in group mode they hold the magic pattern
@@ -309,35 +315,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
       const int mt = t % args.num_m_tiles, nt = t / args.num_m_tiles;
       const int m0 = mt * kTileT, n0 = nt * kTileF;
-      // stage the tile's scales in shared memory
+      // stage the tile's activation scales in shared memory, group-major
       named_bar_epi();
       for (int e = etid; e < kTileT * G; e += kEpiThreads) {
         const int tk = e / G, g = e % G;
         const int64_t m = (int64_t)m0 + tk;
         sx_s[g * L.sx_stride + tk] = m < args.M ? __ldg(args.sx + m * G + g) : 0.f;
       }
-      for (int e = etid; e < kTileF * G; e += kEpiThreads) {
-        const int f = e / G, g = e % G;
-        sw_s[f * L.sw_stride + g] = __ldg(args.sw + (int64_t)(n0 + f) * G + g);
-      }
       named_bar_epi();
 
       const int n = n0 + fr;
-      float y[64];
+      const float* swrow = args.sw + (int64_t)n * G;
+      float sw_next = __ldg(swrow);
+      float2 y[32];
       const float bias = args.bias ? __uint_as_float((uint32_t)__ldg(args.bias + n) << 16) : 0.f;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) y[j] = bias;
+      for (int j = 0; j < 32; ++j) y[j] = make_float2(bias, bias);
       if (LR && ok) {
         if (!mbar_wait(lrfull, lr_phase)) ok = false;
         lr_phase ^= 1;
         if (ok) {
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v[16];
-            tmem_ld16(tmem + lane_base + kColLR + 64 * h + 16 * c, v);
+          for (int c = 0; c < 2; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_base + kColLR + 64 * h + 32 * c, v);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) y[16 * c + j] += __uint_as_float(v[j]);
+            for (int j = 0; j < 16; ++j) {
+              y[16 * c + j].x += __uint_as_float(v[2 * j]);
+              y[16 * c + j].y += __uint_as_float(v[2 * j + 1]);
+            }
           }
           tc_fence_before();
           __syncwarp();
@@ -345,25 +352,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       for (int g = 0; g < G && ok; ++g) {
+        const float sw_g = sw_next;
+        if (g + 1 < G) sw_next = __ldg(swrow + g + 1);
         if (!mbar_wait(&pfull[pb], pph[pb])) { ok = false; break; }
         pph[pb] ^= 1;
         tc_fence_after();
-        const float* sxg = sx_s + g * L.sx_stride + 64 * h;
-        float a = sw_s[fr * L.sw_stride + g] * args.acc_scale;
+        const float4* sxg = reinterpret_cast<const float4*>(sx_s + g * L.sx_stride + 64 * h);
+        float a = sw_g * args.acc_scale;
         float cneg = 0.f;
         if (G64) {
           a = __uint_as_float((__float_as_uint(a) + 2u) & ~3u);   // 22 significant bits
           cneg = -kMagicF * a;                                       // exact
         }
+        const float2 a2 = make_float2(a, a);
+        const float2 c2 = make_float2(cneg, cneg);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[16];
-          const uint32_t taddr = tmem + lane_base + kColP0 + pb * 128 + 64 * h + 16 * c;
-          tmem_ld16(taddr, v);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t v[32];
+          const uint32_t taddr = tmem + lane_base + kColP0 + pb * 128 + 64 * h + 32 * c;
+          tmem_ld32(taddr, v);
           if (DBG) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int64_t m = (int64_t)m0 + 64 * h + 16 * c + j;
+            for (int j = 0; j < 32; ++j) {
+              const int64_t m = (int64_t)m0 + 64 * h + 32 * c + j;
               if (m < args.M) {
                 const int32_t raw = G64 ? (int32_t)(v[j] - kMagicBits) : (int32_t)v[j];
                 const int32_t accv = W4 ? (raw >> 4) : raw;
@@ -373,16 +384,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float b = sxg[16 * c + j];
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 b4 = sxg[8 * c + j4];
+            const float2 blo = make_float2(b4.x, b4.y), bhi = make_float2(b4.z, b4.w);
+            float2& y0 = y[16 * c + 2 * j4];
+            float2& y1 = y[16 * c + 2 * j4 + 1];
             if (G64) {
-              const float tv = fmaf(__uint_as_float(v[j]), a, cneg);
-              y[16 * c + j] = fmaf(tv, b, y[16 * c + j]);
+              const float2 f0 = make_float2(__uint_as_float(v[4 * j4]), __uint_as_float(v[4 * j4 + 1]));
+              const float2 f1 = make_float2(__uint_as_float(v[4 * j4 + 2]), __uint_as_float(v[4 * j4 + 3]));
+              y0 = __ffma2_rn(__ffma2_rn(f0, a2, c2), blo, y0);
+              y1 = __ffma2_rn(__ffma2_rn(f1, a2, c2), bhi, y1);
             } else {
-              y[16 * c + j] = fmaf((float)(int32_t)v[j], a * b, y[16 * c + j]);
+              const float2 f0 = make_float2((float)(int32_t)v[4 * j4], (float)(int32_t)v[4 * j4 + 1]);
+              const float2 f1 = make_float2((float)(int32_t)v[4 * j4 + 2], (float)(int32_t)v[4 * j4 + 3]);
+              y0 = __ffma2_rn(f0, __fmul2_rn(a2, blo), y0);
+              y1 = __ffma2_rn(f1, __fmul2_rn(a2, bhi), y1);
             }
           }
-          if (G64) tmem_fill16(taddr, kMagicBits);
+          if (G64) {
+            tmem_fill16(taddr, kMagicBits);
+            tmem_fill16(taddr + 16, kMagicBits);
+          }
         }
         if (G64) tmem_wait_st();
         tc_fence_before();
@@ -394,18 +416,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       // gate and store: thread (feature n) writes tokens m0 + 64h + j
       const bool sig = args.gate_mode == 1 && n >= args.gate_c0 && n < args.gate_c1;
       const float gv = args.gate_mode == 2 ? __uint_as_float((uint32_t)__ldg(args.gate + n) << 16) : 0.f;
+      const int64_t mbase = (int64_t)m0 + 64 * h;
+      uint16_t* yp = args.y + mbase * args.ldy + n;
+      const uint16_t* rp = args.gate_mode == 2 ? args.residual + mbase * args.ldr + n : nullptr;
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
-        const int64_t m = (int64_t)m0 + 64 * h + j;
-        if (m < args.M) {
-          float o = y[j];
+        if (mbase + j < args.M) {
+          float o = (j & 1) ? y[j >> 1].y : y[j >> 1].x;
           if (sig) {
             o = 1.0f / (1.0f + __expf(-o));
           } else if (args.gate_mode == 2) {
-            const float rres = __uint_as_float((uint32_t)args.residual[m * args.ldr + n] << 16);
+            const float rres = __uint_as_float((uint32_t)rp[(int64_t)j * args.ldr] << 16);
             o = fmaf(gv, o, rres);
           }
-          args.y[m * args.ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+          yp[(int64_t)j * args.ldy] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
         }
       }
     }
@@ -426,6 +450,7 @@ cudaError_t launch_lowbit_gemm(bool w4, bool g64, const CUtensorMap& tm_x, const
                                cudaStream_t st) {
   const bool lr = a.r > 0;
   const SmemLayout L = smem_layout(w4, a.r, a.G);
+  if (L.total > 227u * 1024u) return cudaErrorInvalidConfiguration;
   const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
   const bool dbg = a.acc_debug != nullptr;
 #define RBD_GEMM_CASE(W, G, R, D)                                                                     \

@@ -250,16 +250,22 @@ __global__ void __launch_bounds__(256) rot_quant_kernel(const uint16_t* __restri
 }
 
 // ---------------------------------------------------------------------------
-// Low-rank down product ld[M, r] = X[M, K] @ L1[K, r] (unrotated bf16 input),
-// legacy bf16 mma.sync (m16n8k16), fp32 accumulation.  One CTA = 16 tokens,
-// 4 warps split K and reduce through shared memory.
+// Low-rank down product ld[M, r] = X[M, K] @ L1 (unrotated bf16 input) with L1
+// given output-major as l1t[r, K], on the legacy bf16 mma.sync path
+// (m16n8k16, fp32 accumulation).  One CTA = 16 tokens; its 8 warps split K
+// and reduce through shared memory in a fixed order (deterministic).
+// Fragment loads are 32-bit: A pairs come from consecutive k of one token row,
+// B pairs from consecutive k of one l1t row.
 // ---------------------------------------------------------------------------
+constexpr int kLrWarps = 8;
+
 template <int R>
-__global__ void __launch_bounds__(128) lowrank_down_kernel(const uint16_t* __restrict__ x, int64_t M, int K,
-                                                           int64_t ldx, const uint16_t* __restrict__ l1,
-                                                           uint16_t* __restrict__ ld) {
+__global__ void __launch_bounds__(kLrWarps * 32) lowrank_down_kernel(const uint16_t* __restrict__ x, int64_t M,
+                                                                     int K, int64_t ldx,
+                                                                     const uint16_t* __restrict__ l1t,
+                                                                     uint16_t* __restrict__ ld) {
   constexpr int NT = R / 8;
-  __shared__ float part[4][16][R + 1];
+  __shared__ float part[kLrWarps][16][R + 1];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c4 = lane & 3;
   const int64_t m0 = (int64_t)blockIdx.x * 16;
@@ -268,23 +274,23 @@ __global__ void __launch_bounds__(128) lowrank_down_kernel(const uint16_t* __res
   float acc[NT][4];
 #pragma unroll
   for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-  const int kper = K / 4;
+  const int kper = K / kLrWarps;
   const int kbeg = warp * kper, kend = kbeg + kper;
+  const uint32_t* xa = reinterpret_cast<const uint32_t*>(x + (va ? ra : 0) * ldx);
+  const uint32_t* xb = reinterpret_cast<const uint32_t*>(x + (vb ? rb : 0) * ldx);
+#pragma unroll 4
   for (int k = kbeg; k < kend; k += 16) {
+    const int kw = k >> 1;   // 32-bit word index of k
     uint32_t a[4];
-    const uint32_t* xa = reinterpret_cast<const uint32_t*>(x + ra * ldx + k);
-    const uint32_t* xb = reinterpret_cast<const uint32_t*>(x + rb * ldx + k);
-    a[0] = va ? __ldg(xa + c4) : 0u;
-    a[1] = vb ? __ldg(xb + c4) : 0u;
-    a[2] = va ? __ldg(xa + c4 + 4) : 0u;
-    a[3] = vb ? __ldg(xb + c4 + 4) : 0u;
+    a[0] = va ? __ldg(xa + kw + c4) : 0u;
+    a[1] = vb ? __ldg(xb + kw + c4) : 0u;
+    a[2] = va ? __ldg(xa + kw + c4 + 4) : 0u;
+    a[3] = vb ? __ldg(xb + kw + c4 + 4) : 0u;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-      const int col = n * 8 + g;
-      const uint32_t b0 = (uint32_t)__ldg(l1 + (int64_t)(k + 2 * c4) * R + col) |
-                          ((uint32_t)__ldg(l1 + (int64_t)(k + 2 * c4 + 1) * R + col) << 16);
-      const uint32_t b1 = (uint32_t)__ldg(l1 + (int64_t)(k + 2 * c4 + 8) * R + col) |
-                          ((uint32_t)__ldg(l1 + (int64_t)(k + 2 * c4 + 9) * R + col) << 16);
+      const uint32_t* lb = reinterpret_cast<const uint32_t*>(l1t + (int64_t)(n * 8 + g) * K) + kw;
+      const uint32_t b0 = __ldg(lb + c4);
+      const uint32_t b1 = __ldg(lb + c4 + 4);
       asm volatile(
           "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
           "{%0,%1,%2,%3};"
@@ -304,7 +310,9 @@ __global__ void __launch_bounds__(128) lowrank_down_kernel(const uint16_t* __res
     const int rr = i / R, cc = i % R;
     const int64_t mm = m0 + rr;
     if (mm < M) {
-      const float s = (part[0][rr][cc] + part[1][rr][cc]) + (part[2][rr][cc] + part[3][rr][cc]);
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < kLrWarps; ++w) s += part[w][rr][cc];
       ld[mm * R + cc] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
     }
   }
@@ -383,15 +391,16 @@ cudaError_t launch_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ld
 #undef RBD_RQ_DISPATCH
 }
 
-cudaError_t launch_lowrank_down(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const uint16_t* l1, int r,
+cudaError_t launch_lowrank_down(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const uint16_t* l1t, int r,
                                 uint16_t* ld, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   const dim3 grid(static_cast<unsigned>((M + 15) / 16));
   const int Ki = static_cast<int>(K);
+  const int threads = kLrWarps * 32;
   switch (r) {
-    case 16: lowrank_down_kernel<16><<<grid, 128, 0, st>>>(x, M, Ki, ldx, l1, ld); break;
-    case 32: lowrank_down_kernel<32><<<grid, 128, 0, st>>>(x, M, Ki, ldx, l1, ld); break;
-    case 64: lowrank_down_kernel<64><<<grid, 128, 0, st>>>(x, M, Ki, ldx, l1, ld); break;
+    case 16: lowrank_down_kernel<16><<<grid, threads, 0, st>>>(x, M, Ki, ldx, l1t, ld); break;
+    case 32: lowrank_down_kernel<32><<<grid, threads, 0, st>>>(x, M, Ki, ldx, l1t, ld); break;
+    case 64: lowrank_down_kernel<64><<<grid, threads, 0, st>>>(x, M, Ki, ldx, l1t, ld); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -39,7 +39,7 @@ class RotatedLowBitLinear:
         else:
             raise ValueError("bits must be 4 or 8")
         self.bias = bias.contiguous() if bias is not None else None
-        self.l1 = l1.contiguous() if l1 is not None else None
+        self.l1t = l1.t().contiguous() if l1 is not None else None
         self.l2t = l2.t().contiguous() if l2 is not None else None
         self.rank = 0 if l1 is None else int(l1.shape[1])
         self.gate_mode, self.gate_cols = gate_mode, gate_cols
@@ -61,7 +61,7 @@ class RotatedLowBitLinear:
         M = x.shape[0]
         codes, sx, ld = self.buffers(M, x.device)
         if self.rank:
-            B.rbd_lowrank_fused(x, codes, sx, self.l1, ld, self.bits, self.rot_group, self.scale_group)
+            B.rbd_lowrank_fused(x, codes, sx, self.l1t, ld, self.bits, self.rot_group, self.scale_group)
         else:
             B.rbd_rot_quant_act(x, codes, sx, self.bits, self.rot_group, self.scale_group)
         if out is None:

@@ -103,11 +103,11 @@ def test_lowrank_fused(r, M):
     K = 3072
     xb = I.gaussian_bf16(13, (M, K), 1.0, 0.005, 30.0)
     l1b = I.gaussian_bf16(14, (K, r), 0.01)
-    x, l1 = dev_bf16(xb), dev_bf16(l1b)
+    x, l1t = dev_bf16(xb), dev_bf16(np.ascontiguousarray(l1b.T))
     codes = torch.empty((M, K), dtype=torch.int8, device="cuda")
     scales = torch.empty((M, K // 64), dtype=torch.float32, device="cuda")
     ld = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
-    R.rbd_lowrank_fused(x, codes, scales, l1, ld, 4, 256, 64)
+    R.rbd_lowrank_fused(x, codes, scales, l1t, ld, 4, 256, 64)
     assert R.rbd_check() == 0
     ref_q, ref_s = O.rot_quant(xb, 4, 256, 64)
     assert np.array_equal(codes.cpu().numpy(), ref_q) and np.array_equal(scales.cpu().numpy(), ref_s)
