@@ -127,13 +127,15 @@ rbd_status linear_common(const int8_t* codes, const float* sx, const void* w, co
   if (e.bias && (reinterpret_cast<uintptr_t>(e.bias) & 1u)) return RBD_ERR_ALIGNMENT;
   if (e.acc_debug && (reinterpret_cast<uintptr_t>(e.acc_debug) & 3u)) return RBD_ERR_ALIGNMENT;
 
-  if (rbd::gemm_smem_bytes(W4, e.r, G) > 227u * 1024u) return RBD_ERR_UNSUPPORTED;
+  const bool g64 = cfg.scale_group == 64;
+  if (rbd::gemm_smem_bytes(g64, e.r, G) > 227u * 1024u) return RBD_ERR_UNSUPPORTED;
+  const int tt = rbd::gemm_tile_tokens(g64);
 
   CUtensorMap tm_x{}, tm_w{}, tm_ld{}, tm_l2{};
-  if (!make_map_2d(&tm_x, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, K, 128, 128)) return RBD_ERR_CUDA;
+  if (!make_map_2d(&tm_x, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, K, 128, tt)) return RBD_ERR_CUDA;
   if (!W4 && !make_map_2d(&tm_w, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, K, 128, 128)) return RBD_ERR_CUDA;
   if (e.r) {
-    if (!make_map_2d(&tm_ld, e.ld, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, e.r, M, 2 * e.r, e.r, 128))
+    if (!make_map_2d(&tm_ld, e.ld, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, e.r, M, 2 * e.r, e.r, tt))
       return RBD_ERR_CUDA;
     if (!make_map_2d(&tm_l2, e.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, e.r, N, 2 * e.r, e.r, 128))
       return RBD_ERR_CUDA;
@@ -159,7 +161,7 @@ rbd_status linear_common(const int8_t* codes, const float* sx, const void* w, co
   a.ldy = ldy;
   a.acc_debug = e.acc_debug;
   a.acc_scale = W4 ? 1.0f / 16.0f : 1.0f;
-  a.num_m_tiles = static_cast<int>((M + 127) / 128);
+  a.num_m_tiles = static_cast<int>((M + tt - 1) / tt);
   a.num_tiles = a.num_m_tiles * static_cast<int>(N / 128);
   const int sms = num_sms_current();
   if (sms <= 0) return RBD_ERR_CUDA;

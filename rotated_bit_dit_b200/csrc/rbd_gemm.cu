@@ -8,25 +8,41 @@
 // updates in the GEMM epilogues), plus the parallel low-rank branch of
 // "Krea-2-SVDQuant-ComfyUI", section "LoRA".
 //
-// Orientation ("swap AB"): the MMA's M side is 128 output features (weights),
-// its N side 128 tokens, so TMEM lane = output feature and TMEM column = token.
-//   - W4A4: weights are widened from packed nibbles to INT8 in registers by
-//     four converter warps and written straight into tensor memory with
-//     tcgen05.st; the MMA reads A from TMEM (tcgen05 has no INT4 kind).  A
+// Tile and orientation.  One CTA computes 128 output features x TT tokens:
+// the MMA's M side is the weights (TMEM lane = output feature), its N side the
+// tokens (TMEM column = token).  On B200 one tcgen05.mma kind::i8 instruction
+// (M=128, K=32) takes about the same time for any N up to 256, so wide N is
+// what reaches the tensor pipe's rate.  Both operands are read from shared
+// memory (128-byte swizzled, K-major):
+//   - activation codes (int8) arrive by TMA, TT rows x 128 bytes per stage;
+//   - W8A8 weights arrive by TMA, 128 rows x 128 bytes per stage;
+//   - W4A4 weights are widened from packed nibbles by four converter warps
+//     and written into the same swizzled layout.  tcgen05 has no INT4 kind; a
 //     nibble is placed in the high half of its byte (value 16*q, exact), so
-//     widening is a shift, two masks and two byte permutes per 8 codes; the
-//     accumulator is 16 * acc and the epilogue folds the 1/16 into the scale.
-//   - W8A8: weights come by TMA into shared memory; both operands from smem.
-//   - Activation codes (int8) always come by TMA (128-byte swizzle).
-// Accumulation segments: one segment per tile (row scales) or one per 64-wide
-// K block (group scales).  Two 128-column int32 partial buffers in TMEM
-// alternate, so the tensor core fills one while the epilogue drains the
-// other.  In group mode each partial starts from the bit pattern of
-// 12582912.0f (1.5 * 2^23): the int32 result reinterpreted as float is then
-// exactly 12582912 + 16*acc, and fma(f, a, -12582912*a) yields the correctly
-// rounded 16*acc*a with no int->float conversion.  (a is the weight scale
-// rounded to 22 significant bits so that 12582912*a is exact; the relative
-// change of the scale is below 2^-22.)
+//     widening is a shift, two masks and two byte permutes per 8 codes, and
+//     the epilogue folds the factor 1/16 into the weight scale.
+// Accumulation segments.  NB int32 accumulators of TT columns each rotate in
+// TMEM: the tensor core fills one while the epilogue drains another.  A
+// segment is the whole K range (row scales) or one 64-wide K block (group
+// scales); the low-rank branch, when present, is one more segment per tile,
+// computed with a bf16 MMA (fp32 result) into the same buffers.
+//   - Row scales: TT = 256, NB = 2.  One promotion per tile.
+//   - Group scales: TT = 160, NB = 3 (3 x 160 columns fit the 512 of TMEM).
+//     Every 64-wide K block needs its own promotion, so the epilogue is the
+//     busy side: three buffers let the tensor core run two segments ahead, and
+//     with 80 columns per thread all five TMEM loads of a segment are issued
+//     before a single wait.
+// In group mode each partial starts from the bit pattern of 12582912.0f
+// (1.5 * 2^23): the int32 result read as float is then exactly
+// 12582912 + 16*acc, and fma(f, a, -12582912*a) gives the correctly rounded
+// 16*acc*a without an int->float conversion (a is the weight scale rounded to
+// 22 significant bits so that 12582912*a is exact; the relative change of the
+// scale is below 2^-22).
+//
+// Warp roles (16 warps, registers redistributed per warpgroup with setmaxnreg):
+//   warpgroup 0: warps 0, 2, 3 TMA producers, warp 1 TMEM allocator + MMA issuer;
+//   warpgroup 1: INT4 -> INT8 converters (W4A4 only);
+//   warpgroups 2-3: epilogue, thread = one output feature x TT/2 tokens.
 #include "rbd_common.cuh"
 #include "rbd_internal.cuh"
 
@@ -35,43 +51,61 @@ namespace rbd {
 namespace {
 
 constexpr int kTileF = 128;    // output features per tile (TMEM lanes)
-constexpr int kTileT = 128;    // tokens per tile (MMA N)
-constexpr int kBK = 128;       // K per pipeline stage (one 128-byte swizzle row of codes)
-constexpr int kStages = 4;
-constexpr int kThreads = 448;  // 14 warps
-constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpConv0 = 2, kWarpEpi0 = 6;
+constexpr int kBK = 128;       // K per pipeline stage (one 128-byte swizzle row)
+constexpr int kMaxStages = 4;
+constexpr int kThreads = 512;  // 16 warps
+constexpr int kWarpMma = 1, kWarpConv0 = 4, kWarpEpi0 = 8;
+constexpr int kProducers = 3;  // warps 0, 2, 3
 constexpr int kEpiThreads = 256;
 constexpr uint32_t kMagicBits = 0x4B400000u;  // 12582912.0f
 constexpr float kMagicF = 12582912.0f;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColP0 = 0, kColA = 256, kColLR = 384;
+constexpr uint32_t kWStageBytes = kTileF * kBK;   // 16 KB
+
+__host__ __device__ constexpr int tile_tokens(bool g64) { return g64 ? 160 : 256; }
+__host__ __device__ constexpr int num_bufs(bool g64) { return g64 ? 3 : 2; }
 
 __device__ __forceinline__ void named_bar_epi() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 }  // namespace
 
 struct SmemLayout {
-  uint32_t x_off, w_off, ld_off, l2_off, sx_off, sw_off, bar_off, total;
-  int sx_stride, sw_stride;
+  uint32_t x_off, w_off, ld_off, l2_off, sx_off, bar_off, total, x_stage;
+  int stages, sx_stride;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(bool w4, int r, int G) {
+__host__ __device__ inline SmemLayout smem_layout(int stages, int r, int G, int tt) {
   SmemLayout L{};
   uint32_t off = 0;
+  L.stages = stages;
+  L.x_stage = (uint32_t)tt * kBK;
   L.x_off = off;
-  off += kStages * kTileT * kBK;
+  off += stages * L.x_stage;
+  off = (off + 1023u) & ~1023u;
   L.w_off = off;
-  if (!w4) off += kStages * kTileF * kBK;
+  off += stages * kWStageBytes;
   L.ld_off = off;
-  off += kTileT * r * 2;
+  off += (uint32_t)tt * r * 2;
+  off = (off + 1023u) & ~1023u;
   L.l2_off = off;
   off += kTileF * r * 2;
   off = (off + 1023u) & ~1023u;
-  L.sx_stride = kTileT + 4;
+  L.sx_stride = tt + 4;
   L.sx_off = off;
   off += (uint32_t)G * L.sx_stride * 4;
-  L.sw_stride = 0;
-  L.sw_off = off;
   off = (off + 15u) & ~15u;
   L.bar_off = off;
   off += 32 * 8 + 16;
@@ -79,23 +113,77 @@ __host__ __device__ inline SmemLayout smem_layout(bool w4, int r, int G) {
   return L;
 }
 
+// Number of pipeline stages that fit (up to 4, at least 2); 0 if none.
+__host__ __device__ inline int pick_stages(int r, int G, int tt) {
+  for (int s = kMaxStages; s >= 2; --s)
+    if (smem_layout(s, r, G, tt).total <= 227u * 1024u) return s;
+  return 0;
+}
+
+// Group-scale promotion of NC 16-column chunks (chunks CB .. CB+NC-1 of this
+// thread's columns) from a register buffer holding magic-biased int32 partials:
+// y += (16*acc*a) * b, with (f - 12582912) * a computed by one fma.
+template <int CB, int NC, int NY, bool W4, bool DBG>
+__device__ __forceinline__ void promote_g64(float2 (&y)[NY], const uint32_t (&v)[2][16], const float4* sxg,
+                                            float2 a2, float2 c2, int32_t* dbg, int64_t dbg_stride,
+                                            int64_t mrow0, int64_t M) {
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    if (DBG) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int64_t m = mrow0 + 16 * (CB + c) + j;
+        if (m < M) {
+          const int32_t raw = (int32_t)(v[c][j] - kMagicBits);
+          dbg[m * dbg_stride] = W4 ? (raw >> 4) : raw;
+        }
+      }
+    }
+#pragma unroll
+    for (int j4 = 0; j4 < 4; ++j4) {
+      const float4 b4 = sxg[4 * (CB + c) + j4];
+      const float2 f0 = make_float2(__uint_as_float(v[c][4 * j4]), __uint_as_float(v[c][4 * j4 + 1]));
+      const float2 f1 = make_float2(__uint_as_float(v[c][4 * j4 + 2]), __uint_as_float(v[c][4 * j4 + 3]));
+      float2& y0 = y[8 * (CB + c) + 2 * j4];
+      float2& y1 = y[8 * (CB + c) + 2 * j4 + 1];
+      y0 = __ffma2_rn(__ffma2_rn(f0, a2, c2), make_float2(b4.x, b4.y), y0);
+      y1 = __ffma2_rn(__ffma2_rn(f1, a2, c2), make_float2(b4.z, b4.w), y1);
+    }
+  }
+}
+
+template <int NC>
+__device__ __forceinline__ void tmem_load_chunks(uint32_t taddr, uint32_t (&v)[2][16]) {
+#pragma unroll
+  for (int c = 0; c < NC; ++c) tmem_ld16_async(taddr + 16 * c, v[c]);
+}
+
+template <int NC>
+__device__ __forceinline__ void tmem_fence_chunks(uint32_t (&v)[2][16]) {
+#pragma unroll
+  for (int c = 0; c < NC; ++c) tmem_reg_fence(v[c]);
+}
+
 template <bool W4, bool G64, bool LR, bool DBG>
 __global__ void __launch_bounds__(kThreads, 1)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w8,
                        const __grid_constant__ CUtensorMap tm_ld, const __grid_constant__ CUtensorMap tm_l2,
                        const GemmArgs args) {
+  constexpr int TT = tile_tokens(G64);
+  constexpr int NB = num_bufs(G64);
+  constexpr int EC = TT / 2;       // TMEM columns (tokens) per epilogue thread
+  constexpr int NCH = EC / 16;     // 16-column chunks per epilogue thread
   extern __shared__ unsigned char smem_dyn[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023u) & ~uintptr_t(1023u));
-  const SmemLayout L = smem_layout(W4, LR ? args.r : 0, args.G);
+  const int S = pick_stages(LR ? args.r : 0, args.G, TT);
+  const SmemLayout L = smem_layout(S, LR ? args.r : 0, args.G, TT);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  uint64_t* full = bars;                 // [kStages]
-  uint64_t* empty = bars + kStages;      // [kStages]
-  uint64_t* pfull = bars + 2 * kStages;  // [2]
-  uint64_t* pempty = pfull + 2;          // [2]
-  uint64_t* lrfull = pempty + 2;
-  uint64_t* lrempty = lrfull + 1;
-  uint64_t* lrsfull = lrempty + 1;
+  uint64_t* full = bars;                    // [kMaxStages]
+  uint64_t* empty = bars + kMaxStages;      // [kMaxStages]
+  uint64_t* pfull = bars + 2 * kMaxStages;  // [NB]
+  uint64_t* pempty = pfull + 3;             // [NB]
+  uint64_t* lrsfull = pempty + 3;
   uint64_t* lrsempty = lrsfull + 1;
   uint64_t* drain = lrsempty + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -103,17 +191,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
 
-  if (warp == kWarpProducer && lane == 0) {
-    for (int s = 0; s < kStages; ++s) {
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], W4 ? 1 + 4 : 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NB; ++b) {
       mbar_init(&pfull[b], 1);
       mbar_init(&pempty[b], kEpiThreads / 32);
     }
-    mbar_init(lrfull, 1);
-    mbar_init(lrempty, kEpiThreads / 32);
     mbar_init(lrsfull, 1);
     mbar_init(lrsempty, 1);
     mbar_init(drain, 1);
@@ -136,113 +222,123 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int K = args.K;
   const int nks = K / kBK;
-  const uint32_t x_stage_bytes = kTileT * kBK;
+  const int seg = args.seg;
 
-  if (warp == kWarpProducer) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, lr_phase = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
-        const int mt = t % args.num_m_tiles, nt = t / args.num_m_tiles;
-        const int m0 = mt * kTileT, n0 = nt * kTileF;
-        if (LR) {
-          if (!mbar_wait(lrsempty, lr_phase ^ 1)) { ok = false; break; }
-          const uint32_t bytes = (uint32_t)(kTileT + kTileF) * args.r * 2;
-          mbar_arrive_expect_tx(lrsfull, bytes);
-          tma_load_2d(smem + L.ld_off, &tm_ld, lrsfull, 0, m0);
-          tma_load_2d(smem + L.l2_off, &tm_l2, lrsfull, 0, n0);
-          lr_phase ^= 1;
-        }
-        for (int ks = 0; ks < nks; ++ks) {
-          if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], W4 ? x_stage_bytes : 2 * x_stage_bytes);
-          tma_load_2d(smem + L.x_off + stage * x_stage_bytes, &tm_x, &full[stage], ks * kBK, m0);
-          if (!W4) tma_load_2d(smem + L.w_off + stage * x_stage_bytes, &tm_w8, &full[stage], ks * kBK, n0);
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
-        }
-      }
-      if (!ok) {
-        // let bulk copies already in flight land before the CTA can exit
-        const uint64_t t0 = globaltimer_ns();
-        while (globaltimer_ns() - t0 < 200000ull) {}
-      }
-    }
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issuer
-    if (elect_one()) {
-      const uint32_t idesc = idesc_i8(kTileF, kTileT);
-      const uint32_t idesc_lr = idesc_bf16(kTileF, kTileT);
-      int stage = 0;
-      uint32_t phase = 0, lr_phase = 0;
-      uint32_t pb = 0, pph[2] = {0, 0};
-      bool ok = true;
-      const int seg = args.seg;
-      const uint32_t lr_row_bytes = (uint32_t)args.r * 2;
-      for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
-        if (LR) {
-          if (!mbar_wait(lrsfull, lr_phase) || !mbar_wait(lrempty, lr_phase)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + L.l2_off), b0 = smem_u32(smem + L.ld_off);
-          for (int kk = 0; kk < args.r / 16; ++kk) {
-            mma_bf16_ss(tmem + kColLR, smem_desc_kmajor(a0 + kk * 32, lr_row_bytes),
-                        smem_desc_kmajor(b0 + kk * 32, lr_row_bytes), idesc_lr, kk > 0 ? 1u : 0u);
+  if (warp < 4) {
+    setmaxnreg_dec<40>();
+    if (warp != kWarpMma) {
+      // ---------------------------------------------------------- TMA producers
+      // Warps 0, 2 and 3 own the pipeline stages round-robin: bulk tensor
+      // loads issued by one thread complete one after another, so several
+      // issuing warps keep several stages in flight.  The number of producers
+      // never exceeds the number of stages: a producer's previous wait then
+      // guarantees that the slot it waits on is at most one phase behind, which
+      // is what a parity wait can tell apart.
+      const int nprod = S < kProducers ? S : kProducers;
+      const int pidx = warp == 0 ? 0 : (int)warp - 1;   // 0, 1, 2
+      if (lane == 0 && pidx < nprod) {
+        uint32_t lr_phase = 0;
+        bool ok = true;
+        int i = 0;   // stage counter of this CTA
+        for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
+          const int mt = t % args.num_m_tiles, nt = t / args.num_m_tiles;
+          const int m0 = mt * TT, n0 = nt * kTileF;
+          if (LR && pidx == 0) {
+            if (!mbar_wait(lrsempty, lr_phase ^ 1)) { ok = false; break; }
+            const uint32_t bytes = (uint32_t)(TT + kTileF) * args.r * 2;
+            mbar_arrive_expect_tx(lrsfull, bytes);
+            tma_load_2d(smem + L.ld_off, &tm_ld, lrsfull, 0, m0);
+            tma_load_2d(smem + L.l2_off, &tm_l2, lrsfull, 0, n0);
+            lr_phase ^= 1;
           }
-          tc_commit(lrfull);
-          tc_commit(lrsempty);
-          lr_phase ^= 1;
+          for (int ks = 0; ks < nks; ++ks, ++i) {
+            if (i % nprod != pidx) continue;
+            const int stage = i % S;
+            const uint32_t phase = (uint32_t)(i / S) & 1u;
+            if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+            mbar_arrive_expect_tx(&full[stage], W4 ? L.x_stage : L.x_stage + kWStageBytes);
+            tma_load_2d(smem + L.x_off + stage * L.x_stage, &tm_x, &full[stage], ks * kBK, m0);
+            if (!W4) tma_load_2d(smem + L.w_off + stage * kWStageBytes, &tm_w8, &full[stage], ks * kBK, n0);
+          }
         }
-        for (int ks = 0; ks < nks && ok; ++ks) {
-          if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t xs = smem_u32(smem + L.x_off + stage * x_stage_bytes);
-          const uint64_t bdesc = smem_desc_kmajor(xs, 128);
-          uint64_t adesc = 0;
-          if (!W4) adesc = smem_desc_kmajor(smem_u32(smem + L.w_off + stage * x_stage_bytes), 128);
+        if (!ok) {
+          // let bulk copies already in flight land before the CTA can exit
+          const uint64_t t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 200000ull) {}
+        }
+      }
+    } else {
+      // ---------------------------------------------------------- MMA issuer
+      if (elect_one()) {
+        const uint32_t idesc = idesc_i8(kTileF, TT);
+        const uint32_t idesc_lr = idesc_bf16(kTileF, TT);
+        int stage = 0;
+        uint32_t phase = 0, lr_phase = 0;
+        int pb = 0;
+        uint32_t pph[NB];
 #pragma unroll
-          for (int kk = 0; kk < kBK / 32; ++kk) {
-            const int kpos = ks * kBK + kk * 32;
-            if (kpos % seg == 0) {
-              if (!mbar_wait(&pempty[pb], pph[pb])) { ok = false; break; }
-              pph[pb] ^= 1;
-              tc_fence_after();
+        for (int b = 0; b < NB; ++b) pph[b] = 0;
+        bool ok = true;
+        const uint32_t lr_row_bytes = (uint32_t)args.r * 2;
+        for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
+          if (LR) {
+            if (!mbar_wait(lrsfull, lr_phase) || !mbar_wait(&pempty[pb], pph[pb])) { ok = false; break; }
+            pph[pb] ^= 1;
+            lr_phase ^= 1;
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(smem + L.l2_off), b0 = smem_u32(smem + L.ld_off);
+            for (int kk = 0; kk < args.r / 16; ++kk) {
+              mma_bf16_ss(tmem + pb * TT, smem_desc_kmajor(a0 + kk * 32, lr_row_bytes),
+                          smem_desc_kmajor(b0 + kk * 32, lr_row_bytes), idesc_lr, kk > 0 ? 1u : 0u);
             }
-            const uint32_t acc = G64 ? 1u : (kpos % seg != 0 ? 1u : 0u);
-            const uint32_t d = tmem + kColP0 + pb * 128;
-            if (W4) {
-              mma_i8_ts(d, tmem + kColA + stage * 32 + kk * 8, bdesc + (uint64_t)(kk * 2), idesc, acc);
-            } else {
-              mma_i8_ss(d, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc, acc);
-            }
-            if ((kpos + 32) % seg == 0) {
-              tc_commit(&pfull[pb]);
-              pb ^= 1;
-            }
+            tc_commit(&pfull[pb]);
+            tc_commit(lrsempty);
+            pb = pb + 1 == NB ? 0 : pb + 1;
           }
-          tc_commit(&empty[stage]);
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
+          for (int ks = 0; ks < nks && ok; ++ks) {
+            if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t bdesc = smem_desc_kmajor(smem_u32(smem + L.x_off + stage * L.x_stage), 128);
+            const uint64_t adesc = smem_desc_kmajor(smem_u32(smem + L.w_off + stage * kWStageBytes), 128);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 32; ++kk) {
+              const int kpos = ks * kBK + kk * 32;
+              if (kpos % seg == 0) {
+                if (!mbar_wait(&pempty[pb], pph[pb])) { ok = false; break; }
+                pph[pb] ^= 1;
+                tc_fence_after();
+              }
+              const uint32_t acc = G64 ? 1u : (kpos % seg != 0 ? 1u : 0u);
+              mma_i8_ss(tmem + pb * TT, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc, acc);
+              if ((kpos + 32) % seg == 0) {
+                tc_commit(&pfull[pb]);
+                pb = pb + 1 == NB ? 0 : pb + 1;
+              }
+            }
+            tc_commit(&empty[stage]);
+            if (++stage == S) { stage = 0; phase ^= 1; }
+          }
         }
+        // every issued MMA must complete before TMEM can be released
+        tc_commit(drain);
+        mbar_wait(drain, 0, 100000000ull);
       }
-      // make sure every issued MMA has completed before TMEM can be released
-      tc_commit(drain);
-      mbar_wait(drain, 0, 100000000ull);
+      __syncwarp();
     }
-    __syncwarp();
   } else if (warp < kWarpEpi0) {
+    setmaxnreg_dec<88>();
     // ------------------------------------------------------------ INT4 -> INT8 converters
-    // Each thread owns one weight row of the tile (its TMEM lane).  Packed bytes
-    // are fetched two stages ahead of the stage being widened.
+    // Thread = one weight row of the tile.  Packed bytes are fetched two
+    // stages ahead; widened bytes go to the 128-byte-swizzled A stage.
     if (W4) {
-      const uint32_t q = warp & 3u;
-      const uint32_t lane_base = (32u * q) << 16;
+      const uint32_t fr = (warp - kWarpConv0) * 32 + lane;
       const int half_k = K / 2;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
         const int nt = t / args.num_m_tiles;
-        const int n = nt * kTileF + 32 * q + lane;
+        const int n = nt * kTileF + fr;
         const uint4* wrow = reinterpret_cast<const uint4*>(args.w4 + (int64_t)n * half_k);
         uint4 c0[4], c1[4];
 #pragma unroll
@@ -257,37 +353,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) c2[i] = __ldg(wrow + (ks + 2) * 4 + i);
           }
-          uint32_t outw[32];
+          if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+          unsigned char* arow = smem + L.w_off + stage * kWStageBytes + fr * 128;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
+            // 16 packed bytes = codes k = 32i .. 32i+31 -> 16-byte chunks 2i and 2i+1
             const uint32_t pw[4] = {c0[i].x, c0[i].y, c0[i].z, c0[i].w};
+            uint32_t o[8];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint32_t lo = (pw[j] << 4) & 0xF0F0F0F0u;  // even k, as 16*q
               const uint32_t hi = pw[j] & 0xF0F0F0F0u;         // odd k, as 16*q
-              outw[8 * i + 2 * j] = __byte_perm(lo, hi, 0x5140);
-              outw[8 * i + 2 * j + 1] = __byte_perm(lo, hi, 0x7362);
+              o[2 * j] = __byte_perm(lo, hi, 0x5140);
+              o[2 * j + 1] = __byte_perm(lo, hi, 0x7362);
             }
+            const uint32_t ch0 = (2u * i) ^ (fr & 7u), ch1 = (2u * i + 1u) ^ (fr & 7u);
+            *reinterpret_cast<uint4*>(arow + ch0 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(arow + ch1 * 16) = make_uint4(o[4], o[5], o[6], o[7]);
           }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[stage]);
+          if (++stage == S) { stage = 0; phase ^= 1; }
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             c0[i] = c1[i];
             c1[i] = c2[i];
           }
-          if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
-          tc_fence_after();
-          tmem_st32(tmem + lane_base + kColA + stage * 32, outw);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full[stage]);
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
       }
     }
   } else {
+    setmaxnreg_inc<192>();
     // ------------------------------------------------------------ epilogue
-    // Thread = one output feature (TMEM lane) x 64 tokens (TMEM columns).
+    // Thread = one output feature (TMEM lane) x EC tokens (TMEM columns).
     const uint32_t q = warp & 3u;
     const uint32_t h = (warp - kWarpEpi0) >> 2;   // token half of the tile
     const uint32_t lane_base = (32u * q) << 16;
@@ -295,29 +394,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int G = args.G;
     float* sx_s = reinterpret_cast<float*>(smem + L.sx_off);
     const int fr = 32 * q + lane;  // feature row of this thread in the tile
+    const uint32_t col0 = EC * h;
 
-    // partial buffers start released; in group mode they hold the magic pattern
+    // every partial buffer starts released; in group mode it holds the magic pattern
     if (G64) {
-      for (int b = 0; b < 2; ++b)
-        for (int c = 0; c < 4; ++c) tmem_fill16(tmem + lane_base + kColP0 + b * 128 + 64 * h + 16 * c, kMagicBits);
+      for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) tmem_fill16(tmem + lane_base + b * TT + col0 + 16 * c, kMagicBits);
       tmem_wait_st();
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(&pempty[0]);
-      mbar_arrive(&pempty[1]);
-      if (LR) mbar_arrive(lrempty);
-    }
+    if (lane == 0)
+      for (int b = 0; b < NB; ++b) mbar_arrive(&pempty[b]);
 
-    uint32_t pb = 0, pph[2] = {0, 0}, lr_phase = 0;
+    int pb = 0;
+    uint32_t pph[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) pph[b] = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
       const int mt = t % args.num_m_tiles, nt = t / args.num_m_tiles;
-      const int m0 = mt * kTileT, n0 = nt * kTileF;
+      const int m0 = mt * TT, n0 = nt * kTileF;
       // stage the tile's activation scales in shared memory, group-major
       named_bar_epi();
-      for (int e = etid; e < kTileT * G; e += kEpiThreads) {
+      for (int e = etid; e < TT * G; e += kEpiThreads) {
         const int tk = e / G, g = e % G;
         const int64_t m = (int64_t)m0 + tk;
         sx_s[g * L.sx_stride + tk] = m < args.M ? __ldg(args.sx + m * G + g) : 0.f;
@@ -327,109 +428,230 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = n0 + fr;
       const float* swrow = args.sw + (int64_t)n * G;
       float sw_next = __ldg(swrow);
-      float2 y[32];
+      float2 y[EC / 2];
       const float bias = args.bias ? __uint_as_float((uint32_t)__ldg(args.bias + n) << 16) : 0.f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) y[j] = make_float2(bias, bias);
+      for (int j = 0; j < EC / 2; ++j) y[j] = make_float2(bias, bias);
+
       if (LR && ok) {
-        if (!mbar_wait(lrfull, lr_phase)) ok = false;
-        lr_phase ^= 1;
+        // low-rank segment: fp32 branch result, added once
+        if (!mbar_wait(&pfull[pb], pph[pb])) ok = false;
         if (ok) {
+          pph[pb] ^= 1;
           tc_fence_after();
+          const uint32_t tbase = tmem + lane_base + pb * TT + col0;
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_base + kColLR + 64 * h + 32 * c, v);
+          for (int c = 0; c < NCH; ++c) {
+            uint32_t v[16];
+            tmem_ld16(tbase + 16 * c, v);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              y[16 * c + j].x += __uint_as_float(v[2 * j]);
-              y[16 * c + j].y += __uint_as_float(v[2 * j + 1]);
+            for (int j = 0; j < 8; ++j) {
+              y[8 * c + j].x += __uint_as_float(v[2 * j]);
+              y[8 * c + j].y += __uint_as_float(v[2 * j + 1]);
+            }
+          }
+          if (G64) {
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) tmem_fill16(tbase + 16 * c, kMagicBits);
+            tmem_wait_st();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pempty[pb]);
+          pb = pb + 1 == NB ? 0 : pb + 1;
+        }
+      }
+      if constexpr (G64) {
+        // Group scales, software-pipelined.  Each segment's five 16-column
+        // chunks are processed in three phases ({0,1}, {2,3}, {4}); while one
+        // phase is promoted the next phase's TMEM load is in flight (two
+        // register buffers, X and Y, used alternately; the segment loop is
+        // unrolled by two so the buffer order stays static -- the number of
+        // 64-wide groups is even because K is a multiple of 128).  A drained
+        // buffer is refilled with the magic pattern and released one phase
+        // later, so the store wait is off the critical path.
+        static_assert(NCH == 5, "group-scale tiles hold five chunks per thread");
+        uint32_t vX[2][16], vY[2][16];
+        int rel = -1;
+        const int64_t dstride = args.N;
+        int32_t* dbg_base = DBG ? args.acc_debug + n : nullptr;
+        const int64_t mrow0 = (int64_t)m0 + col0;
+        auto release = [&](int b) {
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pempty[b]);
+        };
+        auto seg_scale = [&](float swv, float2& a2, float2& c2) {
+          float a = swv * args.acc_scale;
+          a = __uint_as_float((__float_as_uint(a) + 2u) & ~3u);   // 22 significant bits
+          a2 = make_float2(a, a);
+          c2 = make_float2(-kMagicF * a, -kMagicF * a);              // exact
+        };
+        if (ok) {
+          if (!mbar_wait(&pfull[pb], pph[pb])) ok = false;
+          else {
+            tc_fence_after();
+            tmem_load_chunks<2>(tmem + lane_base + pb * TT + col0, vX);
+          }
+        }
+        for (int g = 0; g < G && ok; g += 2) {
+          // ------------------------------------------------ segment g (buffer pbA)
+          const int pbA = pb, pbB = pb + 1 == NB ? 0 : pb + 1, pbC = pbB + 1 == NB ? 0 : pbB + 1;
+          const uint32_t tA = tmem + lane_base + pbA * TT + col0;
+          const uint32_t tB = tmem + lane_base + pbB * TT + col0;
+          float2 a2, c2;
+          seg_scale(sw_next, a2, c2);
+          sw_next = __ldg(swrow + g + 1);
+          const float4* sxA = reinterpret_cast<const float4*>(sx_s + g * L.sx_stride + col0);
+          int32_t* dA = DBG ? dbg_base + (int64_t)g * args.M * args.N : nullptr;
+          tmem_wait_ld();
+          tmem_fence_chunks<2>(vX);
+          tmem_load_chunks<2>(tA + 32, vY);
+          promote_g64<0, 2, EC / 2, W4, DBG>(y, vX, sxA, a2, c2, dA, dstride, mrow0, args.M);
+          if (rel >= 0) { release(rel); rel = -1; }
+          tmem_wait_ld();
+          tmem_fence_chunks<2>(vY);
+          tmem_load_chunks<1>(tA + 64, vX);
+          promote_g64<2, 2, EC / 2, W4, DBG>(y, vY, sxA, a2, c2, dA, dstride, mrow0, args.M);
+          tmem_wait_ld();
+          tmem_fence_chunks<1>(vX);
+          pph[pbA] ^= 1;
+          if (!mbar_wait(&pfull[pbB], pph[pbB])) { ok = false; }
+          else {
+            tc_fence_after();
+            tmem_load_chunks<2>(tB, vY);
+          }
+          promote_g64<4, 1, EC / 2, W4, DBG>(y, vX, sxA, a2, c2, dA, dstride, mrow0, args.M);
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) tmem_fill16(tA + 16 * c, kMagicBits);
+          rel = pbA;
+          if (!ok) break;
+          // ------------------------------------------------ segment g+1 (buffer pbB)
+          seg_scale(sw_next, a2, c2);
+          if (g + 2 < G) sw_next = __ldg(swrow + g + 2);
+          const float4* sxB = reinterpret_cast<const float4*>(sx_s + (g + 1) * L.sx_stride + col0);
+          int32_t* dB = DBG ? dbg_base + (int64_t)(g + 1) * args.M * args.N : nullptr;
+          tmem_wait_ld();
+          tmem_fence_chunks<2>(vY);
+          tmem_load_chunks<2>(tB + 32, vX);
+          promote_g64<0, 2, EC / 2, W4, DBG>(y, vY, sxB, a2, c2, dB, dstride, mrow0, args.M);
+          release(rel);
+          rel = -1;
+          tmem_wait_ld();
+          tmem_fence_chunks<2>(vX);
+          tmem_load_chunks<1>(tB + 64, vY);
+          promote_g64<2, 2, EC / 2, W4, DBG>(y, vX, sxB, a2, c2, dB, dstride, mrow0, args.M);
+          tmem_wait_ld();
+          tmem_fence_chunks<1>(vY);
+          pph[pbB] ^= 1;
+          if (g + 2 < G) {
+            if (!mbar_wait(&pfull[pbC], pph[pbC])) { ok = false; }
+            else {
+              tc_fence_after();
+              tmem_load_chunks<2>(tmem + lane_base + pbC * TT + col0, vX);
+            }
+          }
+          promote_g64<4, 1, EC / 2, W4, DBG>(y, vY, sxB, a2, c2, dB, dstride, mrow0, args.M);
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) tmem_fill16(tB + 16 * c, kMagicBits);
+          rel = pbB;
+          pb = pbC;
+        }
+        if (rel >= 0) {
+          tmem_wait_ld();
+          release(rel);
+        }
+      } else {
+        for (int g = 0; g < G && ok; ++g) {
+          const float sw_g = sw_next;
+          if (g + 1 < G) sw_next = __ldg(swrow + g + 1);
+          if (!mbar_wait(&pfull[pb], pph[pb])) { ok = false; break; }
+          pph[pb] ^= 1;
+          tc_fence_after();
+          const uint32_t tbase = tmem + lane_base + pb * TT + col0;
+          const float4* sxg = reinterpret_cast<const float4*>(sx_s + g * L.sx_stride + col0);
+          const float a = sw_g * args.acc_scale;
+          const float2 a2 = make_float2(a, a);
+          {
+            // row scales: one promotion per tile; TMEM loads pipelined two deep
+            uint32_t va[16], vb[16];
+            tmem_ld16_async(tbase, va);
+            tmem_wait_ld();
+            tmem_reg_fence(va);
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+              uint32_t (&v)[16] = (c & 1) ? vb : va;
+              uint32_t (&vn)[16] = (c & 1) ? va : vb;
+              if (c + 1 < NCH) tmem_ld16_async(tbase + 16 * (c + 1), vn);
+              if (DBG) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  const int64_t m = (int64_t)m0 + col0 + 16 * c + j;
+                  if (m < args.M) args.acc_debug[m * args.N + n] = W4 ? ((int32_t)v[j] >> 4) : (int32_t)v[j];
+                }
+              }
+#pragma unroll
+              for (int j4 = 0; j4 < 4; ++j4) {
+                const float4 b4 = sxg[4 * c + j4];
+                const float2 f0 = make_float2((float)(int32_t)v[4 * j4], (float)(int32_t)v[4 * j4 + 1]);
+                const float2 f1 = make_float2((float)(int32_t)v[4 * j4 + 2], (float)(int32_t)v[4 * j4 + 3]);
+                y[8 * c + 2 * j4] = __ffma2_rn(f0, __fmul2_rn(a2, make_float2(b4.x, b4.y)), y[8 * c + 2 * j4]);
+                y[8 * c + 2 * j4 + 1] =
+                    __ffma2_rn(f1, __fmul2_rn(a2, make_float2(b4.z, b4.w)), y[8 * c + 2 * j4 + 1]);
+              }
+              if (c + 1 < NCH) {
+                tmem_wait_ld();
+                tmem_reg_fence(vn);
+              }
             }
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(lrempty);
+          if (lane == 0) mbar_arrive(&pempty[pb]);
+          pb = pb + 1 == NB ? 0 : pb + 1;
         }
-      }
-      for (int g = 0; g < G && ok; ++g) {
-        const float sw_g = sw_next;
-        if (g + 1 < G) sw_next = __ldg(swrow + g + 1);
-        if (!mbar_wait(&pfull[pb], pph[pb])) { ok = false; break; }
-        pph[pb] ^= 1;
-        tc_fence_after();
-        const float4* sxg = reinterpret_cast<const float4*>(sx_s + g * L.sx_stride + 64 * h);
-        float a = sw_g * args.acc_scale;
-        float cneg = 0.f;
-        if (G64) {
-          a = __uint_as_float((__float_as_uint(a) + 2u) & ~3u);   // 22 significant bits
-          cneg = -kMagicF * a;                                       // exact
-        }
-        const float2 a2 = make_float2(a, a);
-        const float2 c2 = make_float2(cneg, cneg);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t v[32];
-          const uint32_t taddr = tmem + lane_base + kColP0 + pb * 128 + 64 * h + 32 * c;
-          tmem_ld32(taddr, v);
-          if (DBG) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int64_t m = (int64_t)m0 + 64 * h + 32 * c + j;
-              if (m < args.M) {
-                const int32_t raw = G64 ? (int32_t)(v[j] - kMagicBits) : (int32_t)v[j];
-                const int32_t accv = W4 ? (raw >> 4) : raw;
-                const int64_t idx = (G64 ? (int64_t)g * args.M * args.N : 0) + m * args.N + n;
-                args.acc_debug[idx] = accv;
-              }
-            }
-          }
-#pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            const float4 b4 = sxg[8 * c + j4];
-            const float2 blo = make_float2(b4.x, b4.y), bhi = make_float2(b4.z, b4.w);
-            float2& y0 = y[16 * c + 2 * j4];
-            float2& y1 = y[16 * c + 2 * j4 + 1];
-            if (G64) {
-              const float2 f0 = make_float2(__uint_as_float(v[4 * j4]), __uint_as_float(v[4 * j4 + 1]));
-              const float2 f1 = make_float2(__uint_as_float(v[4 * j4 + 2]), __uint_as_float(v[4 * j4 + 3]));
-              y0 = __ffma2_rn(__ffma2_rn(f0, a2, c2), blo, y0);
-              y1 = __ffma2_rn(__ffma2_rn(f1, a2, c2), bhi, y1);
-            } else {
-              const float2 f0 = make_float2((float)(int32_t)v[4 * j4], (float)(int32_t)v[4 * j4 + 1]);
-              const float2 f1 = make_float2((float)(int32_t)v[4 * j4 + 2], (float)(int32_t)v[4 * j4 + 3]);
-              y0 = __ffma2_rn(f0, __fmul2_rn(a2, blo), y0);
-              y1 = __ffma2_rn(f1, __fmul2_rn(a2, bhi), y1);
-            }
-          }
-          if (G64) {
-            tmem_fill16(taddr, kMagicBits);
-            tmem_fill16(taddr + 16, kMagicBits);
-          }
-        }
-        if (G64) tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pempty[pb]);
-        pb ^= 1;
       }
       if (!ok) continue;  // keep the named barriers balanced; stop producing output
-      // gate and store: thread (feature n) writes tokens m0 + 64h + j
+
+      // gate and store: thread (feature n) writes tokens m0 + col0 + j
       const bool sig = args.gate_mode == 1 && n >= args.gate_c0 && n < args.gate_c1;
       const float gv = args.gate_mode == 2 ? __uint_as_float((uint32_t)__ldg(args.gate + n) << 16) : 0.f;
-      const int64_t mbase = (int64_t)m0 + 64 * h;
+      const int64_t mbase = (int64_t)m0 + col0;
+      const int64_t rem = (int64_t)args.M - mbase;
+      const int jmax = rem >= EC ? EC : (int)rem;
       uint16_t* yp = args.y + mbase * args.ldy + n;
-      const uint16_t* rp = args.gate_mode == 2 ? args.residual + mbase * args.ldr + n : nullptr;
+      const int64_t ystep = args.ldy;
+      if (args.gate_mode == 2) {
+        const uint16_t* rp = args.residual + mbase * args.ldr + n;
+        const int64_t rstep = args.ldr;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        if (mbase + j < args.M) {
-          float o = (j & 1) ? y[j >> 1].y : y[j >> 1].x;
-          if (sig) {
-            o = 1.0f / (1.0f + __expf(-o));
-          } else if (args.gate_mode == 2) {
-            const float rres = __uint_as_float((uint32_t)rp[(int64_t)j * args.ldr] << 16);
-            o = fmaf(gv, o, rres);
+        for (int j = 0; j < EC; ++j) {
+          if (j < jmax) {
+            const float o = (j & 1) ? y[j >> 1].y : y[j >> 1].x;
+            const float rres = __uint_as_float((uint32_t)*rp << 16);
+            *yp = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(gv, o, rres)));
           }
-          yp[(int64_t)j * args.ldy] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+          yp += ystep;
+          rp += rstep;
+        }
+      } else {
+        // round to bf16 pairs first (halves the live registers), then store
+        uint32_t ob[EC / 2];
+#pragma unroll
+        for (int j2 = 0; j2 < EC / 2; ++j2) {
+          float o0 = y[j2].x, o1 = y[j2].y;
+          if (sig) {
+            o0 = 1.0f / (1.0f + __expf(-o0));
+            o1 = 1.0f / (1.0f + __expf(-o1));
+          }
+          ob[j2] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o0)) |
+                   ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o1)) << 16);
+        }
+#pragma unroll
+        for (int j = 0; j < EC; ++j) {
+          if (j < jmax) *yp = (uint16_t)((j & 1) ? (ob[j >> 1] >> 16) : (ob[j >> 1] & 0xFFFFu));
+          yp += ystep;
         }
       }
     }
@@ -445,20 +667,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // Host launcher
 // ---------------------------------------------------------------------------
+uint32_t gemm_smem_bytes(bool g64, int r, int G) {
+  const int tt = tile_tokens(g64);
+  const int s = pick_stages(r, G, tt);
+  return s ? smem_layout(s, r, G, tt).total : 0xFFFFFFFFu;
+}
+
+int gemm_tile_tokens(bool g64) { return tile_tokens(g64); }
+
+// The warpgroup register split (40 + 88 + 2 x 192 per thread) adds up to the
+// 128 registers per thread the block is launched with; a build that launched
+// with fewer would make setmaxnreg.inc wait forever, so refuse to launch it.
+static bool regs_ok(const void* kern) {
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return false;
+  return fa.numRegs == 128;
+}
+
 cudaError_t launch_lowbit_gemm(bool w4, bool g64, const CUtensorMap& tm_x, const CUtensorMap& tm_w8,
                                const CUtensorMap& tm_ld, const CUtensorMap& tm_l2, const GemmArgs& a, int num_sms,
                                cudaStream_t st) {
   const bool lr = a.r > 0;
-  const SmemLayout L = smem_layout(w4, a.r, a.G);
-  if (L.total > 227u * 1024u) return cudaErrorInvalidConfiguration;
+  const uint32_t smem = gemm_smem_bytes(g64, a.r, a.G);
+  if (smem > 227u * 1024u) return cudaErrorInvalidConfiguration;
   const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
   const bool dbg = a.acc_debug != nullptr;
 #define RBD_GEMM_CASE(W, G, R, D)                                                                     \
   if (w4 == W && g64 == G && lr == R && dbg == D) {                                                  \
     auto kern = lowbit_gemm_kernel<W, G, R, D>;                                                      \
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total); \
+    if (!regs_ok(reinterpret_cast<const void*>(kern))) return cudaErrorInvalidConfiguration;         \
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);    \
     if (e != cudaSuccess) return e;                                                                  \
-    kern<<<grid, kThreads, L.total, st>>>(tm_x, tm_w8, tm_ld, tm_l2, a);                            \
+    kern<<<grid, kThreads, smem, st>>>(tm_x, tm_w8, tm_ld, tm_l2, a);                               \
     return cudaGetLastError();                                                                       \
   }
 #define RBD_GEMM_CASES(W, G, R) RBD_GEMM_CASE(W, G, R, false) RBD_GEMM_CASE(W, G, R, true)
@@ -474,7 +714,5 @@ cudaError_t launch_lowbit_gemm(bool w4, bool g64, const CUtensorMap& tm_x, const
 #undef RBD_GEMM_CASE
   return cudaErrorInvalidValue;
 }
-
-uint32_t gemm_smem_bytes(bool w4, int r, int G) { return smem_layout(w4, r, G).total; }
 
 }  // namespace rbd

@@ -37,6 +37,7 @@ cudaError_t launch_lowbit_gemm(bool w4, bool g64, const CUtensorMap& tm_x, const
                                const CUtensorMap& tm_ld, const CUtensorMap& tm_l2, const GemmArgs& a, int num_sms,
                                cudaStream_t st);
 
-uint32_t gemm_smem_bytes(bool w4, int r, int G);
+uint32_t gemm_smem_bytes(bool g64, int r, int G);   // dynamic shared memory of one GEMM CTA
+int gemm_tile_tokens(bool g64);                     // tokens per GEMM tile
 
 }  // namespace rbd

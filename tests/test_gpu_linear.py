@@ -92,6 +92,16 @@ def test_ragged_tokens_several_tiles(M, bits, sg):
     check_output(y, ref["ref64"], ref["ref_bf16"])
 
 
+@pytest.mark.parametrize("bits,rank", [(8, 0), (4, 32)])
+def test_long_k_group_scales_two_stage_pipeline(bits, rank):
+    # K = 12288 with group scales: the per-tile scale table leaves room for two
+    # pipeline stages only (fewer stages than producer warps)
+    case = build_case(300, 256, 12288, bits, 64, seed=40, rank=rank, bias=True)
+    y, acc, _ = run_layer(case, acc_debug=False)
+    ref = reference(case)
+    check_output(y, ref["ref64"], ref["ref_bf16"])
+
+
 def test_deterministic_run_to_run():
     case = build_case(300, 512, 1024, 4, 64, seed=30, rank=32, bias=True, gate_mode=1, gate_cols=(0, 128))
     y1, _, layer = run_layer(case)
