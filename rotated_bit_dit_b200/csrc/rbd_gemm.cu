@@ -27,22 +27,23 @@
 // scales); the low-rank branch, when present, is one more segment per tile,
 // computed with a bf16 MMA (fp32 result) into the same buffers.
 //   - Row scales: TT = 256, NB = 2.  One promotion per tile.
-//   - Group scales: TT = 160, NB = 3 (3 x 160 columns fit the 512 of TMEM).
+//   - Group scales: TT = 128, NB = 4 (4 x 128 columns fill the 512 of TMEM).
 //     Every 64-wide K block needs its own promotion, so the epilogue is the
-//     busy side: three buffers let the tensor core run two segments ahead, and
-//     with 80 columns per thread all five TMEM loads of a segment are issued
-//     before a single wait.
-// In group mode each partial starts from the bit pattern of 12582912.0f
-// (1.5 * 2^23): the int32 result read as float is then exactly
-// 12582912 + 16*acc, and fma(f, a, -12582912*a) gives the correctly rounded
-// 16*acc*a without an int->float conversion (a is the weight scale rounded to
-// 22 significant bits so that 12582912*a is exact; the relative change of the
-// scale is below 2^-22).
+//     busy side: four buffers let the tensor core run three segments ahead,
+//     and the small tile keeps the epilogue's accumulators and in-flight
+//     TMEM loads in registers (see the group-scale epilogue below).
+// In group mode the epilogue adds the bit pattern of 12582912.0f (1.5 * 2^23)
+// to each int32 partial: read as float the sum is exactly 12582912 + 16*acc,
+// and fma(f, a, -12582912*a) gives the correctly rounded 16*acc*a without an
+// int->float conversion (a is the weight scale rounded to 22 significant bits
+// so that 12582912*a is exact; the relative change of the scale is below
+// 2^-22).
 //
 // Warp roles (16 warps, registers redistributed per warpgroup with setmaxnreg):
 //   warpgroup 0: warps 0, 2, 3 TMA producers, warp 1 TMEM allocator + MMA issuer;
 //   warpgroup 1: INT4 -> INT8 converters (W4A4 only);
-//   warpgroups 2-3: epilogue, thread = one output feature x TT/2 tokens.
+//   warpgroups 2-3: epilogue; row scales: thread = one output feature x TT/2
+//   tokens; group scales: thread = 4 features x 16 tokens.
 #include "rbd_common.cuh"
 #include "rbd_internal.cuh"
 
@@ -62,8 +63,8 @@ constexpr float kMagicF = 12582912.0f;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kWStageBytes = kTileF * kBK;   // 16 KB
 
-__host__ __device__ constexpr int tile_tokens(bool g64) { return g64 ? 160 : 256; }
-__host__ __device__ constexpr int num_bufs(bool g64) { return g64 ? 3 : 2; }
+__host__ __device__ constexpr int tile_tokens(bool g64) { return g64 ? 128 : 256; }
+__host__ __device__ constexpr int num_bufs(bool g64) { return g64 ? 4 : 2; }
 
 __device__ __forceinline__ void named_bar_epi() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -120,48 +121,180 @@ __host__ __device__ inline int pick_stages(int r, int G, int tt) {
   return 0;
 }
 
-// Group-scale promotion of NC 16-column chunks (chunks CB .. CB+NC-1 of this
-// thread's columns) from a register buffer holding magic-biased int32 partials:
-// y += (16*acc*a) * b, with (f - 12582912) * a computed by one fma.
-template <int CB, int NC, int NY, bool W4, bool DBG>
-__device__ __forceinline__ void promote_g64(float2 (&y)[NY], const uint32_t (&v)[2][16], const float4* sxg,
-                                            float2 a2, float2 c2, int32_t* dbg, int64_t dbg_stride,
-                                            int64_t mrow0, int64_t M) {
+// ---------------------------------------------------------------------------
+// Group-scale epilogue (128-token tiles, four TMEM buffers).
+//
+// Thread mapping.  The epilogue warp of lane quarter q and token half h reads
+// TMEM with the 32-lane x 32-bit shape (the fastest TMEM -> register path):
+// thread = one output feature x 64 token columns.  A segment is read in two
+// phases of 32 columns; while one phase is promoted the other is in flight.
+// The activation scales of a column are the same for every lane of the warp,
+// so they are read as shared-memory broadcasts.
+//
+// Each segment's first MMA overwrites its buffer, so TMEM is only read.  The
+// int32 partial v is turned into a float by adding the bit pattern of
+// 12582912.0f (exact: |v| < 2^22) and one fma with -12582912 * a removes the
+// bias while applying the weight scale.
+// ---------------------------------------------------------------------------
+constexpr int kG64Half = 64;   // token columns per epilogue warp
+
+template <int P>
+__device__ __forceinline__ void g64_load_phase(uint32_t tcol, uint32_t (&v)[32]) {
+  tmem_ld16_async(tcol + 32u * P, *reinterpret_cast<uint32_t(*)[16]>(v));
+  tmem_ld16_async(tcol + 32u * P + 16u, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
+}
+
+__device__ __forceinline__ void tmem_reg_fence32(uint32_t (&v)[32]) {
+  tmem_reg_fence(*reinterpret_cast<uint32_t(*)[16]>(v));
+  tmem_reg_fence(*reinterpret_cast<uint32_t(*)[16]>(v + 16));
+}
+
+// y[16 P + j2] += (16*acc*a) * b for the 32 columns of phase P; b4 points at the
+// scales of the phase's first column (broadcast reads).
+template <int P, bool W4, bool DBG>
+__device__ __forceinline__ void g64_promote_phase(float2 (&y)[32], const uint32_t (&v)[32], const float4* b4,
+                                                  float a, float c, int32_t* dbg, int64_t dbg_m0, int64_t M,
+                                                  int64_t N) {
 #pragma unroll
-  for (int c = 0; c < NC; ++c) {
-    if (DBG) {
+  for (int j4 = 0; j4 < 8; ++j4) {
+    const float4 bq = b4[j4];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int64_t m = mrow0 + 16 * (CB + c) + j;
-        if (m < M) {
-          const int32_t raw = (int32_t)(v[c][j] - kMagicBits);
-          dbg[m * dbg_stride] = W4 ? (raw >> 4) : raw;
-        }
+    for (int hh = 0; hh < 2; ++hh) {
+      const int j = 4 * j4 + 2 * hh;
+      const uint32_t u0 = v[j], u1 = v[j + 1];
+      if (DBG) {
+        const int64_t m = dbg_m0 + 32 * P + j;
+        if (m < M) dbg[m * N] = W4 ? ((int32_t)u0 >> 4) : (int32_t)u0;
+        if (m + 1 < M) dbg[(m + 1) * N] = W4 ? ((int32_t)u1 >> 4) : (int32_t)u1;
       }
-    }
-#pragma unroll
-    for (int j4 = 0; j4 < 4; ++j4) {
-      const float4 b4 = sxg[4 * (CB + c) + j4];
-      const float2 f0 = make_float2(__uint_as_float(v[c][4 * j4]), __uint_as_float(v[c][4 * j4 + 1]));
-      const float2 f1 = make_float2(__uint_as_float(v[c][4 * j4 + 2]), __uint_as_float(v[c][4 * j4 + 3]));
-      float2& y0 = y[8 * (CB + c) + 2 * j4];
-      float2& y1 = y[8 * (CB + c) + 2 * j4 + 1];
-      y0 = __ffma2_rn(__ffma2_rn(f0, a2, c2), make_float2(b4.x, b4.y), y0);
-      y1 = __ffma2_rn(__ffma2_rn(f1, a2, c2), make_float2(b4.z, b4.w), y1);
+      const float2 t = make_float2(fmaf(__uint_as_float(u0 + kMagicBits), a, c),
+                                   fmaf(__uint_as_float(u1 + kMagicBits), a, c));
+      const float2 b = hh ? make_float2(bq.z, bq.w) : make_float2(bq.x, bq.y);
+      float2& yy = y[16 * P + j / 2];
+      yy = __ffma2_rn(t, b, yy);
     }
   }
 }
 
-template <int NC>
-__device__ __forceinline__ void tmem_load_chunks(uint32_t taddr, uint32_t (&v)[2][16]) {
+// Low-rank segment (fp32 branch result in TMEM): y += v for phase P.
+template <int P>
+__device__ __forceinline__ void g64_add_phase(float2 (&y)[32], const uint32_t (&v)[32]) {
 #pragma unroll
-  for (int c = 0; c < NC; ++c) tmem_ld16_async(taddr + 16 * c, v[c]);
+  for (int j2 = 0; j2 < 16; ++j2) {
+    y[16 * P + j2].x += __uint_as_float(v[2 * j2]);
+    y[16 * P + j2].y += __uint_as_float(v[2 * j2 + 1]);
+  }
 }
 
-template <int NC>
-__device__ __forceinline__ void tmem_fence_chunks(uint32_t (&v)[2][16]) {
+// One 128 x 128 tile of the group-scale epilogue for this thread (feature n,
+// token columns col0 .. col0+63 of the tile): optional low-rank segment, G
+// promoted segments, gate and store.  tcol = TMEM address of this warp's lane
+// quarter at column col0 of buffer 0; sxc = the scale table at column col0.
+// Returns false if a wait timed out (nothing is stored then).
+template <bool W4, bool LR, bool DBG>
+__device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, uint64_t* pfull, uint64_t* pempty,
+                                         int& pb, uint32_t& pbits, const float* sxc, int sx_stride, int m0, int n,
+                                         int col0, uint32_t lane) {
+  constexpr int TT = 128, NB = 4;
+  const int G = args.G;
+  auto next = [](int b) { return b + 1 == NB ? 0 : b + 1; };
+  auto release = [&](int b) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&pempty[b]);
+  };
+  auto acquire = [&](int b) {
+    if (!mbar_wait(&pfull[b], (pbits >> b) & 1u)) return false;
+    pbits ^= 1u << b;
+    tc_fence_after();
+    return true;
+  };
+
+  float2 y[32];
+  {
+    const float bv = args.bias ? __uint_as_float((uint32_t)__ldg(args.bias + n) << 16) : 0.f;
 #pragma unroll
-  for (int c = 0; c < NC; ++c) tmem_reg_fence(v[c]);
+    for (int j = 0; j < 32; ++j) y[j] = make_float2(bv, bv);
+  }
+
+  if (LR) {
+    if (!acquire(pb)) return false;
+    const uint32_t tb = tcol + pb * TT;
+    uint32_t v[32];
+    g64_load_phase<0>(tb, v); tmem_wait_ld(); tmem_reg_fence32(v); g64_add_phase<0>(y, v);
+    g64_load_phase<1>(tb, v); tmem_wait_ld(); tmem_reg_fence32(v); g64_add_phase<1>(y, v);
+    release(pb);
+    pb = next(pb);
+  }
+
+  // weight scale of this thread's feature, one segment ahead
+  const float* swp = args.sw + (int64_t)n * G;
+  float swn = __ldg(swp);
+  const int64_t dbg_m0 = (int64_t)m0 + col0;
+  int32_t* dbg = DBG ? args.acc_debug + n : nullptr;
+  uint32_t vX[32], vY[32];
+  if (!acquire(pb)) return false;
+  g64_load_phase<0>(tcol + pb * TT, vX);
+  bool ok = true;
+  for (int g = 0; g < G; ++g) {
+    const int pbA = pb, pbB = next(pb);
+    const uint32_t tA = tcol + pbA * TT;
+    const float a = __uint_as_float((__float_as_uint(swn * args.acc_scale) + 2u) & ~3u);   // 22 significant bits
+    const float c = -kMagicF * a;                                                           // exact
+    if (g + 1 < G) swn = __ldg(swp + g + 1);
+    const float4* b4 = reinterpret_cast<const float4*>(sxc + (int64_t)g * sx_stride);
+    int32_t* dg = DBG ? dbg + (int64_t)g * args.M * args.N : nullptr;
+    // phase 0 (columns 0-31) while phase 1 is in flight
+    tmem_wait_ld();
+    tmem_reg_fence32(vX);
+    g64_load_phase<1>(tA, vY);
+    g64_promote_phase<0, W4, DBG>(y, vX, b4, a, c, dg, dbg_m0, args.M, args.N);
+    // phase 1 (columns 32-63) while the next segment's phase 0 is in flight;
+    // the buffer is free as soon as its last load has landed
+    tmem_wait_ld();
+    tmem_reg_fence32(vY);
+    release(pbA);
+    if (g + 1 < G) {
+      if (!acquire(pbB)) ok = false;
+      else g64_load_phase<0>(tcol + pbB * TT, vX);
+    }
+    g64_promote_phase<1, W4, DBG>(y, vY, b4 + 8, a, c, dg, dbg_m0, args.M, args.N);
+    pb = pbB;
+    if (!ok) return false;
+  }
+
+  // gate and store: feature n, tokens m0 + col0 + j (a warp writes 32
+  // consecutive features of one token row per store)
+  const int64_t mbase = (int64_t)m0 + col0;
+  const int64_t rem = (int64_t)args.M - mbase;
+  const int jmax = rem >= kG64Half ? kG64Half : (int)rem;
+  uint16_t* yp = args.y + mbase * args.ldy + n;
+  if (args.gate_mode == 2) {
+    const float gv = __uint_as_float((uint32_t)__ldg(args.gate + n) << 16);
+    const uint16_t* rp = args.residual + mbase * args.ldr + n;
+#pragma unroll
+    for (int j = 0; j < kG64Half; ++j) {
+      if (j < jmax) {
+        const float o = (j & 1) ? y[j >> 1].y : y[j >> 1].x;
+        const float rres = __uint_as_float((uint32_t)*rp << 16);
+        *yp = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(gv, o, rres)));
+      }
+      yp += args.ldy;
+      rp += args.ldr;
+    }
+  } else {
+    const bool sig = args.gate_mode == 1 && n >= args.gate_c0 && n < args.gate_c1;
+#pragma unroll
+    for (int j = 0; j < kG64Half; ++j) {
+      if (j < jmax) {
+        float o = (j & 1) ? y[j >> 1].y : y[j >> 1].x;
+        if (sig) o = 1.0f / (1.0f + __expf(-o));
+        *yp = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+      }
+      yp += args.ldy;
+    }
+  }
+  return true;
 }
 
 template <bool W4, bool G64, bool LR, bool DBG>
@@ -182,8 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = bars;                    // [kMaxStages]
   uint64_t* empty = bars + kMaxStages;      // [kMaxStages]
   uint64_t* pfull = bars + 2 * kMaxStages;  // [NB]
-  uint64_t* pempty = pfull + 3;             // [NB]
-  uint64_t* lrsfull = pempty + 3;
+  uint64_t* pempty = pfull + 4;             // [NB]
+  uint64_t* lrsfull = pempty + 4;
   uint64_t* lrsempty = lrsfull + 1;
   uint64_t* drain = lrsempty + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -222,7 +355,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int K = args.K;
   const int nks = K / kBK;
-  const int seg = args.seg;
 
   if (warp < 4) {
     setmaxnreg_dec<40>();
@@ -239,7 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && pidx < nprod) {
         uint32_t lr_phase = 0;
         bool ok = true;
-        int i = 0;   // stage counter of this CTA
+        int turn = 0, stage = 0;   // round-robin position and pipeline slot of the next stage
+        uint32_t phase = 0;
         for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
           const int mt = t % args.num_m_tiles, nt = t / args.num_m_tiles;
           const int m0 = mt * TT, n0 = nt * kTileF;
@@ -251,14 +384,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(smem + L.l2_off, &tm_l2, lrsfull, 0, n0);
             lr_phase ^= 1;
           }
-          for (int ks = 0; ks < nks; ++ks, ++i) {
-            if (i % nprod != pidx) continue;
-            const int stage = i % S;
-            const uint32_t phase = (uint32_t)(i / S) & 1u;
-            if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
-            mbar_arrive_expect_tx(&full[stage], W4 ? L.x_stage : L.x_stage + kWStageBytes);
-            tma_load_2d(smem + L.x_off + stage * L.x_stage, &tm_x, &full[stage], ks * kBK, m0);
-            if (!W4) tma_load_2d(smem + L.w_off + stage * kWStageBytes, &tm_w8, &full[stage], ks * kBK, n0);
+          for (int ks = 0; ks < nks; ++ks) {
+            const bool mine = turn == pidx;
+            if (++turn == nprod) turn = 0;
+            if (mine) {
+              if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+              mbar_arrive_expect_tx(&full[stage], W4 ? L.x_stage : L.x_stage + kWStageBytes);
+              tma_load_2d(smem + L.x_off + stage * L.x_stage, &tm_x, &full[stage], ks * kBK, m0);
+              if (!W4) tma_load_2d(smem + L.w_off + stage * kWStageBytes, &tm_w8, &full[stage], ks * kBK, n0);
+            }
+            if (++stage == S) { stage = 0; phase ^= 1; }
           }
         }
         if (!ok) {
@@ -269,21 +404,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else {
       // ---------------------------------------------------------- MMA issuer
+      // One thread issues every MMA; the tensor core completes a K=32 step in
+      // about 128 cycles at N=256, so the issue loop is kept free of integer
+      // division and dynamic indexing (segment boundaries are compile-time:
+      // one per tile with row scales, two per stage with group scales).
       if (elect_one()) {
         const uint32_t idesc = idesc_i8(kTileF, TT);
         const uint32_t idesc_lr = idesc_bf16(kTileF, TT);
+        // descriptor address fields are byte offsets >> 4; stage s adds s * stage bytes >> 4
+        const uint64_t bdesc0 = smem_desc_kmajor(smem_u32(smem + L.x_off), 128);
+        const uint64_t adesc0 = smem_desc_kmajor(smem_u32(smem + L.w_off), 128);
         int stage = 0;
         uint32_t phase = 0, lr_phase = 0;
+        uint64_t bdesc = bdesc0, adesc = adesc0;
         int pb = 0;
-        uint32_t pph[NB];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) pph[b] = 0;
+        uint32_t pbits = 0;   // bit b: parity of the next pempty phase of buffer b
         bool ok = true;
         const uint32_t lr_row_bytes = (uint32_t)args.r * 2;
+        auto acquire = [&](int b) {
+          if (!mbar_wait(&pempty[b], (pbits >> b) & 1u)) return false;
+          pbits ^= 1u << b;
+          tc_fence_after();
+          return true;
+        };
+        auto next = [](int b) { return b + 1 == NB ? 0 : b + 1; };
         for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
           if (LR) {
-            if (!mbar_wait(lrsfull, lr_phase) || !mbar_wait(&pempty[pb], pph[pb])) { ok = false; break; }
-            pph[pb] ^= 1;
+            if (!mbar_wait(lrsfull, lr_phase) || !acquire(pb)) { ok = false; break; }
             lr_phase ^= 1;
             tc_fence_after();
             const uint32_t a0 = smem_u32(smem + L.l2_off), b0 = smem_u32(smem + L.ld_off);
@@ -293,30 +440,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_commit(&pfull[pb]);
             tc_commit(lrsempty);
-            pb = pb + 1 == NB ? 0 : pb + 1;
+            pb = next(pb);
           }
-          for (int ks = 0; ks < nks && ok; ++ks) {
+          if (!G64 && !acquire(pb)) { ok = false; break; }
+          for (int ks = 0; ks < nks; ++ks) {
             if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t bdesc = smem_desc_kmajor(smem_u32(smem + L.x_off + stage * L.x_stage), 128);
-            const uint64_t adesc = smem_desc_kmajor(smem_u32(smem + L.w_off + stage * kWStageBytes), 128);
+            if constexpr (G64) {
+              // K columns 0-63 and 64-127 of the stage are two groups, one buffer each
 #pragma unroll
-            for (int kk = 0; kk < kBK / 32; ++kk) {
-              const int kpos = ks * kBK + kk * 32;
-              if (kpos % seg == 0) {
-                if (!mbar_wait(&pempty[pb], pph[pb])) { ok = false; break; }
-                pph[pb] ^= 1;
-                tc_fence_after();
-              }
-              const uint32_t acc = G64 ? 1u : (kpos % seg != 0 ? 1u : 0u);
-              mma_i8_ss(tmem + pb * TT, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc, acc);
-              if ((kpos + 32) % seg == 0) {
+              for (int hg = 0; hg < 2; ++hg) {
+                if (!acquire(pb)) { ok = false; break; }
+                const uint32_t d = tmem + pb * TT;
+                mma_i8_ss(d, adesc + 4 * hg, bdesc + 4 * hg, idesc, 0u);   // overwrite: a new group
+                mma_i8_ss(d, adesc + 4 * hg + 2, bdesc + 4 * hg + 2, idesc, 1u);
                 tc_commit(&pfull[pb]);
-                pb = pb + 1 == NB ? 0 : pb + 1;
+                pb = next(pb);
               }
+              if (!ok) break;
+            } else {
+              const uint32_t d = tmem + pb * TT;
+#pragma unroll
+              for (int kk = 0; kk < kBK / 32; ++kk)
+                mma_i8_ss(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (ks | kk) ? 1u : 0u);
             }
             tc_commit(&empty[stage]);
-            if (++stage == S) { stage = 0; phase ^= 1; }
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1;
+              bdesc = bdesc0;
+              adesc = adesc0;
+            } else {
+              bdesc += L.x_stage >> 4;
+              adesc += kWStageBytes >> 4;
+            }
+          }
+          if (!ok) break;
+          if (!G64) {
+            tc_commit(&pfull[pb]);
+            pb = next(pb);
           }
         }
         // every issued MMA must complete before TMEM can be released
@@ -396,34 +558,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int fr = 32 * q + lane;  // feature row of this thread in the tile
     const uint32_t col0 = EC * h;
 
-    // every partial buffer starts released; in group mode it holds the magic pattern
-    if (G64) {
-      for (int b = 0; b < NB; ++b)
-#pragma unroll
-        for (int c = 0; c < NCH; ++c) tmem_fill16(tmem + lane_base + b * TT + col0 + 16 * c, kMagicBits);
-      tmem_wait_st();
-    }
+    // every partial buffer starts released
     tc_fence_before();
     __syncwarp();
     if (lane == 0)
       for (int b = 0; b < NB; ++b) mbar_arrive(&pempty[b]);
 
     int pb = 0;
-    uint32_t pph[NB];
-#pragma unroll
-    for (int b = 0; b < NB; ++b) pph[b] = 0;
+    uint32_t pbits = 0;   // bit b: parity of the next pfull phase of buffer b
     bool ok = true;
     for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
       const int mt = t % args.num_m_tiles, nt = t / args.num_m_tiles;
       const int m0 = mt * TT, n0 = nt * kTileF;
       // stage the tile's activation scales in shared memory, group-major
       named_bar_epi();
-      for (int e = etid; e < TT * G; e += kEpiThreads) {
-        const int tk = e / G, g = e % G;
-        const int64_t m = (int64_t)m0 + tk;
-        sx_s[g * L.sx_stride + tk] = m < args.M ? __ldg(args.sx + m * G + g) : 0.f;
+      {
+        // warp w stages tokens w, w + 8, ...; its lanes cover the groups
+        const int ew = etid >> 5;
+#pragma unroll 4
+        for (int tk = ew; tk < TT; tk += kEpiThreads / 32) {
+          const int64_t m = (int64_t)m0 + tk;
+          const float* src = args.sx + m * G;
+          for (int g = (int)lane; g < G; g += 32) sx_s[g * L.sx_stride + tk] = m < args.M ? __ldg(src + g) : 0.f;
+        }
       }
       named_bar_epi();
+      if constexpr (G64) {
+        if (ok)
+          ok = g64_tile<W4, LR, DBG>(args, tmem + lane_base + col0, pfull, pempty, pb, pbits, sx_s + col0,
+                                     L.sx_stride, m0, n0 + fr, (int)col0, lane);
+        continue;
+      } else {
 
       const int n = n0 + fr;
       const float* swrow = args.sw + (int64_t)n * G;
@@ -435,9 +600,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (LR && ok) {
         // low-rank segment: fp32 branch result, added once
-        if (!mbar_wait(&pfull[pb], pph[pb])) ok = false;
+        if (!mbar_wait(&pfull[pb], (pbits >> pb) & 1u)) ok = false;
         if (ok) {
-          pph[pb] ^= 1;
+          pbits ^= 1u << pb;
           tc_fence_after();
           const uint32_t tbase = tmem + lane_base + pb * TT + col0;
 #pragma unroll
@@ -450,124 +615,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               y[8 * c + j].y += __uint_as_float(v[2 * j + 1]);
             }
           }
-          if (G64) {
-#pragma unroll
-            for (int c = 0; c < NCH; ++c) tmem_fill16(tbase + 16 * c, kMagicBits);
-            tmem_wait_st();
-          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&pempty[pb]);
           pb = pb + 1 == NB ? 0 : pb + 1;
         }
       }
-      if constexpr (G64) {
-        // Group scales, software-pipelined.  Each segment's five 16-column
-        // chunks are processed in three phases ({0,1}, {2,3}, {4}); while one
-        // phase is promoted the next phase's TMEM load is in flight (two
-        // register buffers, X and Y, used alternately; the segment loop is
-        // unrolled by two so the buffer order stays static -- the number of
-        // 64-wide groups is even because K is a multiple of 128).  A drained
-        // buffer is refilled with the magic pattern and released one phase
-        // later, so the store wait is off the critical path.
-        static_assert(NCH == 5, "group-scale tiles hold five chunks per thread");
-        uint32_t vX[2][16], vY[2][16];
-        int rel = -1;
-        const int64_t dstride = args.N;
-        int32_t* dbg_base = DBG ? args.acc_debug + n : nullptr;
-        const int64_t mrow0 = (int64_t)m0 + col0;
-        auto release = [&](int b) {
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&pempty[b]);
-        };
-        auto seg_scale = [&](float swv, float2& a2, float2& c2) {
-          float a = swv * args.acc_scale;
-          a = __uint_as_float((__float_as_uint(a) + 2u) & ~3u);   // 22 significant bits
-          a2 = make_float2(a, a);
-          c2 = make_float2(-kMagicF * a, -kMagicF * a);              // exact
-        };
-        if (ok) {
-          if (!mbar_wait(&pfull[pb], pph[pb])) ok = false;
-          else {
-            tc_fence_after();
-            tmem_load_chunks<2>(tmem + lane_base + pb * TT + col0, vX);
-          }
-        }
-        for (int g = 0; g < G && ok; g += 2) {
-          // ------------------------------------------------ segment g (buffer pbA)
-          const int pbA = pb, pbB = pb + 1 == NB ? 0 : pb + 1, pbC = pbB + 1 == NB ? 0 : pbB + 1;
-          const uint32_t tA = tmem + lane_base + pbA * TT + col0;
-          const uint32_t tB = tmem + lane_base + pbB * TT + col0;
-          float2 a2, c2;
-          seg_scale(sw_next, a2, c2);
-          sw_next = __ldg(swrow + g + 1);
-          const float4* sxA = reinterpret_cast<const float4*>(sx_s + g * L.sx_stride + col0);
-          int32_t* dA = DBG ? dbg_base + (int64_t)g * args.M * args.N : nullptr;
-          tmem_wait_ld();
-          tmem_fence_chunks<2>(vX);
-          tmem_load_chunks<2>(tA + 32, vY);
-          promote_g64<0, 2, EC / 2, W4, DBG>(y, vX, sxA, a2, c2, dA, dstride, mrow0, args.M);
-          if (rel >= 0) { release(rel); rel = -1; }
-          tmem_wait_ld();
-          tmem_fence_chunks<2>(vY);
-          tmem_load_chunks<1>(tA + 64, vX);
-          promote_g64<2, 2, EC / 2, W4, DBG>(y, vY, sxA, a2, c2, dA, dstride, mrow0, args.M);
-          tmem_wait_ld();
-          tmem_fence_chunks<1>(vX);
-          pph[pbA] ^= 1;
-          if (!mbar_wait(&pfull[pbB], pph[pbB])) { ok = false; }
-          else {
-            tc_fence_after();
-            tmem_load_chunks<2>(tB, vY);
-          }
-          promote_g64<4, 1, EC / 2, W4, DBG>(y, vX, sxA, a2, c2, dA, dstride, mrow0, args.M);
-#pragma unroll
-          for (int c = 0; c < NCH; ++c) tmem_fill16(tA + 16 * c, kMagicBits);
-          rel = pbA;
-          if (!ok) break;
-          // ------------------------------------------------ segment g+1 (buffer pbB)
-          seg_scale(sw_next, a2, c2);
-          if (g + 2 < G) sw_next = __ldg(swrow + g + 2);
-          const float4* sxB = reinterpret_cast<const float4*>(sx_s + (g + 1) * L.sx_stride + col0);
-          int32_t* dB = DBG ? dbg_base + (int64_t)(g + 1) * args.M * args.N : nullptr;
-          tmem_wait_ld();
-          tmem_fence_chunks<2>(vY);
-          tmem_load_chunks<2>(tB + 32, vX);
-          promote_g64<0, 2, EC / 2, W4, DBG>(y, vY, sxB, a2, c2, dB, dstride, mrow0, args.M);
-          release(rel);
-          rel = -1;
-          tmem_wait_ld();
-          tmem_fence_chunks<2>(vX);
-          tmem_load_chunks<1>(tB + 64, vY);
-          promote_g64<2, 2, EC / 2, W4, DBG>(y, vX, sxB, a2, c2, dB, dstride, mrow0, args.M);
-          tmem_wait_ld();
-          tmem_fence_chunks<1>(vY);
-          pph[pbB] ^= 1;
-          if (g + 2 < G) {
-            if (!mbar_wait(&pfull[pbC], pph[pbC])) { ok = false; }
-            else {
-              tc_fence_after();
-              tmem_load_chunks<2>(tmem + lane_base + pbC * TT + col0, vX);
-            }
-          }
-          promote_g64<4, 1, EC / 2, W4, DBG>(y, vY, sxB, a2, c2, dB, dstride, mrow0, args.M);
-#pragma unroll
-          for (int c = 0; c < NCH; ++c) tmem_fill16(tB + 16 * c, kMagicBits);
-          rel = pbB;
-          pb = pbC;
-        }
-        if (rel >= 0) {
-          tmem_wait_ld();
-          release(rel);
-        }
-      } else {
+      {
         for (int g = 0; g < G && ok; ++g) {
           const float sw_g = sw_next;
           if (g + 1 < G) sw_next = __ldg(swrow + g + 1);
-          if (!mbar_wait(&pfull[pb], pph[pb])) { ok = false; break; }
-          pph[pb] ^= 1;
+          if (!mbar_wait(&pfull[pb], (pbits >> pb) & 1u)) { ok = false; break; }
+          pbits ^= 1u << pb;
           tc_fence_after();
           const uint32_t tbase = tmem + lane_base + pb * TT + col0;
           const float4* sxg = reinterpret_cast<const float4*>(sx_s + g * L.sx_stride + col0);
@@ -653,6 +712,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j < jmax) *yp = (uint16_t)((j & 1) ? (ob[j >> 1] >> 16) : (ob[j >> 1] & 0xFFFFu));
           yp += ystep;
         }
+      }
       }
     }
   }
