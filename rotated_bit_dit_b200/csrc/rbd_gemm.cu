@@ -573,13 +573,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // stage the tile's activation scales in shared memory, group-major
       named_bar_epi();
       {
-        // warp w stages tokens w, w + 8, ...; its lanes cover the groups
+        // warp w stages tokens w + 8 i; lane l covers groups g0 + l.  All loads
+        // of a 32-group chunk are issued before the first store, so a chunk
+        // costs one memory latency.
+        constexpr int kTokPerWarp = TT / (kEpiThreads / 32);
         const int ew = etid >> 5;
-#pragma unroll 4
-        for (int tk = ew; tk < TT; tk += kEpiThreads / 32) {
-          const int64_t m = (int64_t)m0 + tk;
-          const float* src = args.sx + m * G;
-          for (int g = (int)lane; g < G; g += 32) sx_s[g * L.sx_stride + tk] = m < args.M ? __ldg(src + g) : 0.f;
+        for (int g0 = 0; g0 < G; g0 += 32) {
+          const int g = g0 + (int)lane;
+          float v[kTokPerWarp];
+#pragma unroll
+          for (int i = 0; i < kTokPerWarp; ++i) {
+            const int64_t m = (int64_t)m0 + ew + 8 * i;
+            v[i] = (g < G && m < args.M) ? __ldg(args.sx + m * G + g) : 0.f;
+          }
+          if (g < G) {
+#pragma unroll
+            for (int i = 0; i < kTokPerWarp; ++i) sx_s[g * L.sx_stride + ew + 8 * i] = v[i];
+          }
         }
       }
       named_bar_epi();
