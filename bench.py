@@ -123,12 +123,16 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(t, cfg, rows_n=1024):
+def cpu_baseline(t, cfg, target_s=10.0):
+    """The oracle timed on a bounded sample of token rows sized to about `target_s` seconds."""
     from oracle import rbd_oracle as O
     wq, sw = O.quantize_weights(t["w"], 4, 256, 64)
     prep = (O.unpack_int4(wq), sw)
+    t0 = time.perf_counter()
+    oracle_sample(t, cfg, prep, np.arange(64))                  # warm, and size the sample
+    per_row = (time.perf_counter() - t0) / 64
+    rows_n = int(min(cfg["M"], max(64, round(target_s / per_row / 64) * 64)))
     rows = np.arange(rows_n)
-    oracle_sample(t, cfg, prep, rows[:8])                       # warm
     t0 = time.perf_counter()
     oracle_sample(t, cfg, prep, rows)
     dt = time.perf_counter() - t0
@@ -165,6 +169,23 @@ def run_reference(args, cfg, t):
             "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "tokens_per_s": rows_n / dt}
     print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- multi-rank host logic
+def max_over_ranks(x: float, device=None) -> float:
+    """The slowest rank's value: every rank calls this with its own number."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, steps: int, units_per_step: float, t_max: float) -> float:
+    """Units all ranks processed divided by the slowest rank's time (weak scaling)."""
+    return world * steps * units_per_step / t_max
 
 
 # ----------------------------------------------------------------------------- GPU leg
@@ -229,15 +250,10 @@ def run_ours(args, cfg, t):
     gemm = [e[1].elapsed_time(e[2]) for e in evs]
     tot = [e[0].elapsed_time(e[2]) for e in evs]
     t_rank = sum(tot) / 1e3           # seconds over K steps, this rank
-    if world > 1:
-        tt = torch.tensor([t_rank], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
-    else:
-        t_max = t_rank
+    t_max = max_over_ranks(t_rank, dev)
     ops_step = 2.0 * M * N * K
-    value = world * args.steps * ops_step / t_max / 1e12
-    tokens_s = world * args.steps * M / t_max
+    value = whole_job_rate(world, args.steps, ops_step, t_max) / 1e12
+    tokens_s = whole_job_rate(world, args.steps, M, t_max)
 
     # ---- end to end through the public layer call with host buffers
     xh = torch.from_numpy(np.ascontiguousarray(t["x"]).view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -257,12 +273,8 @@ def run_ours(args, cfg, t):
         yh.copy_(out, non_blocking=True)
         e2e_ev[i][1].record()
     torch.cuda.synchronize()
-    e2e_t = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / 1e3
-    if world > 1:
-        tt = torch.tensor([e2e_t], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_t = float(tt.item())
-    e2e_value = world * args.steps * ops_step / e2e_t / 1e12
+    e2e_t = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / 1e3, dev)
+    e2e_value = whole_job_rate(world, args.steps, ops_step, e2e_t) / 1e12
 
     if rank == 0:
         peaks, src = load_peaks()
@@ -303,13 +315,39 @@ def run_ours(args, cfg, t):
         dist.destroy_process_group()
 
 
+GEMM_SOURCES = [os.path.join(ROOT, "rotated_bit_dit_b200", "csrc", f)
+                for f in ("rbd_gemm.cu", "rbd_common.cuh", "rbd_internal.cuh")]
+TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "lowbit_gemm_w4a4_qkvg.md")
+
+
+def gemm_source_hash():
+    """First 16 hex digits of the sha256 over the sources the GEMM kernel is built from."""
+    import hashlib
+    h = hashlib.sha256()
+    for p in GEMM_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def _profile_traffic():
-    """DRAM bytes per GEMM launch from the committed ncu summary, when present."""
-    p = os.path.join(ROOT, "profiles", "traffic_w4a4_qkvg.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            return json.load(f).get("dram_bytes_per_launch")
-    return None
+    """DRAM bytes per GEMM launch from the committed ncu summary.  The summary
+    records the hash of the GEMM source it was captured from; a summary of an
+    older kernel gives no figure (null)."""
+    if not os.path.exists(TRAFFIC_SUMMARY):
+        return None
+    fields = {}
+    with open(TRAFFIC_SUMMARY) as f:
+        for ln in f:
+            if ln.startswith("- ") and ":" in ln:
+                k, v = ln[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    if fields.get("source_sha256_16") != gemm_source_hash():
+        return None
+    try:
+        return int(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 def main():
@@ -319,7 +357,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--print-gemm-hash", action="store_true", help="print the GEMM source hash and exit")
     args = ap.parse_args()
+    if args.print_gemm_hash:
+        print(gemm_source_hash())
+        return
+    if args.impl == "reference" and int(os.environ.get("RANK", "0")) != 0:
+        return                      # the oracle arm runs on rank 0 only; other ranks do no work
     from rotated_bit_dit_b200 import inputs as I
     cfg = I.CONFIGS[WORKLOAD]
     t = I.make_layer_inputs(cfg, seed=0)
