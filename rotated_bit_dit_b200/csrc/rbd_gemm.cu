@@ -288,7 +288,7 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
     for (int j = 0; j < kG64Half; ++j) {
       if (j < jmax) {
         float o = (j & 1) ? y[j >> 1].y : y[j >> 1].x;
-        if (sig) o = 1.0f / (1.0f + __expf(-o));
+        if (sig) o = __frcp_rn(1.0f + __expf(-o));
         *yp = __bfloat16_as_ushort(__float2bfloat16_rn(o));
       }
       yp += args.ldy;
@@ -711,8 +711,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j2 = 0; j2 < EC / 2; ++j2) {
           float o0 = y[j2].x, o1 = y[j2].y;
           if (sig) {
-            o0 = 1.0f / (1.0f + __expf(-o0));
-            o1 = 1.0f / (1.0f + __expf(-o1));
+            o0 = __frcp_rn(1.0f + __expf(-o0));
+            o1 = __frcp_rn(1.0f + __expf(-o1));
           }
           ob[j2] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o0)) |
                    ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o1)) << 16);
