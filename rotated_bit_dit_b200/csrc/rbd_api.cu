@@ -44,8 +44,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // Row-major 2D tensor [rows, cols] with row stride `row_bytes`; box = [box_rows, box_cols].
+// Swizzle follows the box's inner size (128/64/32 bytes) unless `plain` asks for
+// an unswizzled row-major box.
 bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint32_t elem_bytes, uint64_t cols,
-                 uint64_t rows, uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows) {
+                 uint64_t rows, uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, bool plain = false) {
   auto fn = encode_fn();
   if (!fn) return false;
   const uint32_t inner_bytes = box_cols * elem_bytes;
@@ -56,6 +58,7 @@ bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uin
     case 32: sw = CU_TENSOR_MAP_SWIZZLE_32B; break;
     default: return false;
   }
+  if (plain) sw = CU_TENSOR_MAP_SWIZZLE_NONE;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_cols, box_rows};
@@ -140,6 +143,9 @@ rbd_status linear_common(const int8_t* codes, const float* sx, const void* w, co
     if (!make_map_2d(&tm_l2, e.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, e.r, N, 2 * e.r, e.r, 128))
       return RBD_ERR_CUDA;
   }
+  CUtensorMap tm_y{};
+  if (g64 && !make_map_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 2 * ldy, 32, 64, true))
+    return RBD_ERR_CUDA;
   GemmArgs a{};
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
@@ -165,7 +171,7 @@ rbd_status linear_common(const int8_t* codes, const float* sx, const void* w, co
   a.num_tiles = a.num_m_tiles * static_cast<int>(N / 128);
   const int sms = num_sms_current();
   if (sms <= 0) return RBD_ERR_CUDA;
-  return cuda_status(rbd::launch_lowbit_gemm(W4, cfg.scale_group == 64, tm_x, tm_w, tm_ld, tm_l2, a, sms,
+  return cuda_status(rbd::launch_lowbit_gemm(W4, cfg.scale_group == 64, tm_x, tm_w, tm_ld, tm_l2, tm_y, a, sms,
                                              as_stream(stream)));
 }
 

@@ -84,9 +84,13 @@ __device__ __forceinline__ void fence_async_smem() {
 }  // namespace
 
 struct SmemLayout {
-  uint32_t x_off, w_off, ld_off, l2_off, sx_off, bar_off, total, x_stage;
+  uint32_t x_off, w_off, ld_off, l2_off, sx_off, out_off, bar_off, total, x_stage;
   int stages, sx_stride;
 };
+
+// Group-scale tiles stage their bf16 output per epilogue warp (32 features x 64
+// tokens, row-major by token) for one bulk tensor store.
+constexpr uint32_t kOutWarpBytes = 32 * 64 * 2;
 
 __host__ __device__ inline SmemLayout smem_layout(int stages, int r, int G, int tt) {
   SmemLayout L{};
@@ -107,6 +111,9 @@ __host__ __device__ inline SmemLayout smem_layout(int stages, int r, int G, int 
   L.sx_stride = tt + 4;
   L.sx_off = off;
   off += (uint32_t)G * L.sx_stride * 4;
+  off = (off + 127u) & ~127u;
+  L.out_off = off;
+  if (tt == tile_tokens(true)) off += 8 * kOutWarpBytes;
   off = (off + 15u) & ~15u;
   L.bar_off = off;
   off += 32 * 8 + 16;
@@ -194,7 +201,7 @@ __device__ __forceinline__ void g64_add_phase(float2 (&y)[32], const uint32_t (&
 template <bool W4, bool LR, bool DBG>
 __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, uint64_t* pfull, uint64_t* pempty,
                                          int& pb, uint32_t& pbits, const float* sxc, int sx_stride, int m0, int n,
-                                         int col0, uint32_t lane) {
+                                         int col0, uint32_t lane, const CUtensorMap* tm_y, uint16_t* sout) {
   constexpr int TT = 128, NB = 4;
   const int G = args.G;
   auto next = [](int b) { return b + 1 == NB ? 0 : b + 1; };
@@ -283,15 +290,24 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
       rp += args.ldr;
     }
   } else {
+    // through shared memory and one bulk tensor store per warp: token row j of
+    // the warp's block holds its 32 features (64 contiguous bytes); rows past M
+    // are clipped by the tensor map.  The previous tile's store must have read
+    // the buffer before it is overwritten.
     const bool sig = args.gate_mode == 1 && n >= args.gate_c0 && n < args.gate_c1;
+    if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
 #pragma unroll
     for (int j = 0; j < kG64Half; ++j) {
-      if (j < jmax) {
-        float o = (j & 1) ? y[j >> 1].y : y[j >> 1].x;
-        if (sig) o = __frcp_rn(1.0f + __expf(-o));
-        *yp = __bfloat16_as_ushort(__float2bfloat16_rn(o));
-      }
-      yp += args.ldy;
+      float o = (j & 1) ? y[j >> 1].y : y[j >> 1].x;
+      if (sig) o = __frcp_rn(1.0f + __expf(-o));
+      sout[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+    }
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tm_y, sout, n - (int)lane, m0 + col0);
+      bulk_commit();
     }
   }
   return true;
@@ -301,7 +317,7 @@ template <bool W4, bool G64, bool LR, bool DBG>
 __global__ void __launch_bounds__(kThreads, 1)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w8,
                        const __grid_constant__ CUtensorMap tm_ld, const __grid_constant__ CUtensorMap tm_l2,
-                       const GemmArgs args) {
+                       const __grid_constant__ CUtensorMap tm_y, const GemmArgs args) {
   constexpr int TT = tile_tokens(G64);
   constexpr int NB = num_bufs(G64);
   constexpr int EC = TT / 2;       // TMEM columns (tokens) per epilogue thread
@@ -343,6 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_ld);
       tma_prefetch_desc(&tm_l2);
     }
+    if (G64) tma_prefetch_desc(&tm_y);
   }
   if (warp == kWarpMma) {
     tmem_alloc(tmem_holder, kTmemCols);
@@ -596,7 +613,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (G64) {
         if (ok)
           ok = g64_tile<W4, LR, DBG>(args, tmem + lane_base + col0, pfull, pempty, pb, pbits, sx_s + col0,
-                                     L.sx_stride, m0, n0 + fr, (int)col0, lane);
+                                     L.sx_stride, m0, n0 + fr, (int)col0, lane, &tm_y,
+                                     reinterpret_cast<uint16_t*>(smem + L.out_off) +
+                                         (warp - kWarpEpi0) * (kOutWarpBytes / 2));
         continue;
       } else {
 
@@ -727,6 +746,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // bulk stores still in flight must complete before the CTA (and its shared memory) goes away
+  if (G64 && warp >= kWarpEpi0 && lane == 0) bulk_wait_all();
   __syncthreads();
   if (warp == kWarpMma) {
     tc_fence_after();
@@ -755,8 +776,8 @@ static bool regs_ok(const void* kern) {
 }
 
 cudaError_t launch_lowbit_gemm(bool w4, bool g64, const CUtensorMap& tm_x, const CUtensorMap& tm_w8,
-                               const CUtensorMap& tm_ld, const CUtensorMap& tm_l2, const GemmArgs& a, int num_sms,
-                               cudaStream_t st) {
+                               const CUtensorMap& tm_ld, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
+                               const GemmArgs& a, int num_sms, cudaStream_t st) {
   const bool lr = a.r > 0;
   const uint32_t smem = gemm_smem_bytes(g64, a.r, a.G);
   if (smem > 227u * 1024u) return cudaErrorInvalidConfiguration;
@@ -768,7 +789,7 @@ cudaError_t launch_lowbit_gemm(bool w4, bool g64, const CUtensorMap& tm_x, const
     if (!regs_ok(reinterpret_cast<const void*>(kern))) return cudaErrorInvalidConfiguration;         \
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);    \
     if (e != cudaSuccess) return e;                                                                  \
-    kern<<<grid, kThreads, smem, st>>>(tm_x, tm_w8, tm_ld, tm_l2, a);                               \
+    kern<<<grid, kThreads, smem, st>>>(tm_x, tm_w8, tm_ld, tm_l2, tm_y, a);                               \
     return cudaGetLastError();                                                                       \
   }
 #define RBD_GEMM_CASES(W, G, R) RBD_GEMM_CASE(W, G, R, false) RBD_GEMM_CASE(W, G, R, true)

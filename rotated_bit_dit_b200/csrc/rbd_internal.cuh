@@ -33,9 +33,10 @@ cudaError_t launch_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ld
                              bool packed, int8_t* codes, float* scales, cudaStream_t st);
 cudaError_t launch_lowrank_down(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const uint16_t* l1t, int r,
                                 uint16_t* ld, cudaStream_t st);
+// tm_y: unswizzled map of Y with 32-feature x 64-token boxes (group-scale tiles store through it)
 cudaError_t launch_lowbit_gemm(bool w4, bool g64, const CUtensorMap& tm_x, const CUtensorMap& tm_w8,
-                               const CUtensorMap& tm_ld, const CUtensorMap& tm_l2, const GemmArgs& a, int num_sms,
-                               cudaStream_t st);
+                               const CUtensorMap& tm_ld, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
+                               const GemmArgs& a, int num_sms, cudaStream_t st);
 
 uint32_t gemm_smem_bytes(bool g64, int r, int G);   // dynamic shared memory of one GEMM CTA
 int gemm_tile_tokens(bool g64);                     // tokens per GEMM tile
