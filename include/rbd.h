@@ -155,6 +155,52 @@ rbd_status rbd_w8a8_linear(const int8_t* codes, const float* sx, const int8_t* w
                            const float* sw, int64_t M, int64_t N, int64_t K, rbd_qcfg cfg,
                            const rbd_epilogue* epi, void* y, int64_t ldy, void* stream);
 
+/* ---- NVFP4 variant ------------------------------------------------------
+ * The same rotated layer with FP4 operands on the block-scaled tensor cores
+ * ("Krea 2 Turbo Nunchaku Lite INT4 r32", Benchmark: the NVFP4 build).  Each
+ * tensor (activations per call, weights once) is quantised in two levels:
+ *   gs = amax(rotated tensor) / (6 * 448)                      float32
+ *   bs = E4M3_RN_satfinite(amax(block of 16) / (6 * gs))       one per 16 elements
+ *   q  = E2M1_RN_satfinite(x / (bs * gs))
+ * (every quotient and product an IEEE float32 operation) and the GEMM computes
+ * y = gs_x * gs_w * sum_k (q_x bs_x)(q_w bs_w) with float32 accumulation.
+ *
+ * Block-scale layout ("tile-interleaved", the layout the MMA's scale operand
+ * is loaded from): rows in tiles of 128, scale columns (one per 16 elements
+ * of K) in steps of 4; byte offset of (row, col) =
+ *   ((row/128 * (K/64) + col/4) * 32 + row%32) * 16 + (row%128)/32 * 4 + col%4.
+ * A buffer holds rbd_nvfp4_scale_bytes(rows, K) bytes (rows rounded up to 128).
+ *
+ * Returns the block-scale buffer size in bytes, or -1 for invalid sizes.      */
+int64_t rbd_nvfp4_scale_bytes(int64_t rows, int64_t K);
+
+/* Rotates (rot_group 256, or 0 for none) and quantises x bf16 [M, ldx] to NVFP4.
+ *   codes        uint8 [M, K/2]: two E2M1 codes per byte, element k (even) in
+ *                the low nibble; 8-byte aligned.
+ *   block_scales uint8, tile-interleaved E4M3 (see above), 16-byte aligned;
+ *                rows past M in the last tile are left untouched.
+ *   tensor_scale one float32 (device): gs.
+ *   work         4 bytes of device scratch holding the running tensor amax
+ *                between the two passes; overwritten, so calls sharing it must
+ *                not run concurrently.
+ *   K % 256 == 0, K <= 16384.  Two passes over x (amax, then quantisation).    */
+rbd_status rbd_nvfp4_quant(const void* x, int64_t M, int64_t K, int64_t ldx, int32_t rot_group,
+                           uint8_t* codes, uint8_t* block_scales, float* tensor_scale,
+                           uint32_t* work, void* stream);
+
+/* NVFP4 linear: y = gs_x gs_w (Q_x . Q_w^T) + epilogue.
+ *   xq uint8 [M, K/2], xbs tile-interleaved scales of the M token rows, xgs the
+ *   activation tensor scale (device float); wq uint8 [N, K/2], wbs, wgs
+ *   likewise for the weights (rbd_nvfp4_quant of W [N, K]).
+ *   K % 256 == 0, N % 128 == 0; all code and scale buffers 16-byte aligned.
+ *   epi: bias and gate modes as for rbd_w4a4_linear; the low-rank branch
+ *   (r != 0) and acc_debug are not supported here (RBD_ERR_UNSUPPORTED).
+ *   y bf16 [M, ldy], ldy >= N, ldy % 8 == 0.                                  */
+rbd_status rbd_nvfp4_linear(const uint8_t* xq, const uint8_t* xbs, const float* xgs,
+                            const uint8_t* wq, const uint8_t* wbs, const float* wgs,
+                            int64_t M, int64_t N, int64_t K, const rbd_epilogue* epi,
+                            void* y, int64_t ldy, void* stream);
+
 /* Synchronises `stream`, then reports the first device-side error recorded
  * since the last rbd_check (RBD_ERR_DEVICE_TIMEOUT) or a CUDA error, and
  * clears the device status word.                                              */

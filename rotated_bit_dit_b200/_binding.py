@@ -19,8 +19,8 @@ STATUS_NAMES = {0: "RBD_OK", 1: "RBD_ERR_INVALID_ARG", 2: "RBD_ERR_UNSUPPORTED",
                 4: "RBD_ERR_CUDA", 5: "RBD_ERR_DEVICE_TIMEOUT"}
 
 EXPORTED = ("rbd_rot_quant_act", "rbd_lowrank_fused", "rbd_pack_weights_int4", "rbd_pack_weights_int8",
-            "rbd_w4a4_linear", "rbd_w8a8_linear", "rbd_check", "rbd_debug_timeout_probe",
-            "rbd_status_string", "rbd_version")
+            "rbd_w4a4_linear", "rbd_w8a8_linear", "rbd_nvfp4_scale_bytes", "rbd_nvfp4_quant",
+            "rbd_nvfp4_linear", "rbd_check", "rbd_debug_timeout_probe", "rbd_status_string", "rbd_version")
 
 
 class RbdError(RuntimeError):
@@ -66,6 +66,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "rbd_pack_weights_int8": [vp, i64, i64, QCfg, vp, vp, vp],
         "rbd_w4a4_linear": [vp, vp, vp, vp, i64, i64, i64, QCfg, ctypes.POINTER(Epilogue), vp, i64, vp],
         "rbd_w8a8_linear": [vp, vp, vp, vp, i64, i64, i64, QCfg, ctypes.POINTER(Epilogue), vp, i64, vp],
+        "rbd_nvfp4_quant": [vp, i64, i64, i64, i32, vp, vp, vp, vp, vp],
+        "rbd_nvfp4_linear": [vp, vp, vp, vp, vp, vp, i64, i64, i64, ctypes.POINTER(Epilogue), vp, i64, vp],
         "rbd_check": [vp],
         "rbd_debug_timeout_probe": [i64, vp],
     }
@@ -73,6 +75,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         f = getattr(lib, name)
         f.argtypes = args
         f.restype = ctypes.c_int
+    lib.rbd_nvfp4_scale_bytes.argtypes = [i64, i64]
+    lib.rbd_nvfp4_scale_bytes.restype = i64
     lib.rbd_status_string.argtypes = [ctypes.c_int]
     lib.rbd_status_string.restype = ctypes.c_char_p
     lib.rbd_version.argtypes = []
@@ -188,6 +192,30 @@ def rbd_w8a8_linear(codes: torch.Tensor, sx: torch.Tensor, w8: torch.Tensor, sw:
     """y bf16 [M, N] = epilogue(dequant(codes @ w8^T))."""
     _linear(load().rbd_w8a8_linear, "rbd_w8a8_linear", codes, sx, w8, sw, y, 8, rot_group,
             scale_group, epi, stream)
+
+
+def rbd_nvfp4_scale_bytes(rows: int, K: int) -> int:
+    """Bytes of a tile-interleaved E4M3 block-scale buffer for `rows` rows of length K."""
+    return int(load().rbd_nvfp4_scale_bytes(rows, K))
+
+
+def rbd_nvfp4_quant(x: torch.Tensor, codes: torch.Tensor, block_scales: torch.Tensor, tensor_scale: torch.Tensor,
+                    work: torch.Tensor, rot_group: int = 256, stream=None) -> None:
+    """x bf16 [M, K] -> codes uint8 [M, K/2] (E2M1 pairs), block_scales uint8 (tile-interleaved E4M3,
+    rbd_nvfp4_scale_bytes(M, K)), tensor_scale float32 [1]; work: 4 bytes of device scratch."""
+    M, K = x.shape
+    _ok(load().rbd_nvfp4_quant(_ptr(x), M, K, _rowstride(x), rot_group, _ptr(codes), _ptr(block_scales),
+                               _ptr(tensor_scale), _ptr(work), _stream(stream)), "rbd_nvfp4_quant")
+
+
+def rbd_nvfp4_linear(xq, xbs, xgs, wq, wbs, wgs, y: torch.Tensor, epi: Optional[Epilogue] = None,
+                     stream=None) -> None:
+    """y bf16 [M, N] = epilogue(gs_x gs_w (Q_x . Q_w^T)) on the block-scaled FP4 tensor cores."""
+    M, K2 = xq.shape
+    N = y.shape[1]
+    e = epi if epi is not None else Epilogue()
+    _ok(load().rbd_nvfp4_linear(_ptr(xq), _ptr(xbs), _ptr(xgs), _ptr(wq), _ptr(wbs), _ptr(wgs), M, N, 2 * K2,
+                                ctypes.byref(e), _ptr(y), _rowstride(y), _stream(stream)), "rbd_nvfp4_linear")
 
 
 def rbd_check(stream=None) -> int:

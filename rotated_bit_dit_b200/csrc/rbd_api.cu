@@ -230,6 +230,78 @@ rbd_status rbd_w8a8_linear(const int8_t* codes, const float* sx, const int8_t* w
   return linear_common<false>(codes, sx, w8, sw, M, N, K, cfg, epi, y, ldy, stream);
 }
 
+int64_t rbd_nvfp4_scale_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K <= 0 || K % 64 != 0) return -1;
+  return (rows + 127) / 128 * 128 * (K / 16);
+}
+
+rbd_status rbd_nvfp4_quant(const void* x, int64_t M, int64_t K, int64_t ldx, int32_t rot_group, uint8_t* codes,
+                           uint8_t* block_scales, float* tensor_scale, uint32_t* work, void* stream) {
+  if (M < 0 || K <= 0) return RBD_ERR_INVALID_ARG;
+  if (rot_group != 256 && rot_group != 0) return RBD_ERR_UNSUPPORTED;
+  if (K % 256 != 0 || K > 16384 || M > (int64_t)INT32_MAX / 2) return RBD_ERR_UNSUPPORTED;
+  if (M == 0) return RBD_OK;
+  if (!x || !codes || !block_scales || !tensor_scale || !work) return RBD_ERR_INVALID_ARG;
+  if (ldx < K) return RBD_ERR_INVALID_ARG;
+  if (!aligned16(x) || (ldx % 8) != 0 || (reinterpret_cast<uintptr_t>(codes) & 7u)) return RBD_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(tensor_scale) & 3u) || (reinterpret_cast<uintptr_t>(work) & 3u))
+    return RBD_ERR_ALIGNMENT;
+  return cuda_status(rbd::launch_nvfp4_quant(static_cast<const uint16_t*>(x), M, K, ldx, rot_group != 0, work, codes,
+                                             block_scales, tensor_scale, as_stream(stream)));
+}
+
+rbd_status rbd_nvfp4_linear(const uint8_t* xq, const uint8_t* xbs, const float* xgs, const uint8_t* wq,
+                            const uint8_t* wbs, const float* wgs, int64_t M, int64_t N, int64_t K,
+                            const rbd_epilogue* epi, void* y, int64_t ldy, void* stream) {
+  if (M < 0 || N <= 0 || K <= 0) return RBD_ERR_INVALID_ARG;
+  if (K % 256 != 0 || N % 128 != 0) return RBD_ERR_UNSUPPORTED;
+  if (M > (int64_t)INT32_MAX / 2 || N > (1 << 24) || K > (1 << 20)) return RBD_ERR_UNSUPPORTED;
+  if (M == 0) return RBD_OK;
+  if (!xq || !xbs || !xgs || !wq || !wbs || !wgs || !y) return RBD_ERR_INVALID_ARG;
+  if (ldy < N) return RBD_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(wq) || !aligned16(xbs) || !aligned16(wbs) || !aligned16(y) || (ldy % 8) != 0)
+    return RBD_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(xgs) & 3u) || (reinterpret_cast<uintptr_t>(wgs) & 3u)) return RBD_ERR_ALIGNMENT;
+  rbd_epilogue e{};
+  if (epi) e = *epi;
+  if (e.r != 0 || e.acc_debug) return RBD_ERR_UNSUPPORTED;
+  if (e.gate_mode < 0 || e.gate_mode > 2) return RBD_ERR_INVALID_ARG;
+  if (e.gate_mode == 1 && (e.gate_col0 < 0 || e.gate_col1 < e.gate_col0 || e.gate_col1 > N))
+    return RBD_ERR_INVALID_ARG;
+  if (e.gate_mode == 2) {
+    if (!e.gate || !e.residual) return RBD_ERR_INVALID_ARG;
+    if (e.ldr < N) return RBD_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(e.residual) & 1u) || (reinterpret_cast<uintptr_t>(e.gate) & 1u))
+      return RBD_ERR_ALIGNMENT;
+  }
+  if (e.bias && (reinterpret_cast<uintptr_t>(e.bias) & 1u)) return RBD_ERR_ALIGNMENT;
+  CUtensorMap tm_x{}, tm_w{};
+  if (!make_map_2d(&tm_x, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, K / 2, 128, 128)) return RBD_ERR_CUDA;
+  if (!make_map_2d(&tm_w, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 128, 128)) return RBD_ERR_CUDA;
+  rbd::NvArgs a{};
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.sfx = xbs;
+  a.sfw = wbs;
+  a.gsx = xgs;
+  a.gsw = wgs;
+  a.bias = static_cast<const uint16_t*>(e.bias);
+  a.gate_mode = e.gate_mode;
+  a.gate_c0 = static_cast<int>(e.gate_col0);
+  a.gate_c1 = static_cast<int>(e.gate_col1);
+  a.gate = static_cast<const uint16_t*>(e.gate);
+  a.residual = static_cast<const uint16_t*>(e.residual);
+  a.ldr = e.ldr;
+  a.y = static_cast<uint16_t*>(y);
+  a.ldy = ldy;
+  a.num_m_tiles = static_cast<int>((M + 127) / 128);
+  a.num_tiles = a.num_m_tiles * static_cast<int>(N / 128);
+  const int sms = num_sms_current();
+  if (sms <= 0) return RBD_ERR_CUDA;
+  return cuda_status(rbd::launch_nvfp4_gemm(tm_x, tm_w, a, sms, as_stream(stream)));
+}
+
 rbd_status rbd_check(void* stream) {
   cudaError_t e = cudaStreamSynchronize(as_stream(stream));
   if (e != cudaSuccess) return RBD_ERR_CUDA;

@@ -38,6 +38,29 @@ cudaError_t launch_lowbit_gemm(bool w4, bool g64, const CUtensorMap& tm_x, const
                                const CUtensorMap& tm_ld, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
                                const GemmArgs& a, int num_sms, cudaStream_t st);
 
+// Arguments of the block-scaled FP4 GEMM.
+struct NvArgs {
+  int M, N, K;
+  const uint8_t* sfx;   // activation E4M3 block scales, tile-interleaved
+  const uint8_t* sfw;   // weight E4M3 block scales, tile-interleaved
+  const float* gsx;     // activation tensor scale (device scalar)
+  const float* gsw;     // weight tensor scale (device scalar)
+  const uint16_t* bias;
+  int gate_mode, gate_c0, gate_c1;
+  const uint16_t* gate;
+  const uint16_t* residual;
+  int64_t ldr;
+  uint16_t* y;
+  int64_t ldy;
+  int num_m_tiles, num_tiles;
+};
+
+cudaError_t launch_nvfp4_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, bool rot, uint32_t* work,
+                               uint8_t* codes, uint8_t* bscale, float* gscale, cudaStream_t st);
+cudaError_t launch_nvfp4_gemm(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const NvArgs& a, int num_sms,
+                              cudaStream_t st);
+uint32_t nvfp4_gemm_smem_bytes();
+
 uint32_t gemm_smem_bytes(bool g64, int r, int G);   // dynamic shared memory of one GEMM CTA
 int gemm_tile_tokens(bool g64);                     // tokens per GEMM tile
 

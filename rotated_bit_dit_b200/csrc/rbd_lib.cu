@@ -4,3 +4,4 @@
 #include "rbd_api.cu"
 #include "rbd_prologue.cu"
 #include "rbd_gemm.cu"
+#include "rbd_nvfp4.cu"

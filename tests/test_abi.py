@@ -15,7 +15,7 @@ HDR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), 
 
 def declared_entry_points():
     text = open(HDR).read()
-    return re.findall(r"^(?:rbd_status|const char\*)\s+(rbd_\w+)\(", text, re.M)
+    return re.findall(r"^(?:rbd_status|const char\*|int64_t)\s+(rbd_\w+)\(", text, re.M)
 
 
 def test_library_loads_and_exports_every_declared_symbol():
@@ -104,3 +104,26 @@ def test_lowrank_and_pack_reject_before_launch():
     assert lib.rbd_pack_weights_int4(FAKE, 4, 256, q(bits=8), FAKE, FAKE, None) == 1
     assert lib.rbd_pack_weights_int8(FAKE, 4, 256, q(bits=4), FAKE, FAKE, None) == 1
     assert lib.rbd_debug_timeout_probe(0, None) == 1
+
+
+def test_nvfp4_validation_without_gpu():
+    lib = R.load()
+    assert lib.rbd_nvfp4_scale_bytes(1, 256) == 128 * 16
+    assert lib.rbd_nvfp4_scale_bytes(129, 512) == 256 * 32
+    assert lib.rbd_nvfp4_scale_bytes(4, 100) == -1
+    null = ctypes.c_void_p(0)
+    # K not a multiple of 256; unsupported rotation group; null output
+    assert lib.rbd_nvfp4_quant(FAKE, 4, 320, 320, 256, FAKE, FAKE, FAKE, FAKE, null) == 2
+    assert lib.rbd_nvfp4_quant(FAKE, 4, 256, 256, 64, FAKE, FAKE, FAKE, FAKE, null) == 2
+    assert lib.rbd_nvfp4_quant(FAKE, 4, 256, 256, 256, null, FAKE, FAKE, FAKE, null) == 1
+    assert lib.rbd_nvfp4_quant(FAKE_MIS, 4, 256, 256, 256, FAKE, FAKE, FAKE, FAKE, null) == 3
+    assert lib.rbd_nvfp4_quant(FAKE, 0, 256, 256, 256, null, null, null, null, null) == 0
+    # linear: N not a multiple of 128, low-rank branch unsupported, misaligned scales
+    e = B.Epilogue()
+    assert lib.rbd_nvfp4_linear(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 256, ctypes.byref(e), FAKE, 64, null) == 2
+    e.r = 16
+    assert lib.rbd_nvfp4_linear(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 128, 256, ctypes.byref(e), FAKE, 128,
+                                null) == 2
+    e.r = 0
+    assert lib.rbd_nvfp4_linear(FAKE, FAKE_MIS, FAKE, FAKE, FAKE, FAKE, 4, 128, 256, ctypes.byref(e), FAKE, 128,
+                                null) == 3
