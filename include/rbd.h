@@ -188,6 +188,22 @@ rbd_status rbd_nvfp4_quant(const void* x, int64_t M, int64_t K, int64_t ldx, int
                            uint8_t* codes, uint8_t* block_scales, float* tensor_scale,
                            uint32_t* work, void* stream);
 
+/* rbd_nvfp4_quant without a caller-provided scratch buffer; the method on the
+ * pages has no counterpart to this call: it only changes where the scratch
+ * lives.  For callers that cannot allocate device memory for the library
+ * (plain C hosts without a device allocator, serving loops that must not
+ * allocate between steps).  The quantiser's one scratch word (the running
+ * tensor amax) lives in a library-owned 256-byte array per device; a call
+ * needing more than that array returns RBD_ERR_UNSUPPORTED.  The first call on
+ * a device looks the array up with cudaGetSymbolAddress (do it before any
+ * stream capture).  The word is cleared at the start of every call.  All calls
+ * on a device share the array, so calls that overlap in time (other streams,
+ * other host threads) race and give wrong results.  Allocates nothing.
+ * Arguments and results as rbd_nvfp4_quant.                                   */
+rbd_status rbd_nvfp4_quant_noalloc(const void* x, int64_t M, int64_t K, int64_t ldx, int32_t rot_group,
+                                   uint8_t* codes, uint8_t* block_scales, float* tensor_scale,
+                                   void* stream);
+
 /* NVFP4 linear: y = gs_x gs_w (Q_x . Q_w^T) + epilogue.
  *   xq uint8 [M, K/2], xbs tile-interleaved scales of the M token rows, xgs the
  *   activation tensor scale (device float); wq uint8 [N, K/2], wbs, wgs

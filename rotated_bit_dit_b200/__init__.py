@@ -24,6 +24,7 @@ from ._binding import (  # noqa: F401
     rbd_w8a8_linear,
     rbd_nvfp4_scale_bytes,
     rbd_nvfp4_quant,
+    rbd_nvfp4_quant_noalloc,
     rbd_nvfp4_linear,
 )
 from .layer import RotatedLowBitLinear  # noqa: F401

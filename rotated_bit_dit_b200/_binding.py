@@ -20,7 +20,7 @@ STATUS_NAMES = {0: "RBD_OK", 1: "RBD_ERR_INVALID_ARG", 2: "RBD_ERR_UNSUPPORTED",
 
 EXPORTED = ("rbd_rot_quant_act", "rbd_lowrank_fused", "rbd_pack_weights_int4", "rbd_pack_weights_int8",
             "rbd_w4a4_linear", "rbd_w8a8_linear", "rbd_nvfp4_scale_bytes", "rbd_nvfp4_quant",
-            "rbd_nvfp4_linear", "rbd_check", "rbd_debug_timeout_probe", "rbd_status_string", "rbd_version")
+            "rbd_nvfp4_quant_noalloc", "rbd_nvfp4_linear", "rbd_check", "rbd_debug_timeout_probe", "rbd_status_string", "rbd_version")
 
 
 class RbdError(RuntimeError):
@@ -67,6 +67,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "rbd_w4a4_linear": [vp, vp, vp, vp, i64, i64, i64, QCfg, ctypes.POINTER(Epilogue), vp, i64, vp],
         "rbd_w8a8_linear": [vp, vp, vp, vp, i64, i64, i64, QCfg, ctypes.POINTER(Epilogue), vp, i64, vp],
         "rbd_nvfp4_quant": [vp, i64, i64, i64, i32, vp, vp, vp, vp, vp],
+        "rbd_nvfp4_quant_noalloc": [vp, i64, i64, i64, i32, vp, vp, vp, vp],
         "rbd_nvfp4_linear": [vp, vp, vp, vp, vp, vp, i64, i64, i64, ctypes.POINTER(Epilogue), vp, i64, vp],
         "rbd_check": [vp],
         "rbd_debug_timeout_probe": [i64, vp],
@@ -206,6 +207,14 @@ def rbd_nvfp4_quant(x: torch.Tensor, codes: torch.Tensor, block_scales: torch.Te
     M, K = x.shape
     _ok(load().rbd_nvfp4_quant(_ptr(x), M, K, _rowstride(x), rot_group, _ptr(codes), _ptr(block_scales),
                                _ptr(tensor_scale), _ptr(work), _stream(stream)), "rbd_nvfp4_quant")
+
+
+def rbd_nvfp4_quant_noalloc(x: torch.Tensor, codes: torch.Tensor, block_scales: torch.Tensor,
+                            tensor_scale: torch.Tensor, rot_group: int = 256, stream=None) -> None:
+    """rbd_nvfp4_quant with its scratch word in library-owned device memory (no scratch argument)."""
+    M, K = x.shape
+    _ok(load().rbd_nvfp4_quant_noalloc(_ptr(x), M, K, _rowstride(x), rot_group, _ptr(codes), _ptr(block_scales),
+                                       _ptr(tensor_scale), _stream(stream)), "rbd_nvfp4_quant_noalloc")
 
 
 def rbd_nvfp4_linear(xq, xbs, xgs, wq, wbs, wgs, y: torch.Tensor, epi: Optional[Epilogue] = None,

@@ -68,6 +68,38 @@ bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uin
   return r == CUDA_SUCCESS;
 }
 
+// ---------------------------------------------------------------------------
+// Library-owned scratch for rbd_nvfp4_quant_noalloc.  Some callers cannot hand
+// the library a scratch buffer: plain C hosts with no device allocator of their
+// own, and serving loops that must not touch an allocator between steps.  For
+// them the NVFP4 quantiser's one scratch word (the running tensor amax between
+// its two passes) lives in this fixed file-scope array instead.  Its size is
+// fixed at build time; calls that would need more are rejected.  Every call
+// clears the word it uses before the first pass, so nothing needs to start at
+// zero.  All calls on a device share the array: calls that overlap in time
+// (concurrent streams, or host threads on the same device) race on it.
+constexpr int kNoallocScratchWords = 64;                    // 256 bytes per device
+constexpr int kNvfp4ScratchWords = 1;                       // what one quantiser call needs
+static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoallocScratchWords];
+
+// Device address of the scratch array for the current device.  The first call
+// on a device resolves it with cudaGetSymbolAddress (a runtime call that should
+// happen before any stream capture); later calls reuse the cached address.
+rbd_status noalloc_scratch(uint32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RBD_ERR_CUDA;
+  static std::mutex mu;
+  static uint32_t* cache[64] = {nullptr};
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RBD_ERR_CUDA;
+    cache[dev] = static_cast<uint32_t*>(p);
+  }
+  *out = cache[dev];
+  return RBD_OK;
+}
+
 int num_sms_current() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -248,6 +280,17 @@ rbd_status rbd_nvfp4_quant(const void* x, int64_t M, int64_t K, int64_t ldx, int
     return RBD_ERR_ALIGNMENT;
   return cuda_status(rbd::launch_nvfp4_quant(static_cast<const uint16_t*>(x), M, K, ldx, rot_group != 0, work, codes,
                                              block_scales, tensor_scale, as_stream(stream)));
+}
+
+rbd_status rbd_nvfp4_quant_noalloc(const void* x, int64_t M, int64_t K, int64_t ldx, int32_t rot_group,
+                                   uint8_t* codes, uint8_t* block_scales, float* tensor_scale, void* stream) {
+  if (kNvfp4ScratchWords > kNoallocScratchWords) return RBD_ERR_UNSUPPORTED;   // scratch request too large
+  if (M <= 0) return rbd_nvfp4_quant(x, M, K, ldx, rot_group, codes, block_scales, tensor_scale, nullptr, stream);
+  if (!x || !codes || !block_scales || !tensor_scale) return RBD_ERR_INVALID_ARG;
+  uint32_t* work = nullptr;
+  const rbd_status s = noalloc_scratch(&work);
+  if (s != RBD_OK) return s;
+  return rbd_nvfp4_quant(x, M, K, ldx, rot_group, codes, block_scales, tensor_scale, work, stream);
 }
 
 rbd_status rbd_nvfp4_linear(const uint8_t* xq, const uint8_t* xbs, const float* xgs, const uint8_t* wq,

@@ -127,3 +127,12 @@ def test_nvfp4_validation_without_gpu():
     e.r = 0
     assert lib.rbd_nvfp4_linear(FAKE, FAKE_MIS, FAKE, FAKE, FAKE, FAKE, 4, 128, 256, ctypes.byref(e), FAKE, 128,
                                 null) == 3
+
+
+def test_nvfp4_noalloc_validation_without_gpu():
+    lib = R.load()
+    null = ctypes.c_void_p(0)
+    assert lib.rbd_nvfp4_quant_noalloc(FAKE, 0, 256, 256, 256, null, null, null, null) == 0
+    assert lib.rbd_nvfp4_quant_noalloc(FAKE, 0, 320, 320, 256, null, null, null, null) == 2
+    assert lib.rbd_nvfp4_quant_noalloc(FAKE, -1, 256, 256, 256, FAKE, FAKE, FAKE, null) == 1
+    assert lib.rbd_nvfp4_quant_noalloc(FAKE, 4, 256, 256, 256, null, FAKE, FAKE, null) == 1
