@@ -330,6 +330,99 @@ def gemm_source_hash():
     return h.hexdigest()[:16]
 
 
+# ----------------------------------------------------------------------------- small-M sweep
+def run_small_m_sweep(args):
+    """K = N = 3072 layer at small token counts (HBM-bound): W4A4 rotated per-row and the NVFP4
+    variant.  Each timed call is a full layer (prologue + GEMM); 128 calls on 128 distinct weight
+    copies (several times L2) are captured in one CUDA graph, so weights stream from HBM and launch
+    gaps do not count.  One JSON line per (format, M)."""
+    import torch
+
+    import rotated_bit_dit_b200 as R
+    from rotated_bit_dit_b200 import _binding as B
+    from rotated_bit_dit_b200 import inputs as I
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    R.load()
+    K = N = 3072
+    copies = 128
+    peaks, src = load_peaks()
+    wb = I.gaussian_bf16(1, (N, K), 0.02)
+    w = torch.from_numpy(np.ascontiguousarray(wb).view(np.int16)).view(torch.bfloat16).to(dev)
+    # W4A4 per-row weights, then NVFP4 weights, each replicated into `copies` distinct buffers
+    wq4 = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    sw4 = torch.empty((N,), dtype=torch.float32, device=dev)
+    B.rbd_pack_weights_int4(w, wq4, sw4, 256, 0)
+    wq4s = [wq4.clone() for _ in range(copies)]
+    sw4s = [sw4.clone() for _ in range(copies)]
+    wqf = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    wbf = torch.empty((B.rbd_nvfp4_scale_bytes(N, K),), dtype=torch.uint8, device=dev)
+    wgf = torch.empty((1,), dtype=torch.float32, device=dev)
+    work = torch.empty((1,), dtype=torch.int32, device=dev)
+    B.rbd_nvfp4_quant(w, wqf, wbf, wgf, work, 256)
+    wqfs = [wqf.clone() for _ in range(copies)]
+    wbfs = [wbf.clone() for _ in range(copies)]
+    torch.cuda.synchronize()
+    for fmt in ("w4a4", "nvfp4"):
+        for M in (1, 16, 64, 256, 1024):
+            xb = I.gaussian_bf16(2 + M, (M, K), 1.0, 0.005, 30.0)
+            x = torch.from_numpy(np.ascontiguousarray(xb).view(np.int16)).view(torch.bfloat16).to(dev)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            if fmt == "w4a4":
+                codes = torch.empty((M, K), dtype=torch.int8, device=dev)
+                sx = torch.empty((M,), dtype=torch.float32, device=dev)
+
+                def call(i):
+                    B.rbd_rot_quant_act(x, codes, sx, 4, 256, 0)
+                    B.rbd_w4a4_linear(codes, sx, wq4s[i], sw4s[i], y, 0, None)
+                wbytes = N * K // 2 + N * 4
+                abytes = M * (2 * K + K + 4 + 2 * N)
+            else:
+                xq = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+                xbs = torch.empty((B.rbd_nvfp4_scale_bytes(M, K),), dtype=torch.uint8, device=dev)
+                xgs = torch.empty((1,), dtype=torch.float32, device=dev)
+
+                def call(i):
+                    B.rbd_nvfp4_quant(x, xq, xbs, xgs, work, 256)
+                    B.rbd_nvfp4_linear(xq, xbs, xgs, wqfs[i], wbfs[i], wgf, y, None)
+                wbytes = N * K // 2 + N * K // 16
+                abytes = M * (2 * K + 2 * K + K // 2 + K // 16 + 2 * N)   # X read twice (two passes)
+            for i in range(3):
+                call(i)
+            torch.cuda.synchronize()
+            assert R.rbd_check() == 0
+            stream = torch.cuda.Stream(device=dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(copies):
+                        call(i)
+            for _ in range(max(args.warmup, 3)):
+                g.replay()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(args.steps):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record()
+                g.replay()
+                b.record()
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b) / 1e3 / copies)
+            assert R.rbd_check() == 0
+            t = statistics.median(ts)
+            gbs = (wbytes + abytes) / t / 1e9
+            print(json.dumps({
+                "sweep": "small-m", "format": fmt, "M": M, "K": K, "N": N, "us_per_layer": t * 1e6,
+                "tokens_per_s": M / t, "tops": 2.0 * M * N * K / t / 1e12, "hbm_gbs": gbs,
+                "hbm_frac": gbs / peaks["hbm_gbs"], "peak_source": f"{src} copy {peaks['hbm_gbs']} GB/s",
+                "algorithmic_bytes": wbytes + abytes,
+                "timing": f"median of {args.steps} replays of a graph of {copies} layer calls on distinct weight copies"}),
+                flush=True)
+            del g
+
+
 def _profile_traffic():
     """DRAM bytes per GEMM launch from the committed ncu summary.  The summary
     records the hash of the GEMM source it was captured from; a summary of an
@@ -358,9 +451,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--print-gemm-hash", action="store_true", help="print the GEMM source hash and exit")
+    ap.add_argument("--sweep", choices=["small-m"], default=None,
+                    help="instead of the headline line, print the small-token-count sweep (one line per case)")
     args = ap.parse_args()
     if args.print_gemm_hash:
         print(gemm_source_hash())
+        return
+    if args.sweep == "small-m":
+        run_small_m_sweep(args)
         return
     if args.impl == "reference" and int(os.environ.get("RANK", "0")) != 0:
         return                      # the oracle arm runs on rank 0 only; other ranks do no work

@@ -197,14 +197,16 @@ __device__ __forceinline__ void g64_add_phase(float2 (&y)[32], const uint32_t (&
 // token columns col0 .. col0+63 of the tile): optional low-rank segment, G
 // promoted segments, gate and store.  tcol = TMEM address of this warp's lane
 // quarter at column col0 of buffer 0; sxc = the scale table at column col0.
-// Returns false if a wait timed out (nothing is stored then).
+// The four buffers are handed over in pairs (pb = pair 0 or 1, buffers 2 pb and
+// 2 pb + 1): the two groups of one 128-wide K stage share a pair, the low-rank
+// segment takes a pair of its own.  Returns false if a wait timed out (nothing
+// is stored then).
 template <bool W4, bool LR, bool DBG>
 __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, uint64_t* pfull, uint64_t* pempty,
                                          int& pb, uint32_t& pbits, const float* sxc, int sx_stride, int m0, int n,
                                          int col0, uint32_t lane, const CUtensorMap* tm_y, uint16_t* sout) {
-  constexpr int TT = 128, NB = 4;
+  constexpr int TT = 128;
   const int G = args.G;
-  auto next = [](int b) { return b + 1 == NB ? 0 : b + 1; };
   auto release = [&](int b) {
     tc_fence_before();
     __syncwarp();
@@ -226,12 +228,12 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
 
   if (LR) {
     if (!acquire(pb)) return false;
-    const uint32_t tb = tcol + pb * TT;
+    const uint32_t tb = tcol + 2 * pb * TT;
     uint32_t v[32];
     g64_load_phase<0>(tb, v); tmem_wait_ld(); tmem_reg_fence32(v); g64_add_phase<0>(y, v);
     g64_load_phase<1>(tb, v); tmem_wait_ld(); tmem_reg_fence32(v); g64_add_phase<1>(y, v);
     release(pb);
-    pb = next(pb);
+    pb ^= 1;
   }
 
   // weight scale of this thread's feature, one segment ahead
@@ -241,11 +243,11 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
   int32_t* dbg = DBG ? args.acc_debug + n : nullptr;
   uint32_t vX[32], vY[32];
   if (!acquire(pb)) return false;
-  g64_load_phase<0>(tcol + pb * TT, vX);
+  g64_load_phase<0>(tcol + 2 * pb * TT, vX);
   bool ok = true;
   for (int g = 0; g < G; ++g) {
-    const int pbA = pb, pbB = next(pb);
-    const uint32_t tA = tcol + pbA * TT;
+    const int odd = g & 1;
+    const uint32_t tA = tcol + (2 * pb + odd) * TT;
     const float a = __uint_as_float((__float_as_uint(swn * args.acc_scale) + 2u) & ~3u);   // 22 significant bits
     const float c = -kMagicF * a;                                                           // exact
     if (g + 1 < G) swn = __ldg(swp + g + 1);
@@ -257,16 +259,20 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
     g64_load_phase<1>(tA, vY);
     g64_promote_phase<0, W4, DBG>(y, vX, b4, a, c, dg, dbg_m0, args.M, args.N);
     // phase 1 (columns 32-63) while the next segment's phase 0 is in flight;
-    // the buffer is free as soon as its last load has landed
+    // a pair is free as soon as the last load of its second buffer has landed
     tmem_wait_ld();
     tmem_reg_fence32(vY);
-    release(pbA);
-    if (g + 1 < G) {
-      if (!acquire(pbB)) ok = false;
-      else g64_load_phase<0>(tcol + pbB * TT, vX);
+    if (!odd) {
+      g64_load_phase<0>(tA + TT, vX);   // second buffer of the same pair
+    } else {
+      release(pb);
+      pb ^= 1;
+      if (g + 1 < G) {
+        if (!acquire(pb)) ok = false;
+        else g64_load_phase<0>(tcol + 2 * pb * TT, vX);
+      }
     }
     g64_promote_phase<1, W4, DBG>(y, vY, b4 + 8, a, c, dg, dbg_m0, args.M, args.N);
-    pb = pbB;
     if (!ok) return false;
   }
 
@@ -447,34 +453,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto next = [](int b) { return b + 1 == NB ? 0 : b + 1; };
         for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
           if (LR) {
+            // group mode: the low-rank segment takes a whole buffer pair (its first buffer)
             if (!mbar_wait(lrsfull, lr_phase) || !acquire(pb)) { ok = false; break; }
             lr_phase ^= 1;
             tc_fence_after();
+            const uint32_t dl = tmem + (G64 ? 2 * pb : pb) * TT;
             const uint32_t a0 = smem_u32(smem + L.l2_off), b0 = smem_u32(smem + L.ld_off);
             for (int kk = 0; kk < args.r / 16; ++kk) {
-              mma_bf16_ss(tmem + pb * TT, smem_desc_kmajor(a0 + kk * 32, lr_row_bytes),
+              mma_bf16_ss(dl, smem_desc_kmajor(a0 + kk * 32, lr_row_bytes),
                           smem_desc_kmajor(b0 + kk * 32, lr_row_bytes), idesc_lr, kk > 0 ? 1u : 0u);
             }
             tc_commit(&pfull[pb]);
             tc_commit(lrsempty);
-            pb = next(pb);
+            pb = G64 ? (pb ^ 1) : next(pb);
           }
           if (!G64 && !acquire(pb)) { ok = false; break; }
           for (int ks = 0; ks < nks; ++ks) {
             if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
             tc_fence_after();
             if constexpr (G64) {
-              // K columns 0-63 and 64-127 of the stage are two groups, one buffer each
+              // K columns 0-63 and 64-127 of the stage are two groups; they fill the two
+              // buffers of pair pb (buffers 2 pb, 2 pb + 1), handed over together
+              if (!acquire(pb)) { ok = false; break; }
 #pragma unroll
               for (int hg = 0; hg < 2; ++hg) {
-                if (!acquire(pb)) { ok = false; break; }
-                const uint32_t d = tmem + pb * TT;
+                const uint32_t d = tmem + (2 * pb + hg) * TT;
                 mma_i8_ss(d, adesc + 4 * hg, bdesc + 4 * hg, idesc, 0u);   // overwrite: a new group
                 mma_i8_ss(d, adesc + 4 * hg + 2, bdesc + 4 * hg + 2, idesc, 1u);
-                tc_commit(&pfull[pb]);
-                pb = next(pb);
               }
-              if (!ok) break;
+              tc_commit(&pfull[pb]);
+              pb ^= 1;
             } else {
               const uint32_t d = tmem + pb * TT;
 #pragma unroll
