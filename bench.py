@@ -423,6 +423,85 @@ def run_small_m_sweep(args):
             del g
 
 
+# ----------------------------------------------------------------------------- 28-block stack
+STACK_LAYERS = (("wq", 3072, 3072), ("wk", 3072, 3072), ("wv", 3072, 3072), ("gate", 3072, 3072),
+                ("wo", 3072, 3072), ("mlp.gate", 3072, 12288), ("mlp.up", 3072, 12288), ("mlp.down", 12288, 3072))
+
+
+def stack_layer_is_int8(block: int, name: str) -> bool:
+    """The 96 protected INT8 layers: every wk and wv, wo of blocks 0-26, mlp.down of blocks 15-27."""
+    return name in ("wk", "wv") or (name == "wo" and block <= 26) or (name == "mlp.down" and block >= 15)
+
+
+def run_stack(args):
+    """Timing of the full 28-block linear stack at M = 16384 tokens: 224 rotated low-bit linears
+    (128 W4A4 per-row, 96 W8A8), each with its own weights and its own rotate/quantise prologue.
+    Inputs are synthetic (N(0,1) with 0.5% outlier channels x30), not chained through the blocks."""
+    import torch
+
+    import rotated_bit_dit_b200 as R
+    from rotated_bit_dit_b200 import _binding as B
+    from rotated_bit_dit_b200 import inputs as I
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    R.load()
+    M, blocks = 16384, 28
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    xs = {}
+    for k in (3072, 12288):
+        xb = I.gaussian_bf16(k, (M, k), 1.0, 0.005, 30.0)
+        xs[k] = torch.from_numpy(np.ascontiguousarray(xb).view(np.int16)).view(torch.bfloat16).to(dev)
+    codes = torch.empty((M, 12288), dtype=torch.int8, device=dev)
+    sx = torch.empty((M,), dtype=torch.float32, device=dev)
+    y = torch.empty((M, 12288), dtype=torch.bfloat16, device=dev)
+    layers, ops, n8 = [], 0.0, 0
+    for b in range(blocks):
+        for name, K, N in STACK_LAYERS:
+            w = (torch.randn((N, K), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+            int8 = stack_layer_is_int8(b, name)
+            wq = torch.empty((N, K) if int8 else (N, K // 2), dtype=torch.int8 if int8 else torch.uint8, device=dev)
+            sw = torch.empty((N,), dtype=torch.float32, device=dev)
+            (B.rbd_pack_weights_int8 if int8 else B.rbd_pack_weights_int4)(w, wq, sw, 256, 0)
+            del w
+            layers.append((int8, K, N, wq, sw))
+            ops += 2.0 * M * N * K
+            n8 += int8
+    torch.cuda.synchronize()
+
+    def stack():
+        for int8, K, N, wq, sw in layers:
+            c = codes.view(-1)[:M * K].view(M, K)          # contiguous [M, K]
+            out = y.view(-1)[:M * N].view(M, N)
+            B.rbd_rot_quant_act(xs[K], c, sx, 8 if int8 else 4, 256, 0)
+            (B.rbd_w8a8_linear if int8 else B.rbd_w4a4_linear)(c, sx, wq, sw, out, 0, None)
+
+    for _ in range(max(args.warmup, 1)):
+        stack()
+    torch.cuda.synchronize()
+    assert R.rbd_check() == 0
+    ts = []
+    with ClockSampler(dev.index) as clk:
+        for _ in range(args.steps):
+            a = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            a.record()
+            stack()
+            e.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(e) / 1e3)
+    assert R.rbd_check() == 0
+    t = statistics.median(ts)
+    peaks, src = load_peaks()
+    print(json.dumps({
+        "sweep": "stack", "blocks": blocks, "linears": len(layers), "int8_linears": n8, "M": M,
+        "ms_per_stack": t * 1e3, "tokens_per_s": M / t, "tops": ops / t / 1e12,
+        "pct_int8_peak": 100.0 * ops / t / 1e12 / (2.0 * peaks["bf16_tflops"]), "total_top": ops / 1e12,
+        "timing": f"median of {args.steps} stacks after {max(args.warmup, 1)} warm-up stacks",
+        "clocks": clk.summary()}), flush=True)
+
+
 def _profile_traffic():
     """DRAM bytes per GEMM launch from the committed ncu summary.  The summary
     records the hash of the GEMM source it was captured from; a summary of an
@@ -451,7 +530,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--print-gemm-hash", action="store_true", help="print the GEMM source hash and exit")
-    ap.add_argument("--sweep", choices=["small-m"], default=None,
+    ap.add_argument("--sweep", choices=["small-m", "stack"], default=None,
                     help="instead of the headline line, print the small-token-count sweep (one line per case)")
     args = ap.parse_args()
     if args.print_gemm_hash:
@@ -459,6 +538,9 @@ def main():
         return
     if args.sweep == "small-m":
         run_small_m_sweep(args)
+        return
+    if args.sweep == "stack":
+        run_stack(args)
         return
     if args.impl == "reference" and int(os.environ.get("RANK", "0")) != 0:
         return                      # the oracle arm runs on rank 0 only; other ranks do no work
