@@ -85,7 +85,10 @@ rbd_status rbd_rot_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, r
  *   l1t     bf16 [r, K] row-major: L1 stored output-major, which is the
  *           nn.Linear weight layout of the down projection.  r in {16, 32, 64}.
  *   ld      bf16 [M, r] row-major (float32 accumulation, rounded once).
- * Enqueues two kernels (rotate/quantise, then the down product).             */
+ * With group-64 scales (cfg.scale_group == 64) one kernel reads X once and
+ * writes codes, scales and ld; with row scales it enqueues two kernels
+ * (rotate/quantise, then the down product).  Codes and scales are identical
+ * to rbd_rot_quant_act's in both cases.                                     */
 rbd_status rbd_lowrank_fused(const void* x, int64_t M, int64_t K, int64_t ldx, rbd_qcfg cfg,
                              int8_t* codes, float* scales, const void* l1t, int32_t r, void* ld,
                              void* stream);

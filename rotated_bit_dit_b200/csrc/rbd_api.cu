@@ -113,8 +113,8 @@ int num_sms_current() {
   return n;
 }
 
-rbd_status quant_common(const void* x, int64_t M, int64_t K, int64_t ld, rbd_qcfg cfg, void* out, float* scales,
-                        bool packed, void* stream) {
+rbd_status quant_validate(const void* x, int64_t M, int64_t K, int64_t ld, rbd_qcfg cfg, const void* out,
+                          const float* scales) {
   if (M < 0) return RBD_ERR_INVALID_ARG;
   rbd_status s = check_qcfg(cfg, K);
   if (s != RBD_OK) return s;
@@ -123,6 +123,13 @@ rbd_status quant_common(const void* x, int64_t M, int64_t K, int64_t ld, rbd_qcf
   if (ld < K) return RBD_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(out) || (ld % 8) != 0) return RBD_ERR_ALIGNMENT;
   if (reinterpret_cast<uintptr_t>(scales) & 3u) return RBD_ERR_ALIGNMENT;
+  return RBD_OK;
+}
+
+rbd_status quant_common(const void* x, int64_t M, int64_t K, int64_t ld, rbd_qcfg cfg, void* out, float* scales,
+                        bool packed, void* stream) {
+  rbd_status s = quant_validate(x, M, K, ld, cfg, out, scales);
+  if (s != RBD_OK || M == 0) return s;
   return cuda_status(rbd::launch_rot_quant(static_cast<const uint16_t*>(x), M, K, ld, cfg.bits, cfg.rot_group != 0,
                                            cfg.scale_group == 64, packed, static_cast<int8_t*>(out), scales,
                                            as_stream(stream)));
@@ -231,8 +238,16 @@ rbd_status rbd_lowrank_fused(const void* x, int64_t M, int64_t K, int64_t ldx, r
   if (r != 16 && r != 32 && r != 64) return RBD_ERR_UNSUPPORTED;
   if (M > 0 && (!l1t || !ld)) return RBD_ERR_INVALID_ARG;
   if (M > 0 && (!aligned16(l1t) || !aligned16(ld))) return RBD_ERR_ALIGNMENT;
-  rbd_status s = quant_common(x, M, K, ldx, cfg, codes, scales, false, stream);
+  rbd_status s = quant_validate(x, M, K, ldx, cfg, codes, scales);
   if (s != RBD_OK || M == 0) return s;
+  if (cfg.scale_group == 64) {
+    // group scales: one pass over X yields codes, scales and the down product
+    return cuda_status(rbd::launch_rot_quant_lowrank(static_cast<const uint16_t*>(x), M, K, ldx, cfg.bits,
+                                                     cfg.rot_group != 0, static_cast<const uint16_t*>(l1t), r,
+                                                     codes, scales, static_cast<uint16_t*>(ld), as_stream(stream)));
+  }
+  s = quant_common(x, M, K, ldx, cfg, codes, scales, false, stream);
+  if (s != RBD_OK) return s;
   return cuda_status(rbd::launch_lowrank_down(static_cast<const uint16_t*>(x), M, K, ldx,
                                               static_cast<const uint16_t*>(l1t), r, static_cast<uint16_t*>(ld),
                                               as_stream(stream)));

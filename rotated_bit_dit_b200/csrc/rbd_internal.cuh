@@ -31,6 +31,10 @@ struct GemmArgs {
 
 cudaError_t launch_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot, bool g64,
                              bool packed, int8_t* codes, float* scales, cudaStream_t st);
+// Group-scale prologue and low-rank down product in one pass over X.
+cudaError_t launch_rot_quant_lowrank(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot,
+                                     const uint16_t* l1t, int r, int8_t* codes, float* scales, uint16_t* ld,
+                                     cudaStream_t st);
 cudaError_t launch_lowrank_down(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const uint16_t* l1t, int r,
                                 uint16_t* ld, cudaStream_t st);
 // tm_y: unswizzled map of Y with 32-feature x 64-token boxes (group-scale tiles store through it)

@@ -261,6 +261,181 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_down_kernel(const uint1
 }
 
 // ---------------------------------------------------------------------------
+// Single-pass group-scale prologue: rotated group-64 codes and scales plus the
+// low-rank down product from one read of X.
+//
+// One CTA = 16 tokens = 16 teams; the CTA walks the 256-blocks of its rows in
+// order.  For block g every team loads its token's 256 bf16 values (thread tau:
+// elements 16 tau .. 16 tau + 15, prefetched two blocks ahead), copies them to
+// a shared-memory slab [16 tokens][256], and rotates/quantises them exactly as
+// rot_quant_kernel does (same float64 rotation, same scale and rounding
+// operations, so codes and scales are identical).  After one barrier the eight
+// warps run the low-rank MMAs on the slab: warp w owns k-steps 2w and 2w + 1
+// of every block (m16n8k16, bf16 in, fp32 accumulate, A fragments by ldmatrix,
+// B fragments from l1t), and at the end the eight partial sums are added in a
+// fixed order (deterministic) and rounded to bf16 once.
+// The slab is double-buffered, so one barrier per block suffices: a warp that
+// reaches block g + 1's barrier has finished block g's MMAs.
+// ---------------------------------------------------------------------------
+constexpr int kFuseTok = 16;     // tokens per CTA (one team each)
+constexpr int kSlabPitch = 264;  // bf16 per slab row: 256 + 8 (conflict-free ldmatrix rows)
+constexpr size_t kFuseXbufBytes = (size_t)kFuseTok * 256 * sizeof(double);
+constexpr size_t kFuseSlabBytes = 2 * (size_t)kFuseTok * kSlabPitch * sizeof(uint16_t);
+
+__host__ __device__ constexpr size_t fuse_smem_bytes(int r) {
+  const size_t main = kFuseXbufBytes + kFuseSlabBytes;
+  const size_t red = (size_t)kLrWarps * kFuseTok * (r + 1) * sizeof(float);
+  return main > red ? main : red;
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&a)[4], const uint16_t* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <bool ROT, int R>
+__global__ void __launch_bounds__(kLrWarps * 32, R <= 32 ? 3 : 2)
+    rot_quant_lowrank_kernel(const uint16_t* __restrict__ x, int64_t M, int K, int64_t ldx, float qmax,
+                             const uint16_t* __restrict__ l1t, int8_t* __restrict__ codes,
+                             float* __restrict__ scales, uint16_t* __restrict__ ld) {
+  constexpr int NT = R / 8;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* xbuf = reinterpret_cast<double*>(smem_raw);
+  uint16_t* slab = reinterpret_cast<uint16_t*>(smem_raw + kFuseXbufBytes);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int team = tid >> 4, tau = tid & 15;
+  const int64_t m0 = (int64_t)blockIdx.x * kFuseTok;
+  const int64_t m = m0 + team;
+  const bool row_ok = m < M;
+  const int G = K >> 8;
+  double* tb = xbuf + team * 256;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (row_ok ? m : 0) * ldx + tau * 16);
+  auto fetch = [&](uint4 (&r)[2], int g) {
+    if (row_ok) {
+      r[0] = __ldg(src + g * 32);
+      r[1] = __ldg(src + g * 32 + 1);
+    } else {
+      r[0] = make_uint4(0, 0, 0, 0);
+      r[1] = make_uint4(0, 0, 0, 0);
+    }
+  };
+  const int g4 = lane >> 2, c4 = lane & 3;
+  float acc[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  uint4 cur[2], nxt[2];
+  fetch(cur, 0);
+  if (G > 1) fetch(nxt, 1);
+  for (int g = 0; g < G; ++g) {
+    const uint4 lo = cur[0], hi = cur[1];
+    cur[0] = nxt[0];
+    cur[1] = nxt[1];
+    if (g + 2 < G) fetch(nxt, g + 2);
+    uint16_t* sb = slab + (g & 1) * kFuseTok * kSlabPitch;
+    *reinterpret_cast<uint4*>(sb + team * kSlabPitch + tau * 16) = lo;
+    *reinterpret_cast<uint4*>(sb + team * kSlabPitch + tau * 16 + 8) = hi;
+
+    // ---- rotate, group-64 scales, quantise (register i = position tau + 16 i
+    // with the rotation, 16 tau + i without)
+    float xr[16];
+    if constexpr (ROT) {
+      rotate256_team(lo, hi, tau, tb, xr);
+    } else {
+      load16_f32(lo, hi, xr);
+    }
+    float inv_g[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      float am = 0.f;
+      if constexpr (ROT) {
+#pragma unroll
+        for (int i = 4 * a; i < 4 * a + 4; ++i) am = fmaxf(am, fabsf(xr[i]));
+        for (int off = 8; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(xr[i]));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+        am = __shfl_sync(0xffffffffu, am, (lane & 16) + 4 * a);
+      }
+      inv_g[a] = am > 0.f ? __fdiv_rn(qmax, am) : 0.f;
+      if (row_ok && tau == a) scales[m * (K / 64) + g * 4 + a] = __fdiv_rn(am, qmax);
+    }
+    uint32_t w[4];
+    if constexpr (ROT) {
+      unsigned char* cb = reinterpret_cast<unsigned char*>(tb);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        cb[tau + 16 * i] = static_cast<unsigned char>(static_cast<int8_t>(quant1(xr[i], inv_g[i >> 2], qmax)));
+      __syncwarp();
+      const uint4 q4 = *reinterpret_cast<const uint4*>(cb + 16 * tau);
+      __syncwarp();
+      w[0] = q4.x; w[1] = q4.y; w[2] = q4.z; w[3] = q4.w;
+    } else {
+#pragma unroll
+      for (int wv = 0; wv < 4; ++wv) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          word |= (static_cast<uint32_t>(quant1(xr[4 * wv + b], inv_g[tau >> 2], qmax)) & 0xFFu) << (8 * b);
+        w[wv] = word;
+      }
+    }
+    if (row_ok)
+      *reinterpret_cast<uint4*>(codes + m * (int64_t)K + (int64_t)g * 256 + tau * 16) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+
+    // ---- low-rank MMAs on the slab
+    __syncthreads();
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int kk = (2 * warp + s) * 16;
+      uint32_t a[4];
+      ldmatrix_x4(a, sb + (lane & 15) * kSlabPitch + kk + (lane >> 4) * 8);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const uint32_t* lb =
+            reinterpret_cast<const uint32_t*>(l1t + (int64_t)(n * 8 + g4) * K + (int64_t)g * 256 + kk);
+        mma_bf16_16816(acc[n], a, __ldg(lb + c4), __ldg(lb + c4 + 4));
+      }
+    }
+  }
+
+  // ---- fixed-order reduction of the eight warps' partial sums
+  __syncthreads();
+  float* part = reinterpret_cast<float*>(smem_raw);   // [8 warps][16 tokens][R + 1]
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    float* p0 = part + ((size_t)warp * kFuseTok + g4) * (R + 1) + n * 8 + 2 * c4;
+    float* p1 = p0 + 8 * (R + 1);
+    p0[0] = acc[n][0];
+    p0[1] = acc[n][1];
+    p1[0] = acc[n][2];
+    p1[1] = acc[n][3];
+  }
+  __syncthreads();
+  for (int i = tid; i < kFuseTok * R; i += blockDim.x) {
+    const int rr = i / R, cc = i % R;
+    const int64_t mm = m0 + rr;
+    if (mm < M) {
+      float s = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < kLrWarps; ++w2) s += part[((size_t)w2 * kFuseTok + rr) * (R + 1) + cc];
+      ld[mm * R + cc] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
 namespace {
@@ -346,6 +521,39 @@ cudaError_t launch_lowrank_down(const uint16_t* x, int64_t M, int64_t K, int64_t
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+cudaError_t launch_rot_quant_lowrank(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot,
+                                     const uint16_t* l1t, int r, int8_t* codes, float* scales, uint16_t* ld,
+                                     cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  const dim3 grid(static_cast<unsigned>((M + kFuseTok - 1) / kFuseTok));
+  const float qmax = bits == 4 ? 7.f : 127.f;
+  const int Ki = static_cast<int>(K);
+#define RBD_RQL_CASE(ROT_, R_)                                                                          \
+  {                                                                                                     \
+    auto kern = rot_quant_lowrank_kernel<ROT_, R_>;                                                     \
+    const size_t smem = fuse_smem_bytes(R_);                                                            \
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    if (e != cudaSuccess) return e;                                                                     \
+    kern<<<grid, kLrWarps * 32, smem, st>>>(x, M, Ki, ldx, qmax, l1t, codes, scales, ld);               \
+    return cudaGetLastError();                                                                          \
+  }
+  if (rot) {
+    switch (r) {
+      case 16: RBD_RQL_CASE(true, 16)
+      case 32: RBD_RQL_CASE(true, 32)
+      case 64: RBD_RQL_CASE(true, 64)
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  switch (r) {
+    case 16: RBD_RQL_CASE(false, 16)
+    case 32: RBD_RQL_CASE(false, 32)
+    case 64: RBD_RQL_CASE(false, 64)
+    default: return cudaErrorInvalidValue;
+  }
+#undef RBD_RQL_CASE
 }
 
 }  // namespace rbd

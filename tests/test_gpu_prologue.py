@@ -118,6 +118,53 @@ def test_lowrank_fused(r, M):
     assert np.all(err <= np.abs(ref_ld) * 2.0 ** -8 + 1e-4 * np.abs(ref_ld).max())
 
 
+@pytest.mark.parametrize("M,K,bits,rot,r", [
+    (3, 256, 4, 256, 32),      # one 256-block (no prefetch beyond the first)
+    (17, 768, 8, 256, 16),     # ragged token tile, INT8 codes
+    (33, 12288, 4, 0, 64),     # no rotation, long rows
+    (16, 16384, 8, 0, 32),     # K at the supported maximum
+    (200, 3072, 4, 256, 64),
+])
+def test_lowrank_fused_shapes(M, K, bits, rot, r):
+    # group-scale prologue in one pass: codes and scales bit-exact, the down
+    # product within the float32-accumulation bound
+    xb = I.gaussian_bf16(16 + M + K, (M, K), 1.0, 0.005, 30.0)
+    l1b = I.gaussian_bf16(17 + r, (K, r), 0.01)
+    x, l1t = dev_bf16(xb), dev_bf16(np.ascontiguousarray(l1b.T))
+    codes = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    scales = torch.empty((M, K // 64), dtype=torch.float32, device="cuda")
+    ld = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    R.rbd_lowrank_fused(x, codes, scales, l1t, ld, bits, rot, 64)
+    assert R.rbd_check() == 0
+    ref_q, ref_s = O.rot_quant(xb, bits, rot, 64)
+    assert np.array_equal(codes.cpu().numpy(), ref_q)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ref_s.view(np.uint32))
+    ref_ld = O.lowrank_down(xb, l1b)
+    err = np.abs(ld.float().cpu().numpy().astype(np.float64) - ref_ld)
+    assert np.all(err <= np.abs(ref_ld) * 2.0 ** -8 + 1e-4 * np.abs(ref_ld).max())
+
+
+def test_lowrank_fused_strided_input_and_row_scales():
+    # a row stride larger than K, and the row-scale configuration (two kernels)
+    M, K, ldx, r = 21, 1024, 1536, 32
+    full = I.gaussian_bf16(18, (M, ldx), 1.0, 0.01, 20.0)
+    l1b = I.gaussian_bf16(19, (K, r), 0.01)
+    x, l1t = dev_bf16(full)[:, :K], dev_bf16(np.ascontiguousarray(l1b.T))
+    xb = np.ascontiguousarray(full[:, :K])
+    for sg in (64, 0):
+        codes = torch.empty((M, K), dtype=torch.int8, device="cuda")
+        scales = torch.empty((M, K // 64) if sg else (M,), dtype=torch.float32, device="cuda")
+        ld = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+        R.rbd_lowrank_fused(x, codes, scales, l1t, ld, 4, 256, sg)
+        assert R.rbd_check() == 0
+        ref_q, ref_s = O.rot_quant(xb, 4, 256, sg)
+        assert np.array_equal(codes.cpu().numpy(), ref_q)
+        assert np.array_equal(scales.cpu().numpy().view(np.uint32), ref_s.view(np.uint32))
+        ref_ld = O.lowrank_down(xb, l1b)
+        err = np.abs(ld.float().cpu().numpy().astype(np.float64) - ref_ld)
+        assert np.all(err <= np.abs(ref_ld) * 2.0 ** -8 + 1e-4 * np.abs(ref_ld).max())
+
+
 def test_device_timeout_is_reported_and_context_survives():
     R.rbd_debug_timeout_probe(50_000_000)          # 50 ms bound on a wait nobody satisfies
     assert R.rbd_check() == 5                       # RBD_ERR_DEVICE_TIMEOUT
