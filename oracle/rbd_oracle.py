@@ -33,11 +33,15 @@ What it computes (plain, slow, float64 unless a step fixes the precision):
 6. NVFP4 variant: E2M1 codes with an E4M3 scale per 16 elements and a float32
    tensor scale.  Source: Nunchaku Lite INT4 r32 card, "Benchmark" (NVFP4 build
    on native FP4 tensor cores).
+7. Normalising prologue: RMSNorm and adaLN-style modulation ahead of the
+   rotation.  Source: OrbitQuant W4A4 card, "Fused transformer" (the RMSNorm
+   and modulation run in the activation quantisation prologues).
 
 Readings of points the pages leave open are listed where they are used.
 """
 from __future__ import annotations
 
+import math
 from fractions import Fraction
 
 import numpy as np
@@ -246,6 +250,50 @@ def rot_quant(x_bits: np.ndarray, bits: int, rot_group: int = GROUP, scale_group
     """The activation path: bf16 x [M,K] -> (codes int8 [M,K], scales)."""
     xr = rotate(bf16_to_f64(x_bits), rot_group)
     return quantize(xr, bits, scale_group)
+
+
+def norm_modulate(x_bits: np.ndarray, gamma_bits=None, shift_bits=None, scale_bits=None,
+                  eps: float = 1e-6) -> np.ndarray:
+    """RMSNorm and adaLN-style modulation of bf16 rows, returned as bf16 patterns.
+
+    Source: Krea 2 Turbo OrbitQuant W4A4, "Fused transformer": the RMSNorm and
+    the modulation run in the activation quantisation prologues.  The pages
+    print no formula; the readings (plainest ones) are:
+      - RMS over the whole row: S = sum_k x_k^2 (exact, rounded once to
+        float64), ms = S / K, d = ms + eps, r = 1 / sqrt(d), all float64 IEEE
+        operations; r is rounded once to float32.  A row with d == 0 gets r = 0.
+      - per element, single IEEE float32 operations in this order:
+        u = x * r;  u = u * gamma (when given);  v = u * (1 + scale);
+        v = v + shift;  gamma, shift, scale are bf16 [K] vectors (batch 1: one
+        modulation vector per call), 1 + scale rounded to float32 first.
+      - the result is rounded once to bf16, the activation dtype the quantiser
+        receives in an unfused pipeline.
+    eps is the float32 value the caller passes, used exactly.
+    """
+    x = bf16_to_f64(x_bits)
+    rows, k = x.shape
+    eps64 = float(np.float32(eps))
+    r32 = np.empty(rows, dtype=np.float32)
+    for i in range(rows):
+        s = math.fsum(float(v) * float(v) for v in x[i])      # exact squares, one rounding
+        d = s / k + eps64
+        r32[i] = np.float32(1.0 / math.sqrt(d)) if d > 0 else np.float32(0.0)
+    u = (x.astype(np.float32) * r32[:, None]).astype(np.float32)
+    if gamma_bits is not None:
+        u = (u * bf16_to_f64(gamma_bits).astype(np.float32)[None, :]).astype(np.float32)
+    if scale_bits is not None:
+        a = (np.float32(1.0) + bf16_to_f64(scale_bits).astype(np.float32)).astype(np.float32)
+        u = (u * a[None, :]).astype(np.float32)
+    if shift_bits is not None:
+        u = (u + bf16_to_f64(shift_bits).astype(np.float32)[None, :]).astype(np.float32)
+    return f64_to_bf16(u.astype(np.float64))
+
+
+def norm_rot_quant(x_bits: np.ndarray, bits: int, rot_group: int = GROUP, scale_group: int = 0,
+                   gamma_bits=None, shift_bits=None, scale_bits=None, eps: float = 1e-6):
+    """The normalising prologue: norm_modulate, then the activation path (rot_quant)."""
+    xm = norm_modulate(x_bits, gamma_bits, shift_bits, scale_bits, eps)
+    return rot_quant(xm, bits, rot_group, scale_group)
 
 
 def pack_int4(q: np.ndarray) -> np.ndarray:

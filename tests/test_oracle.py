@@ -343,3 +343,63 @@ def test_nvfp4_block_error_bound_and_scale_range():
     assert np.all(np.abs(xr - deq) <= step / 2 * 1.0001 + 1e-30)
     rel = np.linalg.norm(xr - deq) / np.linalg.norm(xr)
     assert rel < 0.12
+
+
+# --------------------------------------------------------------- normalising prologue
+def _bits(a) -> np.ndarray:
+    return (np.asarray(a, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_norm_hand_worked_example():
+    # x = (3, 4): mean square 12.5, r = 1/sqrt(12.5) -> u = (0.848528, 1.131371);
+    # 1 + scale = (2, 1), shift = (0.5, -1): v = (2.197056, 0.131371) -> bf16
+    # 2.203125 (1.1015625 * 2) and 0.1318359375 (1.0546875 / 8)
+    out = O.bf16_to_f64(O.norm_modulate(_bits([[3.0, 4.0]]), None, _bits([0.5, -1.0]), _bits([1.0, 0.0]), 0.0))
+    assert out.tolist() == [[2.203125, 0.1318359375]]
+
+
+def test_norm_power_of_two_scale_invariance():
+    # without eps, scaling a row by 2^j changes nothing, bit for bit (catches a
+    # missing square root or a wrong power of the mean)
+    xb = I.gaussian_bf16(30, (6, 512), 1.0, 0.01, 20.0)
+    base = O.norm_modulate(xb, eps=0.0)
+    for j in (-7, 3, 20):
+        scaled = _bits(O.bf16_to_f64(xb) * 2.0 ** j)
+        assert np.array_equal(O.norm_modulate(scaled, eps=0.0), base)
+    # with eps the invariance is gone: eps is added to the mean square
+    assert not np.array_equal(O.norm_modulate(_bits(O.bf16_to_f64(xb) * 2.0 ** -12), eps=1e-3), base)
+
+
+def test_norm_unit_rms_and_constant_rows():
+    xb = I.gaussian_bf16(31, (5, 3072), 1.0, 0.005, 30.0)
+    u = O.bf16_to_f64(O.norm_modulate(xb, eps=0.0))
+    # mean of squares is 1 up to the bf16 rounding of each element (catches sum-instead-of-mean)
+    assert np.all(np.abs((u ** 2).mean(axis=1) - 1.0) < 2.0 ** -7)
+    # a constant row normalises to +-1 exactly; a zero row stays zero
+    const = np.full((3, 256), 3.0, np.float32)
+    const[1] = -0.375
+    const[2] = 0.0
+    c = O.bf16_to_f64(O.norm_modulate(_bits(const), eps=0.0))
+    assert np.all(c[0] == 1.0) and np.all(c[1] == -1.0) and np.all(c[2] == 0.0)
+
+
+def test_norm_matches_float64_formula_and_each_vector_acts_per_channel():
+    xb = I.gaussian_bf16(32, (7, 768), 1.0, 0.01, 25.0)
+    gamma = _bits(1.0 + O.bf16_to_f64(I.gaussian_bf16(33, (768,), 0.1)))
+    shift, scale = I.gaussian_bf16(34, (768,), 0.5), I.gaussian_bf16(35, (768,), 0.3)
+    x = O.bf16_to_f64(xb)
+    ref = (x / np.sqrt((x ** 2).mean(axis=1, keepdims=True) + 1e-6) * O.bf16_to_f64(gamma)
+           * (1.0 + O.bf16_to_f64(scale)) + O.bf16_to_f64(shift))
+    got = O.bf16_to_f64(O.norm_modulate(xb, gamma, shift, scale, 1e-6))
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -7 + 1e-6)
+    # swapping shift and scale (or dropping one) is detected
+    swapped = O.bf16_to_f64(O.norm_modulate(xb, gamma, scale, shift, 1e-6))
+    assert np.abs(swapped - ref).max() > 0.1
+
+
+def test_norm_rot_quant_is_the_composition():
+    xb = I.gaussian_bf16(36, (4, 512), 1.0, 0.01, 30.0)
+    shift = I.gaussian_bf16(37, (512,), 0.2)
+    q, s = O.norm_rot_quant(xb, 4, 256, 64, None, shift, None, 1e-6)
+    q2, s2 = O.rot_quant(O.norm_modulate(xb, None, shift, None, 1e-6), 4, 256, 64)
+    assert np.array_equal(q, q2) and np.array_equal(s, s2)
