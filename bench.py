@@ -423,6 +423,71 @@ def run_small_m_sweep(args):
             del g
 
 
+# ----------------------------------------------------------------------------- prologue sweep
+def run_prologue_sweep(args):
+    """The memory-bound activation prologues at the layer shapes: rotate/quantise, the normalising
+    prologue (RMSNorm + modulation ahead of it) and the single-pass low-rank prologue.  Each timed
+    call follows a 256 MB L2 flush; CUDA events on the launching stream.  One JSON line per case,
+    achieved HBM bandwidth from the algorithmic bytes (read X once, write codes and scales)."""
+    import torch
+
+    import rotated_bit_dit_b200 as R
+    from rotated_bit_dit_b200 import _binding as B
+    from rotated_bit_dit_b200 import inputs as I
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    R.load()
+    peaks, src = load_peaks()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    shapes = (("w4a4_qkvg input", 4096, 3072, 4, 64), ("w8a8_ffdown input", 4096, 12288, 8, 0),
+              ("stack mlp input", 16384, 3072, 4, 0))
+    for name, M, K, bits, sg in shapes:
+        x = up(I.gaussian_bf16(3, (M, K), 1.0, 0.005, 30.0))
+        gamma = up(I.f32_to_bf16_bits(1.0 + 0.1 * np.random.default_rng(4).standard_normal(K).astype(np.float32)))
+        shift, scale = up(I.gaussian_bf16(5, (K,), 0.5)), up(I.gaussian_bf16(6, (K,), 0.3))
+        codes = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sx = torch.empty((M, K // 64) if sg else (M,), dtype=torch.float32, device=dev)
+        r = 32
+        l1t = up(I.gaussian_bf16(7, (r, K), 0.01))
+        ld = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+        base = M * K * 2 + M * K + (M * (K // 64) if sg else M) * 4
+        cases = [("rot_quant", lambda: B.rbd_rot_quant_act(x, codes, sx, bits, 256, sg), base),
+                 ("norm_rot_quant", lambda: B.rbd_norm_rot_quant_act(x, codes, sx, gamma, shift, scale, 1e-6,
+                                                                     bits, 256, sg), base + 3 * K * 2)]
+        if sg == 64:
+            cases.append(("rot_quant_lowrank", lambda: B.rbd_lowrank_fused(x, codes, sx, l1t, ld, bits, 256, sg),
+                          base + M * r * 2 + r * K * 2))
+        for cname, fn, nbytes in cases:
+            for _ in range(max(args.warmup, 3)):
+                flush.zero_()
+                fn()
+            torch.cuda.synchronize()
+            assert R.rbd_check() == 0
+            ts = []
+            for _ in range(args.steps):
+                flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b) / 1e3)
+            assert R.rbd_check() == 0
+            t = statistics.median(ts)
+            gbs = nbytes / t / 1e9
+            print(json.dumps({
+                "sweep": "prologue", "call": cname, "shape": name, "M": M, "K": K, "bits": bits,
+                "scale_group": sg, "us": t * 1e6, "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                "peak_source": f"{src} copy {peaks['hbm_gbs']} GB/s", "algorithmic_bytes": nbytes,
+                "timing": f"median of {args.steps} calls, each after a 256 MB L2 flush"}), flush=True)
+
+
 # ----------------------------------------------------------------------------- 28-block stack
 STACK_LAYERS = (("wq", 3072, 3072), ("wk", 3072, 3072), ("wv", 3072, 3072), ("gate", 3072, 3072),
                 ("wo", 3072, 3072), ("mlp.gate", 3072, 12288), ("mlp.up", 3072, 12288), ("mlp.down", 12288, 3072))
@@ -530,7 +595,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--print-gemm-hash", action="store_true", help="print the GEMM source hash and exit")
-    ap.add_argument("--sweep", choices=["small-m", "stack"], default=None,
+    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue"], default=None,
                     help="instead of the headline line, print the small-token-count sweep (one line per case)")
     args = ap.parse_args()
     if args.print_gemm_hash:
@@ -541,6 +606,9 @@ def main():
         return
     if args.sweep == "stack":
         run_stack(args)
+        return
+    if args.sweep == "prologue":
+        run_prologue_sweep(args)
         return
     if args.impl == "reference" and int(os.environ.get("RANK", "0")) != 0:
         return                      # the oracle arm runs on rank 0 only; other ranks do no work

@@ -79,6 +79,27 @@ typedef struct rbd_qcfg {
 rbd_status rbd_rot_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, rbd_qcfg cfg,
                              int8_t* codes, float* scales, void* stream);
 
+/* RMSNorm and adaLN-style modulation fused ahead of rbd_rot_quant_act
+ * (Krea 2 Turbo OrbitQuant W4A4, "Fused transformer": the RMSNorm and the
+ * modulation run in the activation quantisation prologues).  Per row:
+ *   r = 1 / sqrt(sum_k x_k^2 / K + eps), float64 IEEE operations on the exact
+ *       squares, rounded once to float32 (r = 0 when the radicand is 0);
+ *   per element, single float32 operations in this order:
+ *       u = x * r;  u = u * gamma[k];  u = u * (1 + scale[k]);  u = u + shift[k];
+ *   u is rounded to bf16, then rotated and quantised exactly as
+ *   rbd_rot_quant_act does.
+ *   gamma, shift, scale  bf16 [K], 16-byte aligned, or NULL (the step is then
+ *           skipped); one modulation vector for all rows (batch 1).
+ *   eps     finite, >= 0 (RBD_ERR_INVALID_ARG otherwise).
+ * The float64 sum is exact when the squares of a row span fewer than about
+ * 53 - 16 - log2(K) binades; outside that the device's summation order can
+ * differ from the exact sum in the last float64 bit, which changes r only when
+ * r lies within that distance of a float32 rounding boundary.
+ * Other arguments, layouts and errors as rbd_rot_quant_act.                  */
+rbd_status rbd_norm_rot_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
+                                  const void* shift, const void* scale, float eps, rbd_qcfg cfg,
+                                  int8_t* codes, float* scales, void* stream);
+
 /* rbd_rot_quant_act plus the first factor of the low-rank branch on the
  * UNROTATED input: ld = X L1 (Krea-2-SVDQuant-ComfyUI, "LoRA": the branch is a
  * parallel linear, (W + L1 L2)-style, W x + L2 (L1 x)).

@@ -18,6 +18,7 @@ from ._binding import (  # noqa: F401
     rbd_pack_weights_int4,
     rbd_pack_weights_int8,
     rbd_rot_quant_act,
+    rbd_norm_rot_quant_act,
     rbd_status_string,
     rbd_version,
     rbd_w4a4_linear,

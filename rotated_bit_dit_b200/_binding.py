@@ -18,7 +18,7 @@ RBD_OK = 0
 STATUS_NAMES = {0: "RBD_OK", 1: "RBD_ERR_INVALID_ARG", 2: "RBD_ERR_UNSUPPORTED", 3: "RBD_ERR_ALIGNMENT",
                 4: "RBD_ERR_CUDA", 5: "RBD_ERR_DEVICE_TIMEOUT"}
 
-EXPORTED = ("rbd_rot_quant_act", "rbd_lowrank_fused", "rbd_pack_weights_int4", "rbd_pack_weights_int8",
+EXPORTED = ("rbd_rot_quant_act", "rbd_norm_rot_quant_act", "rbd_lowrank_fused", "rbd_pack_weights_int4", "rbd_pack_weights_int8",
             "rbd_w4a4_linear", "rbd_w8a8_linear", "rbd_nvfp4_scale_bytes", "rbd_nvfp4_quant",
             "rbd_nvfp4_quant_noalloc", "rbd_nvfp4_linear", "rbd_check", "rbd_debug_timeout_probe", "rbd_status_string", "rbd_version")
 
@@ -61,6 +61,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     i64, i32, vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p
     sigs = {
         "rbd_rot_quant_act": [vp, i64, i64, i64, QCfg, vp, vp, vp],
+        "rbd_norm_rot_quant_act": [vp, i64, i64, i64, vp, vp, vp, ctypes.c_float, QCfg, vp, vp, vp],
         "rbd_lowrank_fused": [vp, i64, i64, i64, QCfg, vp, vp, vp, i32, vp, vp],
         "rbd_pack_weights_int4": [vp, i64, i64, QCfg, vp, vp, vp],
         "rbd_pack_weights_int8": [vp, i64, i64, QCfg, vp, vp, vp],
@@ -124,6 +125,21 @@ def rbd_rot_quant_act(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor
     M, K = x.shape
     _ok(load().rbd_rot_quant_act(_ptr(x), M, K, _rowstride(x), _qcfg(bits, rot_group, scale_group),
                                  _ptr(codes), _ptr(scales), _stream(stream)), "rbd_rot_quant_act")
+
+
+def rbd_norm_rot_quant_act(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+                           gamma: Optional[torch.Tensor] = None, shift: Optional[torch.Tensor] = None,
+                           scale: Optional[torch.Tensor] = None, eps: float = 1e-6, bits: int = 4,
+                           rot_group: int = 256, scale_group: int = 0, stream=None) -> None:
+    """RMSNorm (optional gamma) and modulation x*(1 + scale) + shift, then rbd_rot_quant_act.
+    gamma, shift, scale: bf16 [K] or None."""
+    M, K = x.shape
+    for name, v in (("gamma", gamma), ("shift", shift), ("scale", scale)):
+        if v is not None and (v.numel() != K or not v.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous bf16 vector of length K")
+    _ok(load().rbd_norm_rot_quant_act(_ptr(x), M, K, _rowstride(x), _ptr(gamma), _ptr(shift), _ptr(scale),
+                                      float(eps), _qcfg(bits, rot_group, scale_group), _ptr(codes),
+                                      _ptr(scales), _stream(stream)), "rbd_norm_rot_quant_act")
 
 
 def rbd_lowrank_fused(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, l1t: torch.Tensor,

@@ -7,6 +7,8 @@
 
 #include <cudaTypedefs.h>
 
+#include <cmath>
+
 #include "rbd_common.cuh"
 
 #include "rbd_internal.cuh"
@@ -231,6 +233,20 @@ extern "C" {
 rbd_status rbd_rot_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, rbd_qcfg cfg, int8_t* codes,
                              float* scales, void* stream) {
   return quant_common(x, M, K, ldx, cfg, codes, scales, false, stream);
+}
+
+rbd_status rbd_norm_rot_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
+                                  const void* shift, const void* scale, float eps, rbd_qcfg cfg, int8_t* codes,
+                                  float* scales, void* stream) {
+  if (!(eps >= 0.0f) || !(eps < INFINITY)) return RBD_ERR_INVALID_ARG;   // rejects NaN too
+  if ((gamma && !aligned16(gamma)) || (shift && !aligned16(shift)) || (scale && !aligned16(scale)))
+    return RBD_ERR_ALIGNMENT;
+  rbd_status s = quant_validate(x, M, K, ldx, cfg, codes, scales);
+  if (s != RBD_OK || M == 0) return s;
+  return cuda_status(rbd::launch_norm_rot_quant(
+      static_cast<const uint16_t*>(x), M, K, ldx, cfg.bits, cfg.rot_group != 0, cfg.scale_group == 64,
+      static_cast<const uint16_t*>(gamma), static_cast<const uint16_t*>(shift),
+      static_cast<const uint16_t*>(scale), eps, codes, scales, as_stream(stream)));
 }
 
 rbd_status rbd_lowrank_fused(const void* x, int64_t M, int64_t K, int64_t ldx, rbd_qcfg cfg, int8_t* codes,

@@ -31,6 +31,10 @@ struct GemmArgs {
 
 cudaError_t launch_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot, bool g64,
                              bool packed, int8_t* codes, float* scales, cudaStream_t st);
+// RMSNorm + modulation, then rotate/quantise (activation codes, one byte each).
+cudaError_t launch_norm_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot,
+                                  bool g64, const uint16_t* gamma, const uint16_t* shift, const uint16_t* scale,
+                                  float eps, int8_t* codes, float* scales, cudaStream_t st);
 // Group-scale prologue and low-rank down product in one pass over X.
 cudaError_t launch_rot_quant_lowrank(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot,
                                      const uint16_t* l1t, int r, int8_t* codes, float* scales, uint16_t* ld,

@@ -39,16 +39,36 @@ __device__ __forceinline__ int quant1(float v, float inv, float qmax) {
 
 }  // namespace
 
+// RMSNorm + modulation ahead of the rotation (NORM variant).  gamma, shift and
+// scale are bf16 [K] vectors or null.
+struct NormArgs {
+  const uint16_t* gamma;
+  const uint16_t* shift;
+  const uint16_t* scale;
+  float eps;
+};
+
 // One CTA handles `rows` rows; each row is handled by T = 16 * teams threads;
 // team `tm` of a row processes 256-blocks g = tm, tm + teams, ... (at most CMAX).
 // OUT_PACKED: write packed INT4 bytes instead of one code per byte.
-template <bool ROT, bool G64, bool OUT_PACKED, int CMAX>
+// NORM: the row (all of it is in registers) is first normalised and modulated
+// -- "Krea 2 Turbo OrbitQuant W4A4", section "Fused transformer": the RMSNorm
+// and modulation run in the activation quantisation prologues.  The sum of the
+// exact squares is accumulated in float64 and reduced across the row's
+// threads; r = 1 / sqrt(sum / K + eps) (float64 IEEE operations) is rounded
+// once to float32; then per element, as single float32 operations,
+// u = x * r, u *= gamma, u *= (1 + scale), u += shift, rounded once to bf16.
+// A row whose mean square plus eps is zero gets r = 0.
+template <bool ROT, bool G64, bool OUT_PACKED, int CMAX, bool NORM = false>
 __global__ void __launch_bounds__(256) rot_quant_kernel(const uint16_t* __restrict__ x, int64_t M, int K,
                                                         int64_t ldx, float qmax, int teams, int rows,
-                                                        int8_t* __restrict__ codes, float* __restrict__ scales) {
+                                                        int8_t* __restrict__ codes, float* __restrict__ scales,
+                                                        NormArgs norm) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* xbuf = reinterpret_cast<double*>(smem_raw);        // [teams*rows][256]
   float* red = reinterpret_cast<float*>(smem_raw + (size_t)blockDim.x / kTeam * 256 * sizeof(double));
+  double* red64 = reinterpret_cast<double*>(smem_raw + (size_t)blockDim.x / kTeam * 256 * sizeof(double) +
+                                            64 * sizeof(float));
 
   const int T = kTeam * teams;
   const int tid = threadIdx.x;
@@ -73,6 +93,76 @@ __global__ void __launch_bounds__(256) rot_quant_kernel(const uint16_t* __restri
     } else {
       raw[c][0] = make_uint4(0, 0, 0, 0);
       raw[c][1] = make_uint4(0, 0, 0, 0);
+    }
+  }
+
+  if constexpr (NORM) {
+    // the per-channel vectors of a block are fetched after the row reduction
+    // (fetching them earlier raises the register count and measured slower)
+    auto fetch_vec = [&](const uint16_t* v, int g, uint4 (&d)[2]) {
+      if (v) {
+        const uint4* p = reinterpret_cast<const uint4*>(v + (int64_t)g * 256 + tau * 16);
+        d[0] = __ldg(p);
+        d[1] = __ldg(p + 1);
+      }
+    };
+    // ---- sum of squares (exact squares; blocks past the row end hold zeros)
+    double ss = 0.0;
+#pragma unroll
+    for (int c = 0; c < CMAX; ++c) {
+      const uint32_t w[8] = {raw[c][0].x, raw[c][0].y, raw[c][0].z, raw[c][0].w,
+                             raw[c][1].x, raw[c][1].y, raw[c][1].z, raw[c][1].w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const double lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xFFFF0000u);
+        ss = fma(lo, lo, ss);
+        ss = fma(hi, hi, ss);
+      }
+    }
+    if (T <= 32) {
+      for (int off = T / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    } else {
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      const int wpr = T / 32;
+      if ((tid & 31) == 0) red64[tid / 32] = ss;
+      __syncthreads();
+      ss = 0.0;
+      for (int w = 0; w < wpr; ++w) ss += red64[rloc * wpr + w];
+    }
+    const double d = ss / static_cast<double>(K) + static_cast<double>(norm.eps);
+    const float r = d > 0.0 ? __double2float_rn(1.0 / sqrt(d)) : 0.f;
+    // ---- per element: u = x r, * gamma, * (1 + scale), + shift, one bf16 rounding
+#pragma unroll
+    for (int c = 0; c < CMAX; ++c) {
+      const int g = team + c * teams;
+      if (g >= G) continue;   // blocks past the row end stay zero
+      uint4 vg[2], vs[2], vc[2];
+      fetch_vec(norm.gamma, g, vg);
+      fetch_vec(norm.shift, g, vs);
+      fetch_vec(norm.scale, g, vc);
+      uint32_t* w = reinterpret_cast<uint32_t*>(&raw[c][0]);   // raw[c][0..1] are contiguous
+      const uint32_t* wg = reinterpret_cast<const uint32_t*>(&vg[0]);
+      const uint32_t* ws = reinterpret_cast<const uint32_t*>(&vs[0]);
+      const uint32_t* wc = reinterpret_cast<const uint32_t*>(&vc[0]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float u0 = __fmul_rn(__uint_as_float(w[j] << 16), r);
+        float u1 = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), r);
+        if (norm.gamma) {
+          u0 = __fmul_rn(u0, __uint_as_float(wg[j] << 16));
+          u1 = __fmul_rn(u1, __uint_as_float(wg[j] & 0xFFFF0000u));
+        }
+        if (norm.scale) {
+          u0 = __fmul_rn(u0, __fadd_rn(1.0f, __uint_as_float(wc[j] << 16)));
+          u1 = __fmul_rn(u1, __fadd_rn(1.0f, __uint_as_float(wc[j] & 0xFFFF0000u)));
+        }
+        if (norm.shift) {
+          u0 = __fadd_rn(u0, __uint_as_float(ws[j] << 16));
+          u1 = __fadd_rn(u1, __uint_as_float(ws[j] & 0xFFFF0000u));
+        }
+        w[j] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(u0)) |
+               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(u1)) << 16);
+      }
     }
   }
 
@@ -454,21 +544,21 @@ Geometry geometry(int64_t K) {
   gm.T = kTeam * teams;
   gm.rows = gm.T >= 256 ? 1 : 256 / gm.T;
   gm.threads = gm.T * gm.rows;
-  gm.smem = (size_t)(gm.threads / kTeam) * 256 * sizeof(double) + 64 * sizeof(float);
+  gm.smem = (size_t)(gm.threads / kTeam) * 256 * sizeof(double) + 64 * sizeof(float) + 64 * sizeof(double);
   return gm;
 }
 
-template <bool ROT, bool G64, bool PK>
+template <bool ROT, bool G64, bool PK, bool NORM = false>
 cudaError_t launch_rq_c(int cmax, dim3 grid, int threads, size_t smem, cudaStream_t st, const uint16_t* x,
                         int64_t M, int K, int64_t ldx, float qmax, int teams, int rows, int8_t* codes,
-                        float* scales) {
+                        float* scales, NormArgs norm = NormArgs{}) {
   switch (cmax) {
 #define RBD_RQ_CASE(C)                                                                                    \
   case C: {                                                                                               \
-    auto kern = rot_quant_kernel<ROT, G64, PK, C>;                                                        \
+    auto kern = rot_quant_kernel<ROT, G64, PK, C, NORM>;                                                  \
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
     if (e != cudaSuccess) return e;                                                                       \
-    kern<<<grid, threads, smem, st>>>(x, M, K, ldx, qmax, teams, rows, codes, scales);                   \
+    kern<<<grid, threads, smem, st>>>(x, M, K, ldx, qmax, teams, rows, codes, scales, norm);             \
     return cudaGetLastError();                                                                            \
   }
     RBD_RQ_CASE(1)
@@ -506,6 +596,26 @@ cudaError_t launch_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ld
     }
   }
 #undef RBD_RQ_DISPATCH
+}
+
+cudaError_t launch_norm_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot,
+                                  bool g64, const uint16_t* gamma, const uint16_t* shift, const uint16_t* scale,
+                                  float eps, int8_t* codes, float* scales, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  const Geometry gm = geometry(K);
+  const float qmax = bits == 4 ? 7.f : 127.f;
+  const dim3 grid(static_cast<unsigned>((M + gm.rows - 1) / gm.rows));
+  const int Ki = static_cast<int>(K);
+  const NormArgs norm{gamma, shift, scale, eps};
+#define RBD_NRQ(R_, G_)                                                                                \
+  return launch_rq_c<R_, G_, false, true>(gm.cmax, grid, gm.threads, gm.smem, st, x, M, Ki, ldx, qmax, \
+                                          gm.teams, gm.rows, codes, scales, norm)
+  if (rot) {
+    if (g64) RBD_NRQ(true, true); else RBD_NRQ(true, false);
+  } else {
+    if (g64) RBD_NRQ(false, true); else RBD_NRQ(false, false);
+  }
+#undef RBD_NRQ
 }
 
 cudaError_t launch_lowrank_down(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const uint16_t* l1t, int r,

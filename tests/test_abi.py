@@ -136,3 +136,18 @@ def test_nvfp4_noalloc_validation_without_gpu():
     assert lib.rbd_nvfp4_quant_noalloc(FAKE, 0, 320, 320, 256, null, null, null, null) == 2
     assert lib.rbd_nvfp4_quant_noalloc(FAKE, -1, 256, 256, 256, FAKE, FAKE, FAKE, null) == 1
     assert lib.rbd_nvfp4_quant_noalloc(FAKE, 4, 256, 256, 256, null, FAKE, FAKE, null) == 1
+
+
+def test_norm_rot_quant_validation_without_gpu():
+    lib = R.load()
+    null = ctypes.c_void_p(0)
+    eps = ctypes.c_float(1e-6)
+    assert lib.rbd_norm_rot_quant_act(FAKE, 4, 256, 256, None, None, None, -1.0, q(), FAKE, FAKE, None) == 1
+    assert lib.rbd_norm_rot_quant_act(FAKE, 4, 256, 256, None, None, None, float("nan"), q(), FAKE, FAKE, None) == 1
+    assert lib.rbd_norm_rot_quant_act(FAKE, 4, 256, 256, None, None, None, float("inf"), q(), FAKE, FAKE, None) == 1
+    assert lib.rbd_norm_rot_quant_act(FAKE, 4, 256, 256, FAKE_MIS, None, None, eps, q(), FAKE, FAKE, None) == 3
+    assert lib.rbd_norm_rot_quant_act(FAKE, 4, 256, 256, None, FAKE_MIS, None, eps, q(), FAKE, FAKE, None) == 3
+    assert lib.rbd_norm_rot_quant_act(FAKE, 4, 100, 100, None, None, None, eps, q(), FAKE, FAKE, None) == 2
+    assert lib.rbd_norm_rot_quant_act(FAKE, 4, 256, 256, None, None, None, eps, q(bits=5), FAKE, FAKE, None) == 1
+    assert lib.rbd_norm_rot_quant_act(FAKE, 4, 256, 256, None, None, None, eps, q(), null, FAKE, None) == 1
+    assert lib.rbd_norm_rot_quant_act(FAKE, 0, 256, 256, None, None, None, eps, q(), null, null, None) == 0
