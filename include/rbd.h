@@ -114,6 +114,16 @@ rbd_status rbd_lowrank_fused(const void* x, int64_t M, int64_t K, int64_t ldx, r
                              int8_t* codes, float* scales, const void* l1t, int32_t r, void* ld,
                              void* stream);
 
+/* The low-rank branch's first factor alone, ld = X L1 on the unrotated input
+ * (Krea-2-SVDQuant-ComfyUI, "LoRA"), for paths whose quantiser is not
+ * rbd_lowrank_fused (the NVFP4 variant).
+ *   x       bf16 [M, ldx], 16-byte aligned, ldx % 8 == 0; K % 128 == 0, K <= 16384.
+ *   l1t     bf16 [r, K] row-major (L1 stored output-major), r in {16, 32, 64}.
+ *   ld      bf16 [M, r] row-major (float32 accumulation, a fixed-order
+ *           reduction, rounded once).                                          */
+rbd_status rbd_lowrank_down(const void* x, int64_t M, int64_t K, int64_t ldx, const void* l1t,
+                            int32_t r, void* ld, void* stream);
+
 /* Offline weight rotate + quantise + pack to signed INT4 (INT4 tensorwise card,
  * header: "packed signed INT4 weights with group-256 ... rotation").
  * Each output row of W is rotated and quantised exactly like a token.
@@ -233,8 +243,12 @@ rbd_status rbd_nvfp4_quant_noalloc(const void* x, int64_t M, int64_t K, int64_t 
  *   activation tensor scale (device float); wq uint8 [N, K/2], wbs, wgs
  *   likewise for the weights (rbd_nvfp4_quant of W [N, K]).
  *   K % 256 == 0, N % 128 == 0; all code and scale buffers 16-byte aligned.
- *   epi: bias and gate modes as for rbd_w4a4_linear; the low-rank branch
- *   (r != 0) and acc_debug are not supported here (RBD_ERR_UNSUPPORTED).
+ *   epi: bias, low-rank branch and gate modes as for rbd_w4a4_linear
+ *   (Krea-2-SVDQuant-ComfyUI, "LoRA": the same parallel branch beside the
+ *   FP4 product): y = gs_x gs_w acc + bias + (ld l2)[m, n], the branch
+ *   computed by a bf16 MMA with float32 accumulation (ld from
+ *   rbd_lowrank_down, r in {16, 32, 64}); acc_debug is not supported here
+ *   (RBD_ERR_UNSUPPORTED).
  *   y bf16 [M, ldy], ldy >= N, ldy % 8 == 0.                                  */
 rbd_status rbd_nvfp4_linear(const uint8_t* xq, const uint8_t* xbs, const float* xgs,
                             const uint8_t* wq, const uint8_t* wbs, const float* wgs,

@@ -15,6 +15,7 @@ from ._binding import (  # noqa: F401
     rbd_check,
     rbd_debug_timeout_probe,
     rbd_lowrank_fused,
+    rbd_lowrank_down,
     rbd_pack_weights_int4,
     rbd_pack_weights_int8,
     rbd_rot_quant_act,

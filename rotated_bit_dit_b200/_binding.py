@@ -18,7 +18,7 @@ RBD_OK = 0
 STATUS_NAMES = {0: "RBD_OK", 1: "RBD_ERR_INVALID_ARG", 2: "RBD_ERR_UNSUPPORTED", 3: "RBD_ERR_ALIGNMENT",
                 4: "RBD_ERR_CUDA", 5: "RBD_ERR_DEVICE_TIMEOUT"}
 
-EXPORTED = ("rbd_rot_quant_act", "rbd_norm_rot_quant_act", "rbd_lowrank_fused", "rbd_pack_weights_int4", "rbd_pack_weights_int8",
+EXPORTED = ("rbd_rot_quant_act", "rbd_norm_rot_quant_act", "rbd_lowrank_fused", "rbd_lowrank_down", "rbd_pack_weights_int4", "rbd_pack_weights_int8",
             "rbd_w4a4_linear", "rbd_w8a8_linear", "rbd_nvfp4_scale_bytes", "rbd_nvfp4_quant",
             "rbd_nvfp4_quant_noalloc", "rbd_nvfp4_linear", "rbd_check", "rbd_debug_timeout_probe", "rbd_status_string", "rbd_version")
 
@@ -63,6 +63,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "rbd_rot_quant_act": [vp, i64, i64, i64, QCfg, vp, vp, vp],
         "rbd_norm_rot_quant_act": [vp, i64, i64, i64, vp, vp, vp, ctypes.c_float, QCfg, vp, vp, vp],
         "rbd_lowrank_fused": [vp, i64, i64, i64, QCfg, vp, vp, vp, i32, vp, vp],
+        "rbd_lowrank_down": [vp, i64, i64, i64, vp, i32, vp, vp],
         "rbd_pack_weights_int4": [vp, i64, i64, QCfg, vp, vp, vp],
         "rbd_pack_weights_int8": [vp, i64, i64, QCfg, vp, vp, vp],
         "rbd_w4a4_linear": [vp, vp, vp, vp, i64, i64, i64, QCfg, ctypes.POINTER(Epilogue), vp, i64, vp],
@@ -153,6 +154,16 @@ def rbd_lowrank_fused(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor
     _ok(load().rbd_lowrank_fused(_ptr(x), M, K, _rowstride(x), _qcfg(bits, rot_group, scale_group),
                                  _ptr(codes), _ptr(scales), _ptr(l1t), r, _ptr(ld), _stream(stream)),
         "rbd_lowrank_fused")
+
+
+def rbd_lowrank_down(x: torch.Tensor, l1t: torch.Tensor, ld: torch.Tensor, stream=None) -> None:
+    """ld = X @ L1 alone (l1t = L1^T bf16 [r, K], ld bf16 [M, r])."""
+    M, K = x.shape
+    r = l1t.shape[0]
+    if _rowstride(l1t) != K:
+        raise ValueError("l1t must be a contiguous [r, K] tensor")
+    _ok(load().rbd_lowrank_down(_ptr(x), M, K, _rowstride(x), _ptr(l1t), r, _ptr(ld), _stream(stream)),
+        "rbd_lowrank_down")
 
 
 def rbd_pack_weights_int4(w: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, rot_group: int = 256,

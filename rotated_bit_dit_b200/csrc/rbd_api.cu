@@ -269,6 +269,20 @@ rbd_status rbd_lowrank_fused(const void* x, int64_t M, int64_t K, int64_t ldx, r
                                               as_stream(stream)));
 }
 
+rbd_status rbd_lowrank_down(const void* x, int64_t M, int64_t K, int64_t ldx, const void* l1t, int32_t r, void* ld,
+                            void* stream) {
+  if (r != 16 && r != 32 && r != 64) return RBD_ERR_UNSUPPORTED;
+  if (M < 0 || K <= 0) return RBD_ERR_INVALID_ARG;
+  if (K % 128 != 0 || K > 16384 || M > (int64_t)INT32_MAX / 2) return RBD_ERR_UNSUPPORTED;
+  if (M == 0) return RBD_OK;
+  if (!x || !l1t || !ld) return RBD_ERR_INVALID_ARG;
+  if (ldx < K) return RBD_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(l1t) || !aligned16(ld) || (ldx % 8) != 0) return RBD_ERR_ALIGNMENT;
+  return cuda_status(rbd::launch_lowrank_down(static_cast<const uint16_t*>(x), M, K, ldx,
+                                              static_cast<const uint16_t*>(l1t), r, static_cast<uint16_t*>(ld),
+                                              as_stream(stream)));
+}
+
 rbd_status rbd_pack_weights_int4(const void* w, int64_t N, int64_t K, rbd_qcfg cfg, uint8_t* packed, float* scales,
                                  void* stream) {
   if (cfg.bits != 4) return RBD_ERR_INVALID_ARG;
@@ -338,7 +352,10 @@ rbd_status rbd_nvfp4_linear(const uint8_t* xq, const uint8_t* xbs, const float* 
   if ((reinterpret_cast<uintptr_t>(xgs) & 3u) || (reinterpret_cast<uintptr_t>(wgs) & 3u)) return RBD_ERR_ALIGNMENT;
   rbd_epilogue e{};
   if (epi) e = *epi;
-  if (e.r != 0 || e.acc_debug) return RBD_ERR_UNSUPPORTED;
+  if (e.acc_debug) return RBD_ERR_UNSUPPORTED;
+  if (e.r != 0 && e.r != 16 && e.r != 32 && e.r != 64) return RBD_ERR_UNSUPPORTED;
+  if (e.r && (!e.ld || !e.l2t)) return RBD_ERR_INVALID_ARG;
+  if (e.r && (!aligned16(e.ld) || !aligned16(e.l2t))) return RBD_ERR_ALIGNMENT;
   if (e.gate_mode < 0 || e.gate_mode > 2) return RBD_ERR_INVALID_ARG;
   if (e.gate_mode == 1 && (e.gate_col0 < 0 || e.gate_col1 < e.gate_col0 || e.gate_col1 > N))
     return RBD_ERR_INVALID_ARG;
@@ -349,9 +366,15 @@ rbd_status rbd_nvfp4_linear(const uint8_t* xq, const uint8_t* xbs, const float* 
       return RBD_ERR_ALIGNMENT;
   }
   if (e.bias && (reinterpret_cast<uintptr_t>(e.bias) & 1u)) return RBD_ERR_ALIGNMENT;
-  CUtensorMap tm_x{}, tm_w{};
+  CUtensorMap tm_x{}, tm_w{}, tm_ld{}, tm_l2{};
   if (!make_map_2d(&tm_x, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, K / 2, 128, 128)) return RBD_ERR_CUDA;
   if (!make_map_2d(&tm_w, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 128, 128)) return RBD_ERR_CUDA;
+  if (e.r) {
+    if (!make_map_2d(&tm_ld, e.ld, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, e.r, M, 2 * e.r, e.r, 128))
+      return RBD_ERR_CUDA;
+    if (!make_map_2d(&tm_l2, e.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, e.r, N, 2 * e.r, e.r, 128))
+      return RBD_ERR_CUDA;
+  }
   rbd::NvArgs a{};
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
@@ -371,9 +394,10 @@ rbd_status rbd_nvfp4_linear(const uint8_t* xq, const uint8_t* xbs, const float* 
   a.ldy = ldy;
   a.num_m_tiles = static_cast<int>((M + 127) / 128);
   a.num_tiles = a.num_m_tiles * static_cast<int>(N / 128);
+  a.r = static_cast<int>(e.r);
   const int sms = num_sms_current();
   if (sms <= 0) return RBD_ERR_CUDA;
-  return cuda_status(rbd::launch_nvfp4_gemm(tm_x, tm_w, a, sms, as_stream(stream)));
+  return cuda_status(rbd::launch_nvfp4_gemm(tm_x, tm_w, tm_ld, tm_l2, a, sms, as_stream(stream)));
 }
 
 rbd_status rbd_check(void* stream) {

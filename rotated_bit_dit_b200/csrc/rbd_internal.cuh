@@ -61,12 +61,13 @@ struct NvArgs {
   uint16_t* y;
   int64_t ldy;
   int num_m_tiles, num_tiles;
+  int r;                // low-rank branch rank (0: none); ld / l2t come by tensor map
 };
 
 cudaError_t launch_nvfp4_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, bool rot, uint32_t* work,
                                uint8_t* codes, uint8_t* bscale, float* gscale, cudaStream_t st);
-cudaError_t launch_nvfp4_gemm(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const NvArgs& a, int num_sms,
-                              cudaStream_t st);
+cudaError_t launch_nvfp4_gemm(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const CUtensorMap& tm_ld,
+                              const CUtensorMap& tm_l2, const NvArgs& a, int num_sms, cudaStream_t st);
 uint32_t nvfp4_gemm_smem_bytes();
 
 uint32_t gemm_smem_bytes(bool g64, int r, int G);   // dynamic shared memory of one GEMM CTA

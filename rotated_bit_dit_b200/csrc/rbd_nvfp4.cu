@@ -210,24 +210,34 @@ constexpr uint32_t kNvOpBytes = 128 * 128;    // one operand stage
 constexpr uint32_t kNvSfBytes = 4 * 512;      // one scale stage (4 K steps)
 constexpr int kNvStages = 4;
 constexpr uint32_t kNvStageBytes = 2 * kNvOpBytes + 2 * kNvSfBytes;
-constexpr uint32_t kNvSmem = kNvStages * kNvStageBytes + 1024 + 256;
+constexpr uint32_t kNvLrBytes = 2 * 128 * 128;  // low-rank tiles: l2t [128 x r] and ld [128 x r], r <= 64
+constexpr uint32_t kNvSmem = kNvStages * kNvStageBytes + kNvLrBytes + 1024 + 256;
 constexpr uint32_t kNvAccCols = 2 * kNvTile;  // two accumulator buffers
+constexpr uint32_t kNvLrCol = 384;            // low-rank accumulator (after the scale regions)
 }  // namespace
 
 __global__ void __launch_bounds__(kNvThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                      const __grid_constant__ CUtensorMap tm_ld, const __grid_constant__ CUtensorMap tm_l2,
                       const NvArgs args) {
   extern __shared__ unsigned char smem_dyn[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023u) & ~uintptr_t(1023u));
   // stage s: A (weights) | B (tokens) | SFA | SFB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kNvStages * kNvStageBytes);
+  // low-rank tiles after the stages: l2t rows (A side) then ld rows (B side)
+  unsigned char* lr_a = smem + kNvStages * kNvStageBytes;
+  unsigned char* lr_b = lr_a + kNvLrBytes / 2;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kNvStages * kNvStageBytes + kNvLrBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + kNvStages;
   uint64_t* tfull = bars + 2 * kNvStages;    // [2]
   uint64_t* tempty = tfull + 2;              // [2]
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* lrsfull = drain + 1;             // low-rank tiles landed in shared memory
+  uint64_t* lrsempty = lrsfull + 1;          // low-rank MMAs done with them
+  uint64_t* lrtempty = lrsempty + 1;         // epilogue has read the low-rank accumulator
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(lrtempty + 1);
+  const int R = args.r;
   const uint32_t warp = warp_id(), lane = lane_id();
   const int nks = args.K / kNvBK;
 
@@ -241,9 +251,16 @@ __global__ void __launch_bounds__(kNvThreads, 1)
       mbar_init(&tempty[b], (kNvThreads / 32) - kNvWarpEpi0);
     }
     mbar_init(drain, 1);
+    mbar_init(lrsfull, 1);
+    mbar_init(lrsempty, 1);
+    mbar_init(lrtempty, (kNvThreads / 32) - kNvWarpEpi0);
     fence_barrier_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
+    if (R) {
+      tma_prefetch_desc(&tm_ld);
+      tma_prefetch_desc(&tm_l2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, 512);
@@ -258,10 +275,18 @@ __global__ void __launch_bounds__(kNvThreads, 1)
     // ---------------------------------------------------------- producer
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0;
+      uint32_t phase = 0, lr_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
         const int mt = t % args.num_m_tiles, nt = t / args.num_m_tiles;
+        if (R) {
+          // the tile's low-rank operands, consumed after its K loop
+          if (!mbar_wait(lrsempty, lr_phase ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(lrsfull, 2u * kNvTile * (uint32_t)R * 2u);
+          tma_load_2d(lr_a, &tm_l2, lrsfull, 0, nt * kNvTile);
+          tma_load_2d(lr_b, &tm_ld, lrsfull, 0, mt * kNvTile);
+          lr_phase ^= 1;
+        }
         for (int ks = 0; ks < nks; ++ks) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           unsigned char* st = smem + stage * kNvStageBytes;
@@ -285,8 +310,10 @@ __global__ void __launch_bounds__(kNvThreads, 1)
     // ---------------------------------------------------------- MMA issuer
     if (elect_one()) {
       const uint32_t idesc = idesc_nvf4(kNvTile, kNvTile);
+      const uint32_t idesc_lr = idesc_bf16(kNvTile, kNvTile);
+      const uint32_t lr_row_bytes = (uint32_t)R * 2u;
       int stage = 0;
-      uint32_t phase = 0, tph = 0;
+      uint32_t phase = 0, tph = 0, lr_phase = 0;
       int ab = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
@@ -313,6 +340,18 @@ __global__ void __launch_bounds__(kNvThreads, 1)
           if (++stage == kNvStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
+        if (R) {
+          // low-rank segment into its own accumulator; the tile's tfull commit
+          // below covers these MMAs too
+          if (!mbar_wait(lrsfull, lr_phase) || !mbar_wait(lrtempty, lr_phase ^ 1)) { ok = false; break; }
+          lr_phase ^= 1;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(lr_a), b0 = smem_u32(lr_b);
+          for (int kk = 0; kk < R / 16; ++kk)
+            mma_bf16_ss(tmem + kNvLrCol, smem_desc_kmajor(a0 + kk * 32, lr_row_bytes),
+                        smem_desc_kmajor(b0 + kk * 32, lr_row_bytes), idesc_lr, kk > 0 ? 1u : 0u);
+          tc_commit(lrsempty);
+        }
         tc_commit(&tfull[ab]);
         ab ^= 1;
       }
@@ -332,16 +371,28 @@ __global__ void __launch_bounds__(kNvThreads, 1)
       if (!mbar_wait(&tfull[ab], (tph >> ab) & 1u)) break;
       tph ^= 1u << ab;
       tc_fence_after();
-      uint32_t v[4][16];
+      uint32_t v[4][16], vl[4][16];
       const uint32_t tb = tmem + lane_base + ab * kNvTile + 64u * h;
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld16_async(tb + 16u * c, v[c]);
+      if (R) {
+        const uint32_t tl = tmem + lane_base + kNvLrCol + 64u * h;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld16_async(tl + 16u * c, vl[c]);
+      }
       tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_reg_fence(v[c]);
+      if (R) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_reg_fence(vl[c]);
+      }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[ab]);
+      if (lane == 0) {
+        mbar_arrive(&tempty[ab]);
+        if (R) mbar_arrive(lrtempty);
+      }
       ab ^= 1;
 
       const int n = nt * kNvTile + 32 * (int)q + (int)lane;
@@ -354,6 +405,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
         const int64_t m = mbase + j;
         if (m < args.M) {
           float o = fmaf(__uint_as_float(v[j >> 4][j & 15]), gsc, bias);
+          if (R) o += __uint_as_float(vl[j >> 4][j & 15]);
           if (args.gate_mode == 2) {
             o = fmaf(gv, o, __uint_as_float((uint32_t)args.residual[m * args.ldr + n] << 16));
           } else if (sig) {
@@ -373,12 +425,12 @@ __global__ void __launch_bounds__(kNvThreads, 1)
 
 uint32_t nvfp4_gemm_smem_bytes() { return kNvSmem; }
 
-cudaError_t launch_nvfp4_gemm(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const NvArgs& a, int num_sms,
-                              cudaStream_t st) {
+cudaError_t launch_nvfp4_gemm(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const CUtensorMap& tm_ld,
+                              const CUtensorMap& tm_l2, const NvArgs& a, int num_sms, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kNvSmem);
   if (e != cudaSuccess) return e;
   const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
-  nvfp4_gemm_kernel<<<grid, kNvThreads, kNvSmem, st>>>(tm_x, tm_w, a);
+  nvfp4_gemm_kernel<<<grid, kNvThreads, kNvSmem, st>>>(tm_x, tm_w, tm_ld, tm_l2, a);
   return cudaGetLastError();
 }
 

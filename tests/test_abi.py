@@ -118,12 +118,19 @@ def test_nvfp4_validation_without_gpu():
     assert lib.rbd_nvfp4_quant(FAKE, 4, 256, 256, 256, null, FAKE, FAKE, FAKE, null) == 1
     assert lib.rbd_nvfp4_quant(FAKE_MIS, 4, 256, 256, 256, FAKE, FAKE, FAKE, FAKE, null) == 3
     assert lib.rbd_nvfp4_quant(FAKE, 0, 256, 256, 256, null, null, null, null, null) == 0
-    # linear: N not a multiple of 128, low-rank branch unsupported, misaligned scales
+    # linear: N not a multiple of 128, unsupported rank, rank without factors, misaligned scales
     e = B.Epilogue()
     assert lib.rbd_nvfp4_linear(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 64, 256, ctypes.byref(e), FAKE, 64, null) == 2
-    e.r = 16
+    e.r = 24
     assert lib.rbd_nvfp4_linear(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 128, 256, ctypes.byref(e), FAKE, 128,
                                 null) == 2
+    e.r = 16
+    assert lib.rbd_nvfp4_linear(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 128, 256, ctypes.byref(e), FAKE, 128,
+                                null) == 1
+    e.ld, e.l2t = FAKE_MIS.value, FAKE.value
+    assert lib.rbd_nvfp4_linear(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 128, 256, ctypes.byref(e), FAKE, 128,
+                                null) == 3
+    e.ld = e.l2t = None
     e.r = 0
     assert lib.rbd_nvfp4_linear(FAKE, FAKE_MIS, FAKE, FAKE, FAKE, FAKE, 4, 128, 256, ctypes.byref(e), FAKE, 128,
                                 null) == 3
@@ -151,3 +158,14 @@ def test_norm_rot_quant_validation_without_gpu():
     assert lib.rbd_norm_rot_quant_act(FAKE, 4, 256, 256, None, None, None, eps, q(bits=5), FAKE, FAKE, None) == 1
     assert lib.rbd_norm_rot_quant_act(FAKE, 4, 256, 256, None, None, None, eps, q(), null, FAKE, None) == 1
     assert lib.rbd_norm_rot_quant_act(FAKE, 0, 256, 256, None, None, None, eps, q(), null, null, None) == 0
+
+
+def test_lowrank_down_validation_without_gpu():
+    lib = R.load()
+    null = ctypes.c_void_p(0)
+    assert lib.rbd_lowrank_down(FAKE, 4, 256, 256, FAKE, 24, FAKE, None) == 2      # rank
+    assert lib.rbd_lowrank_down(FAKE, 4, 192, 192, FAKE, 32, FAKE, None) == 2      # K % 128
+    assert lib.rbd_lowrank_down(FAKE, 4, 256, 256, null, 32, FAKE, None) == 1      # no factor
+    assert lib.rbd_lowrank_down(FAKE, 4, 256, 128, FAKE, 32, FAKE, None) == 1      # ldx < K
+    assert lib.rbd_lowrank_down(FAKE_MIS, 4, 256, 256, FAKE, 32, FAKE, None) == 3
+    assert lib.rbd_lowrank_down(FAKE, 0, 256, 256, null, 32, null, None) == 0      # empty batch

@@ -72,14 +72,21 @@ def test_nvfp4_quant_zero_tensor():
     assert not scales_from_tiles(bs.cpu().numpy(), 5, 512).any()
 
 
-def run_linear(xb, wb, bias=None, gate_mode=0, gate_cols=(0, 0), gate=None, residual=None):
+def run_linear(xb, wb, bias=None, gate_mode=0, gate_cols=(0, 0), gate=None, residual=None, l1=None, l2=None):
     M, K = xb.shape
     N = wb.shape[0]
     xq, xbs, xgs = gpu_quant(xb)
     wq, wbs, wgs = gpu_quant(wb)
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     dv = lambda a: None if a is None else dev_bf16(a)
-    epi = R.make_epilogue(dv(bias), None, None, gate_mode, gate_cols, dv(gate), dv(residual))
+    ld = l2t = None
+    if l1 is not None:
+        # the branch's first factor from the unrotated input, then L2 as the GEMM's second MMA
+        r = l1.shape[1]
+        ld = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+        R.rbd_lowrank_down(dev_bf16(xb), dev_bf16(np.ascontiguousarray(l1.T)), ld)
+        l2t = dev_bf16(np.ascontiguousarray(l2.T))
+    epi = R.make_epilogue(dv(bias), ld, l2t, gate_mode, gate_cols, dv(gate), dv(residual))
     R.rbd_nvfp4_linear(xq, xbs, xgs, wq, wbs, wgs, y, epi)
     assert R.rbd_check() == 0
     return host_u16(y)
@@ -87,7 +94,10 @@ def run_linear(xb, wb, bias=None, gate_mode=0, gate_cols=(0, 0), gate=None, resi
 
 def reference(xb, wb, **kw):
     y = O.nvfp4_linear(xb, wb)
-    y = O.epilogue(y, kw.get("bias"), None, None, kw.get("gate_mode", 0), kw.get("gate_cols", (0, 0)),
+    # the branch's first factor crosses the ABI as bf16 [M, r]; the oracle's own
+    # value, rounded the same way, is what the GEMM receives
+    ld = O.bf16_to_f64(O.f64_to_bf16(O.lowrank_down(xb, kw["l1"]))) if kw.get("l1") is not None else None
+    y = O.epilogue(y, kw.get("bias"), ld, kw.get("l2"), kw.get("gate_mode", 0), kw.get("gate_cols", (0, 0)),
                    kw.get("gate"), kw.get("residual"))
     return y, O.f64_to_bf16(y)
 
@@ -97,6 +107,10 @@ CASES = {
     "bias": dict(bias=True),
     "sigmoid": dict(gate_mode=1),
     "gated_residual": dict(gate_mode=2),
+    "rank16": dict(rank=16),
+    "rank32": dict(rank=32),
+    "rank64": dict(rank=64),
+    "all": dict(bias=True, rank=32, gate_mode=1),
 }
 
 
@@ -113,6 +127,10 @@ def test_nvfp4_linear_matches_oracle(case, M, N, K):
     if kw.get("gate_mode") == 2:
         kw["gate"] = I.gaussian_bf16(403, (N,), 1.0)
         kw["residual"] = I.gaussian_bf16(404, (M, N), 1.0)
+    rank = kw.pop("rank", 0)
+    if rank:
+        kw["l1"] = I.gaussian_bf16(405 + rank, (K, rank), 0.05)
+        kw["l2"] = I.gaussian_bf16(406 + rank, (rank, N), 0.05)
     y = run_linear(xb, wb, **kw)
     ref64, ref_bf16 = reference(xb, wb, **kw)
     check_output(y, ref64, ref_bf16)
@@ -127,3 +145,31 @@ def test_nvfp4_linear_small_m_sweep_shape():
     ref64, ref_bf16 = reference(xb, wb)
     stats = check_output(y, ref64, ref_bf16)
     assert stats["rel64"] < 5e-3
+
+
+def test_nvfp4_linear_low_rank_branch_is_added():
+    # the branch must change the output by exactly its own contribution (within tolerance):
+    # the same layer with L2 = 0 gives the plain result
+    M, N, K, r = 96, 256, 512, 32
+    xb = I.gaussian_bf16(420, (M, K), 1.0, 0.005, 30.0)
+    wb = I.gaussian_bf16(421, (N, K), 0.02)
+    l1 = I.gaussian_bf16(422, (K, r), 0.05)
+    zero = np.zeros((r, N), np.uint16)
+    assert np.array_equal(run_linear(xb, wb, l1=l1, l2=zero), run_linear(xb, wb))
+    l2 = I.gaussian_bf16(423, (r, N), 0.05)
+    y = run_linear(xb, wb, l1=l1, l2=l2)
+    ref64, ref_bf16 = reference(xb, wb, l1=l1, l2=l2)
+    check_output(y, ref64, ref_bf16)
+
+
+@pytest.mark.parametrize("r", [16, 32, 64])
+@pytest.mark.parametrize("M,K", [(1, 3072), (45, 256), (300, 1024)])
+def test_lowrank_down_alone(r, M, K):
+    xb = I.gaussian_bf16(430 + M, (M, K), 1.0, 0.005, 30.0)
+    l1b = I.gaussian_bf16(431 + r, (K, r), 0.01)
+    ld = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    R.rbd_lowrank_down(dev_bf16(xb), dev_bf16(np.ascontiguousarray(l1b.T)), ld)
+    assert R.rbd_check() == 0
+    ref = O.lowrank_down(xb, l1b)
+    err = np.abs(ld.float().cpu().numpy().astype(np.float64) - ref)
+    assert np.all(err <= np.abs(ref) * 2.0 ** -8 + 1e-4 * np.abs(ref).max())
