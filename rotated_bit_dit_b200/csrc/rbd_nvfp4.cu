@@ -211,11 +211,14 @@ constexpr uint32_t kNvSfBytes = 4 * 512;      // one scale stage (4 K steps)
 constexpr int kNvStages = 4;
 constexpr uint32_t kNvStageBytes = 2 * kNvOpBytes + 2 * kNvSfBytes;
 constexpr uint32_t kNvLrBytes = 2 * 128 * 128;  // low-rank tiles: l2t [128 x r] and ld [128 x r], r <= 64
-constexpr uint32_t kNvSmem = kNvStages * kNvStageBytes + kNvLrBytes + 1024 + 256;
+__host__ __device__ constexpr uint32_t nv_smem_bytes(bool lr) {
+  return kNvStages * kNvStageBytes + (lr ? kNvLrBytes : 0u) + 1024 + 256;
+}
 constexpr uint32_t kNvAccCols = 2 * kNvTile;  // two accumulator buffers
 constexpr uint32_t kNvLrCol = 384;            // low-rank accumulator (after the scale regions)
 }  // namespace
 
+template <bool LR>
 __global__ void __launch_bounds__(kNvThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                       const __grid_constant__ CUtensorMap tm_ld, const __grid_constant__ CUtensorMap tm_l2,
@@ -227,7 +230,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
   // low-rank tiles after the stages: l2t rows (A side) then ld rows (B side)
   unsigned char* lr_a = smem + kNvStages * kNvStageBytes;
   unsigned char* lr_b = lr_a + kNvLrBytes / 2;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kNvStages * kNvStageBytes + kNvLrBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kNvStages * kNvStageBytes + (LR ? kNvLrBytes : 0u));
   uint64_t* full = bars;
   uint64_t* empty = bars + kNvStages;
   uint64_t* tfull = bars + 2 * kNvStages;    // [2]
@@ -237,7 +240,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
   uint64_t* lrsempty = lrsfull + 1;          // low-rank MMAs done with them
   uint64_t* lrtempty = lrsempty + 1;         // epilogue has read the low-rank accumulator
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(lrtempty + 1);
-  const int R = args.r;
+  const int R = LR ? args.r : 0;
   const uint32_t warp = warp_id(), lane = lane_id();
   const int nks = args.K / kNvBK;
 
@@ -423,14 +426,17 @@ __global__ void __launch_bounds__(kNvThreads, 1)
   }
 }
 
-uint32_t nvfp4_gemm_smem_bytes() { return kNvSmem; }
+uint32_t nvfp4_gemm_smem_bytes() { return nv_smem_bytes(true); }
 
 cudaError_t launch_nvfp4_gemm(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const CUtensorMap& tm_ld,
                               const CUtensorMap& tm_l2, const NvArgs& a, int num_sms, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kNvSmem);
-  if (e != cudaSuccess) return e;
   const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
-  nvfp4_gemm_kernel<<<grid, kNvThreads, kNvSmem, st>>>(tm_x, tm_w, tm_ld, tm_l2, a);
+  const bool lr = a.r != 0;
+  auto kern = lr ? nvfp4_gemm_kernel<true> : nvfp4_gemm_kernel<false>;
+  const uint32_t smem = nv_smem_bytes(lr);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kNvThreads, smem, st>>>(tm_x, tm_w, tm_ld, tm_l2, a);
   return cudaGetLastError();
 }
 
