@@ -36,6 +36,9 @@ What it computes (plain, slow, float64 unless a step fixes the precision):
 7. Normalising prologue: RMSNorm and adaLN-style modulation ahead of the
    rotation.  Source: OrbitQuant W4A4 card, "Fused transformer" (the RMSNorm
    and modulation run in the activation quantisation prologues).
+8. INT4 KV-cache codec: packed codes with one float32 scale per token, head
+   and group, groups inside the 44 | 42 | 42 rotary bands.  Source: the Krea
+   Realtime 14B essay, Study 6 (the cache goes to four bits).
 
 Readings of points the pages leave open are listed where they are used.
 """
@@ -498,3 +501,65 @@ def nvfp4_linear(x_bits, w_bits, rot_group: int = GROUP) -> np.ndarray:
     xd = xq * np.repeat(xbs, 16, axis=1) * float(xgs)
     wd = wq * np.repeat(wbs, 16, axis=1) * float(wgs)
     return xd @ wd.T
+
+
+# ---------------------------------------------------------------------------
+# 8. INT4 KV-cache codec
+# ---------------------------------------------------------------------------
+# Source: "Krea Realtime 14B on one RTX 4090" essay, Study 6: the cache stores
+# int4 packed two values per byte with one scale per token, per head, per
+# rotary band; rotary splits the 128 channels of a head into bands of 44
+# (time), 42 (height) and 42 (width); groups are subdivided inside the bands
+# and never across them (three, six or twelve groups per head); reading
+# unpacks and scales in one pass.
+# Readings (the pages give the structure, not the arithmetic):
+#   - a band of b channels split into n groups is cut into contiguous runs whose
+#     sizes differ by at most one, the longer runs first;
+#   - each group is quantised like an activation row: amax, s = amax / 7,
+#     inv = 7 / amax (float32 IEEE divisions), q = clamp(rint(x * inv), -8, 7);
+#     an all-zero group gets s = 0 and q = 0; scales are stored as float32;
+#   - two codes per byte, the even channel in the low nibble;
+#   - reading gives RN_bf16(q * s), the product a float32 multiplication.
+
+KV_HEAD_DIM = 128
+KV_BANDS = (44, 42, 42)
+
+
+def kv4_group_sizes(groups_per_band: int) -> list:
+    """Group sizes along the 128 channels of a head, band by band."""
+    if groups_per_band not in (1, 2, 4):
+        raise ValueError("groups_per_band must be 1, 2 or 4")
+    sizes = []
+    for b in KV_BANDS:
+        base, extra = divmod(b, groups_per_band)
+        sizes += [base + 1 if i < extra else base for i in range(groups_per_band)]
+    return sizes
+
+
+def kv4_encode(x_bits: np.ndarray, groups_per_band: int):
+    """bf16 [T, H, 128] -> (packed uint8 [T, H, 64], scales float32 [T, H, G])."""
+    x = bf16_to_f64(x_bits).astype(np.float32)
+    t, h, d = x.shape
+    if d != KV_HEAD_DIM:
+        raise ValueError("head dimension must be 128")
+    sizes = kv4_group_sizes(groups_per_band)
+    q = np.zeros((t, h, d), dtype=np.int8)
+    scales = np.zeros((t, h, len(sizes)), dtype=np.float32)
+    c0 = 0
+    for gi, n in enumerate(sizes):
+        seg = x[:, :, c0:c0 + n].reshape(t * h, n)
+        qs, ss = quantize(seg, 4, 0)               # one group = one "row" of the activation quantiser
+        q[:, :, c0:c0 + n] = qs.reshape(t, h, n)
+        scales[:, :, gi] = ss.reshape(t, h)
+        c0 += n
+    packed = pack_int4(q.reshape(t * h, d)).reshape(t, h, d // 2)
+    return packed, scales
+
+
+def kv4_decode(packed: np.ndarray, scales: np.ndarray, groups_per_band: int) -> np.ndarray:
+    """(packed [T, H, 64], scales [T, H, G]) -> bf16 patterns [T, H, 128]."""
+    t, h, _ = packed.shape
+    q = unpack_int4(packed.reshape(t * h, -1)).reshape(t, h, KV_HEAD_DIM).astype(np.float32)
+    sizes = kv4_group_sizes(groups_per_band)
+    s = np.repeat(scales, sizes, axis=2).astype(np.float32)
+    return f64_to_bf16((q * s).astype(np.float32).astype(np.float64))

@@ -403,3 +403,49 @@ def test_norm_rot_quant_is_the_composition():
     q, s = O.norm_rot_quant(xb, 4, 256, 64, None, shift, None, 1e-6)
     q2, s2 = O.rot_quant(O.norm_modulate(xb, None, shift, None, 1e-6), 4, 256, 64)
     assert np.array_equal(q, q2) and np.array_equal(s, s2)
+
+
+# --------------------------------------------------------------- INT4 KV-cache codec
+def test_kv4_groups_follow_the_rotary_bands():
+    for n in (1, 2, 4):
+        sizes = O.kv4_group_sizes(n)
+        edges = set(np.cumsum([0] + sizes).tolist())
+        assert len(sizes) == 3 * n and sum(sizes) == 128
+        assert {0, 44, 86, 128} <= edges           # no group straddles the 44 | 42 | 42 split
+        assert max(sizes) - min(sizes) <= 1 + (44 - 42) // n
+
+
+def test_kv4_hand_worked_head():
+    # time band 7.0 -> scale 1, code 7; height band -3.5 -> scale 0.5, code -7; width band 0
+    x = np.zeros((1, 1, 128), np.float32)
+    x[0, 0, :44] = 7.0
+    x[0, 0, 44:86] = -3.5
+    xb = I.f32_to_bf16_bits(x)
+    packed, scales = O.kv4_encode(xb, 1)
+    assert scales.tolist() == [[[1.0, 0.5, 0.0]]]
+    assert np.all(packed[0, 0, :22] == 0x77) and np.all(packed[0, 0, 22:43] == 0x99)
+    assert np.all(packed[0, 0, 43:] == 0x00)
+    assert np.array_equal(O.kv4_decode(packed, scales, 1), xb)
+
+
+def test_kv4_band_isolation_and_error_bound():
+    xb = I.gaussian_bf16(50, (5, 3, 128), 1.0)
+    spiked = O.bf16_to_f64(xb).copy()
+    spiked[:, :, 60] *= 1000.0                       # inside the height band
+    sb = O.f64_to_bf16(spiked)
+    for n in (1, 2, 4):
+        p0, s0 = O.kv4_encode(xb, n)
+        p1, s1 = O.kv4_encode(sb, n)
+        sizes = O.kv4_group_sizes(n)
+        gh = np.searchsorted(np.cumsum(sizes), 60, side="right")   # the group holding channel 60
+        keep = [g for g in range(len(sizes)) if g != gh]
+        assert np.array_equal(s0[:, :, keep], s1[:, :, keep])
+        c0 = int(np.sum(sizes[:gh]))
+        q0 = O.unpack_int4(p0.reshape(15, 64)).reshape(5, 3, 128)
+        q1 = O.unpack_int4(p1.reshape(15, 64)).reshape(5, 3, 128)
+        outside = np.r_[0:c0, c0 + sizes[gh]:128]
+        assert np.array_equal(q0[:, :, outside], q1[:, :, outside])
+        # reconstruction within half a step (plus the bf16 rounding of the product)
+        y = O.bf16_to_f64(O.kv4_decode(p0, s0, n))
+        s = np.repeat(s0, sizes, axis=2)
+        assert np.all(np.abs(y - O.bf16_to_f64(xb)) <= s / 2 + np.abs(y) * 2.0 ** -8 + 1e-30)
