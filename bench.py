@@ -488,6 +488,57 @@ def run_prologue_sweep(args):
                 "timing": f"median of {args.steps} calls, each after a 256 MB L2 flush"}), flush=True)
 
 
+# ----------------------------------------------------------------------------- KV-cache codec
+def run_kv4_sweep(args):
+    """INT4 KV-cache codec at 16384 tokens x 40 heads x 128 channels (a 168 MB bf16 slice, beyond L2):
+    encode (slice write) and decode (slice read) for 3, 6 and 12 groups per head.  Each timed call
+    follows a 256 MB L2 flush; bytes = bf16 slice + codes + scales."""
+    import torch
+
+    import rotated_bit_dit_b200 as R
+    from rotated_bit_dit_b200 import _binding as B
+    from rotated_bit_dit_b200 import inputs as I
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    R.load()
+    peaks, src = load_peaks()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    T, H = 16384, 40
+    x = torch.from_numpy(np.ascontiguousarray(I.gaussian_bf16(9, (T, H * 128), 1.0, 0.01, 20.0)).view(np.int16))
+    x = x.view(torch.bfloat16).to(dev)
+    y = torch.empty_like(x)
+    for n in (1, 2, 4):
+        codes = torch.empty((T, H, 64), dtype=torch.uint8, device=dev)
+        scales = torch.empty((T, H, 3 * n), dtype=torch.float32, device=dev)
+        nbytes = T * H * (256 + 64 + 12 * n)
+        for op, fn in (("encode", lambda: B.rbd_kv4_encode(x, codes, scales, n)),
+                       ("decode", lambda: B.rbd_kv4_decode(codes, scales, y, n))):
+            for _ in range(max(args.warmup, 3)):
+                flush.zero_()
+                fn()
+            torch.cuda.synchronize()
+            assert R.rbd_check() == 0
+            ts = []
+            for _ in range(args.steps):
+                flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b) / 1e3)
+            assert R.rbd_check() == 0
+            t = statistics.median(ts)
+            gbs = nbytes / t / 1e9
+            print(json.dumps({
+                "sweep": "kv4", "op": op, "tokens": T, "heads": H, "groups_per_head": 3 * n, "us": t * 1e6,
+                "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "peak_source": f"{src} copy {peaks['hbm_gbs']} GB/s",
+                "algorithmic_bytes": nbytes, "timing": f"median of {args.steps} calls, each after a 256 MB L2 flush"}),
+                flush=True)
+
+
 # ----------------------------------------------------------------------------- 28-block stack
 STACK_LAYERS = (("wq", 3072, 3072), ("wk", 3072, 3072), ("wv", 3072, 3072), ("gate", 3072, 3072),
                 ("wo", 3072, 3072), ("mlp.gate", 3072, 12288), ("mlp.up", 3072, 12288), ("mlp.down", 12288, 3072))
@@ -595,7 +646,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--print-gemm-hash", action="store_true", help="print the GEMM source hash and exit")
-    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue"], default=None,
+    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4"], default=None,
                     help="instead of the headline line, print the small-token-count sweep (one line per case)")
     args = ap.parse_args()
     if args.print_gemm_hash:
@@ -609,6 +660,9 @@ def main():
         return
     if args.sweep == "prologue":
         run_prologue_sweep(args)
+        return
+    if args.sweep == "kv4":
+        run_kv4_sweep(args)
         return
     if args.impl == "reference" and int(os.environ.get("RANK", "0")) != 0:
         return                      # the oracle arm runs on rank 0 only; other ranks do no work

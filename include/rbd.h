@@ -255,6 +255,31 @@ rbd_status rbd_nvfp4_linear(const uint8_t* xq, const uint8_t* xbs, const float* 
                             int64_t M, int64_t N, int64_t K, const rbd_epilogue* epi,
                             void* y, int64_t ldy, void* stream);
 
+/* INT4 KV-cache codec ("Krea Realtime 14B on one RTX 4090" essay, Study 6:
+ * int4 packed two values per byte, one scale per token, per head, per rotary
+ * band; the 128 channels of a head split into rotary bands of 44, 42 and 42;
+ * groups subdivide the bands and never cross them; reading unpacks and scales
+ * in one pass).
+ *   groups_per_band n in {1, 2, 4}: 3, 6 or 12 groups per head; a band of b
+ *           channels is cut into n contiguous runs whose sizes differ by at
+ *           most one, longer runs first.
+ *   Per group, float32 IEEE: amax, s = amax / 7, inv = 7 / amax,
+ *   q = clamp(rint_even(x * inv), -8, 7); an all-zero group gets s = 0.
+ *   The cache is a ring of `capacity` token slots: input token t (0 <= t < T)
+ *   is slot (slot0 + t) mod capacity; T <= capacity, 0 <= slot0 < capacity.
+ *   codes   uint8 [capacity, H, 64], 16-byte aligned: byte i of a head holds
+ *           channel 2i in the low nibble, 2i + 1 in the high nibble.
+ *   scales  float32 [capacity, H, 3n].
+ *   x / y   bf16 [T, ldt] row-major, one row per token holding H heads of 128
+ *           channels (head h at h * 128); ldt >= 128 H, ldt % 8 == 0,
+ *           16-byte aligned.
+ * Encode writes the T slots; decode reads them back as RN_bf16(q * s).       */
+rbd_status rbd_kv4_encode(const void* x, int64_t T, int64_t H, int64_t ldt, int32_t groups_per_band,
+                          uint8_t* codes, float* scales, int64_t capacity, int64_t slot0, void* stream);
+rbd_status rbd_kv4_decode(const uint8_t* codes, const float* scales, int64_t capacity, int64_t slot0,
+                          int64_t T, int64_t H, int32_t groups_per_band, void* y, int64_t ldt,
+                          void* stream);
+
 /* Synchronises `stream`, then reports the first device-side error recorded
  * since the last rbd_check (RBD_ERR_DEVICE_TIMEOUT) or a CUDA error, and
  * clears the device status word.                                              */

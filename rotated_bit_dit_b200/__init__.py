@@ -28,5 +28,7 @@ from ._binding import (  # noqa: F401
     rbd_nvfp4_quant,
     rbd_nvfp4_quant_noalloc,
     rbd_nvfp4_linear,
+    rbd_kv4_encode,
+    rbd_kv4_decode,
 )
 from .layer import RotatedLowBitLinear  # noqa: F401

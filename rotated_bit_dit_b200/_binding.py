@@ -20,7 +20,7 @@ STATUS_NAMES = {0: "RBD_OK", 1: "RBD_ERR_INVALID_ARG", 2: "RBD_ERR_UNSUPPORTED",
 
 EXPORTED = ("rbd_rot_quant_act", "rbd_norm_rot_quant_act", "rbd_lowrank_fused", "rbd_lowrank_down", "rbd_pack_weights_int4", "rbd_pack_weights_int8",
             "rbd_w4a4_linear", "rbd_w8a8_linear", "rbd_nvfp4_scale_bytes", "rbd_nvfp4_quant",
-            "rbd_nvfp4_quant_noalloc", "rbd_nvfp4_linear", "rbd_check", "rbd_debug_timeout_probe", "rbd_status_string", "rbd_version")
+            "rbd_nvfp4_quant_noalloc", "rbd_nvfp4_linear", "rbd_kv4_encode", "rbd_kv4_decode", "rbd_check", "rbd_debug_timeout_probe", "rbd_status_string", "rbd_version")
 
 
 class RbdError(RuntimeError):
@@ -71,6 +71,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "rbd_nvfp4_quant": [vp, i64, i64, i64, i32, vp, vp, vp, vp, vp],
         "rbd_nvfp4_quant_noalloc": [vp, i64, i64, i64, i32, vp, vp, vp, vp],
         "rbd_nvfp4_linear": [vp, vp, vp, vp, vp, vp, i64, i64, i64, ctypes.POINTER(Epilogue), vp, i64, vp],
+        "rbd_kv4_encode": [vp, i64, i64, i64, i32, vp, vp, i64, i64, vp],
+        "rbd_kv4_decode": [vp, vp, i64, i64, i64, i64, i32, vp, i64, vp],
         "rbd_check": [vp],
         "rbd_debug_timeout_probe": [i64, vp],
     }
@@ -269,3 +271,22 @@ def rbd_status_string(status: int) -> str:
 
 def rbd_version() -> str:
     return load().rbd_version().decode()
+
+
+def rbd_kv4_encode(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, groups_per_band: int = 1,
+                   slot0: int = 0, stream=None) -> None:
+    """x bf16 [T, H*128] (row stride may be larger) -> cache slots (slot0 + t) mod capacity of
+    codes uint8 [capacity, H, 64] and scales float32 [capacity, H, 3*groups_per_band]."""
+    T = x.shape[0]
+    capacity, H = codes.shape[0], codes.shape[1]
+    _ok(load().rbd_kv4_encode(_ptr(x), T, H, _rowstride(x), groups_per_band, _ptr(codes), _ptr(scales),
+                              capacity, slot0, _stream(stream)), "rbd_kv4_encode")
+
+
+def rbd_kv4_decode(codes: torch.Tensor, scales: torch.Tensor, y: torch.Tensor, groups_per_band: int = 1,
+                   slot0: int = 0, stream=None) -> None:
+    """Cache slots (slot0 + t) mod capacity, t < y.shape[0] -> y bf16 [T, H*128]."""
+    T = y.shape[0]
+    capacity, H = codes.shape[0], codes.shape[1]
+    _ok(load().rbd_kv4_decode(_ptr(codes), _ptr(scales), capacity, slot0, T, H, groups_per_band, _ptr(y),
+                              _rowstride(y), _stream(stream)), "rbd_kv4_decode")

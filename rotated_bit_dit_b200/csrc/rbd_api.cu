@@ -228,6 +228,23 @@ __global__ void timeout_probe_kernel(int64_t timeout_ns) {
 
 }  // namespace
 
+namespace {
+rbd_status kv4_validate(int64_t T, int64_t H, int64_t ldt, int32_t n, const void* x, const void* codes,
+                        const float* scales, int64_t capacity, int64_t slot0) {
+  if (n != 1 && n != 2 && n != 4) return RBD_ERR_UNSUPPORTED;
+  if (T < 0 || H <= 0 || capacity <= 0) return RBD_ERR_INVALID_ARG;
+  // 32-bit unit indices, with room for a warp's units past the end
+  if (H > 65536 || T > ((int64_t)INT32_MAX - 64) / H || capacity > (int64_t)INT32_MAX / H) return RBD_ERR_UNSUPPORTED;
+  if (T > capacity || slot0 < 0 || slot0 >= capacity) return RBD_ERR_INVALID_ARG;
+  if (T == 0) return RBD_OK;
+  if (!x || !codes || !scales) return RBD_ERR_INVALID_ARG;
+  if (ldt < H * 128) return RBD_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || (ldt % 8) != 0 || (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return RBD_ERR_ALIGNMENT;
+  return RBD_OK;
+}
+}  // namespace
+
 extern "C" {
 
 rbd_status rbd_rot_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, rbd_qcfg cfg, int8_t* codes,
@@ -281,6 +298,24 @@ rbd_status rbd_lowrank_down(const void* x, int64_t M, int64_t K, int64_t ldx, co
   return cuda_status(rbd::launch_lowrank_down(static_cast<const uint16_t*>(x), M, K, ldx,
                                               static_cast<const uint16_t*>(l1t), r, static_cast<uint16_t*>(ld),
                                               as_stream(stream)));
+}
+
+rbd_status rbd_kv4_encode(const void* x, int64_t T, int64_t H, int64_t ldt, int32_t groups_per_band,
+                          uint8_t* codes, float* scales, int64_t capacity, int64_t slot0, void* stream) {
+  rbd_status s = kv4_validate(T, H, ldt, groups_per_band, x, codes, scales, capacity, slot0);
+  if (s != RBD_OK || T == 0) return s;
+  return cuda_status(rbd::launch_kv4_encode(static_cast<const uint16_t*>(x), static_cast<int>(T),
+                                            static_cast<int>(H), ldt, groups_per_band, codes, scales, capacity,
+                                            slot0, as_stream(stream)));
+}
+
+rbd_status rbd_kv4_decode(const uint8_t* codes, const float* scales, int64_t capacity, int64_t slot0, int64_t T,
+                          int64_t H, int32_t groups_per_band, void* y, int64_t ldt, void* stream) {
+  rbd_status s = kv4_validate(T, H, ldt, groups_per_band, y, codes, scales, capacity, slot0);
+  if (s != RBD_OK || T == 0) return s;
+  return cuda_status(rbd::launch_kv4_decode(codes, scales, capacity, slot0, static_cast<int>(T),
+                                            static_cast<int>(H), groups_per_band, static_cast<uint16_t*>(y), ldt,
+                                            as_stream(stream)));
 }
 
 rbd_status rbd_pack_weights_int4(const void* w, int64_t N, int64_t K, rbd_qcfg cfg, uint8_t* packed, float* scales,

@@ -70,6 +70,12 @@ cudaError_t launch_nvfp4_gemm(const CUtensorMap& tm_x, const CUtensorMap& tm_w, 
                               const CUtensorMap& tm_l2, const NvArgs& a, int num_sms, cudaStream_t st);
 uint32_t nvfp4_gemm_smem_bytes();
 
+// INT4 KV-cache codec (n = groups per rotary band: 1, 2 or 4).
+cudaError_t launch_kv4_encode(const uint16_t* x, int T, int H, int64_t ldt, int n, uint8_t* codes, float* scales,
+                              int64_t capacity, int64_t slot0, cudaStream_t st);
+cudaError_t launch_kv4_decode(const uint8_t* codes, const float* scales, int64_t capacity, int64_t slot0, int T,
+                              int H, int n, uint16_t* y, int64_t ldt, cudaStream_t st);
+
 uint32_t gemm_smem_bytes(bool g64, int r, int G);   // dynamic shared memory of one GEMM CTA
 int gemm_tile_tokens(bool g64);                     // tokens per GEMM tile
 

@@ -5,3 +5,4 @@
 #include "rbd_prologue.cu"
 #include "rbd_gemm.cu"
 #include "rbd_nvfp4.cu"
+#include "rbd_kv4.cu"

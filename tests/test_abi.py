@@ -169,3 +169,18 @@ def test_lowrank_down_validation_without_gpu():
     assert lib.rbd_lowrank_down(FAKE, 4, 256, 128, FAKE, 32, FAKE, None) == 1      # ldx < K
     assert lib.rbd_lowrank_down(FAKE_MIS, 4, 256, 256, FAKE, 32, FAKE, None) == 3
     assert lib.rbd_lowrank_down(FAKE, 0, 256, 256, null, 32, null, None) == 0      # empty batch
+
+
+def test_kv4_validation_without_gpu():
+    lib = R.load()
+    null = ctypes.c_void_p(0)
+    enc, dec = lib.rbd_kv4_encode, lib.rbd_kv4_decode
+    assert enc(FAKE, 4, 2, 256, 3, FAKE, FAKE, 8, 0, None) == 2          # groups per band
+    assert enc(FAKE, 9, 2, 256, 1, FAKE, FAKE, 8, 0, None) == 1          # slice longer than the ring
+    assert enc(FAKE, 4, 2, 256, 1, FAKE, FAKE, 8, 8, None) == 1          # slot0 outside the ring
+    assert enc(FAKE, 4, 2, 200, 1, FAKE, FAKE, 8, 0, None) == 1          # ldt < 128 H
+    assert enc(FAKE_MIS, 4, 2, 256, 1, FAKE, FAKE, 8, 0, None) == 3
+    assert enc(FAKE, 4, 2, 260, 1, FAKE, FAKE, 8, 0, None) == 3          # row stride not 16-byte aligned
+    assert enc(FAKE, 0, 2, 256, 1, null, null, 8, 0, None) == 0          # empty slice
+    assert dec(FAKE, FAKE, 8, 0, 4, 0, 1, FAKE, 256, None) == 1          # no heads
+    assert dec(null, FAKE, 8, 0, 4, 2, 1, FAKE, 256, None) == 1
