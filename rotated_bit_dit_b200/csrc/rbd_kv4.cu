@@ -19,6 +19,8 @@
 // the low nibble of byte i), scales [capacity][H][3 n] float32.
 // Thread mapping: a warp handles a few (token, head) units; lane l owns
 // channels 4l .. 4l+3 of each (one 8-byte access).
+#include <cuda_bf16.h>
+
 #include "rbd_common.cuh"
 #include "rbd_internal.cuh"
 
@@ -28,7 +30,6 @@ namespace {
 
 constexpr int kKvDim = 128;
 constexpr int kKvWarps = 8;
-constexpr int kKvUnits = 4;   // (token, head) units per warp
 
 // Group of channel c when every band is cut into N groups.
 template <int N>
@@ -45,72 +46,110 @@ __device__ __forceinline__ int kv4_group_of(int c) {
 
 }  // namespace
 
+// Units per warp, and rounds of 32 (unit, group) pairs: pair p = u * G + g
+// lives on lane p % 32 in round p / 32, which does that pair's divisions.
+__host__ __device__ constexpr int kv4_units(int n) { return n == 1 ? 8 : (n == 2 ? 5 : 4); }
+__host__ __device__ constexpr int kv4_rounds(int n) { return (kv4_units(n) * 3 * n + 31) / 32; }
+
+// Value of pair p (held on lane p % 32 in round p / 32), for every lane.
+template <int R>
+__device__ __forceinline__ float kv4_pair_value(const float (&v)[R], int p) {
+  float r = __shfl_sync(0xffffffffu, v[0], p & 31);
+#pragma unroll
+  for (int k = 1; k < R; ++k) {
+    const float o = __shfl_sync(0xffffffffu, v[k], p & 31);
+    if ((p >> 5) == k) r = o;
+  }
+  return r;
+}
+
 // A group has at least 10 channels, so the 4 channels of a lane belong to at
-// most two groups (ga, and gb = ga or ga + 1).  Each warp handles kKvUnits
-// consecutive (token, head) units and issues all their loads first.
+// most two groups (ga, and gb = ga or ga + 1).  A warp handles U consecutive
+// (token, head) units and issues all their loads first; then the group maxima
+// of every unit (one redux.sync per group), one inverse and one scale per
+// (unit, group) on its own lane, and the codes with the inverses shuffled in.
 template <int N>
 __global__ void __launch_bounds__(kKvWarps * 32) kv4_encode_kernel(const uint16_t* __restrict__ x, int T, int H,
                                                                    int64_t ldt, uint8_t* __restrict__ codes,
                                                                    float* __restrict__ scales, int64_t capacity,
                                                                    int64_t slot0) {
   constexpr int G = 3 * N;
+  constexpr int U = kv4_units(N);
   const int lane = threadIdx.x & 31;
   const int total = T * H;
-  const int unit0 = (blockIdx.x * kKvWarps + (threadIdx.x >> 5)) * kKvUnits;
+  const int unit0 = (blockIdx.x * kKvWarps + (threadIdx.x >> 5)) * U;
   const int ga = kv4_group_of<N>(4 * lane), gb = kv4_group_of<N>(4 * lane + 3);
   bool in_b[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) in_b[j] = kv4_group_of<N>(4 * lane + j) != ga;
-  // the first unit's token and head; later units step through the heads
-  int t = unit0 / H, h = unit0 - t * H;
-  uint2 raw[kKvUnits];
-  int64_t dst[kKvUnits];   // (slot * H + h) of each unit
+  uint2 raw[U];
+  int64_t dst[U];   // (slot * H + h) of each unit
   {
-    int tt = t, hh = h;
+    int tt = unit0 / H, hh = unit0 - tt * H;
 #pragma unroll
-    for (int u = 0; u < kKvUnits; ++u) {
+    for (int u = 0; u < U; ++u) {
       if (unit0 + u < total) {
         raw[u] = *reinterpret_cast<const uint2*>(x + (int64_t)tt * ldt + (int64_t)hh * kKvDim + 4 * lane);
         int64_t slot = slot0 + tt;               // < 2 capacity: one wrap at most
         if (slot >= capacity) slot -= capacity;
         dst[u] = slot * H + hh;
+      } else {
+        raw[u] = make_uint2(0u, 0u);
       }
       if (++hh == H) { hh = 0; ++tt; }
     }
   }
+  // group maxima; pair u * G + g keeps that of (unit u, group g).  Float bit
+  // patterns of non-negative values order like unsigned integers.
+  constexpr int R = kv4_rounds(N);
+  uint32_t amax_lane[R];
 #pragma unroll
-  for (int u = 0; u < kKvUnits; ++u) {
-    if (unit0 + u >= total) break;   // uniform across the warp
-    const float v[4] = {__uint_as_float(raw[u].x << 16), __uint_as_float(raw[u].x & 0xFFFF0000u),
-                        __uint_as_float(raw[u].y << 16), __uint_as_float(raw[u].y & 0xFFFF0000u)};
-    // the lane's maxima in its (at most) two groups; float bit patterns of
-    // non-negative values order like unsigned integers
+  for (int k = 0; k < R; ++k) amax_lane[k] = 0u;
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
     uint32_t ma = 0u, mb = 0u;
+    const uint32_t w[4] = {raw[u].x << 16, raw[u].x & 0xFFFF0000u, raw[u].y << 16, raw[u].y & 0xFFFF0000u};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t a = __float_as_uint(fabsf(v[j]));
+      const uint32_t a = w[j] & 0x7FFFFFFFu;     // |x|
       if (in_b[j]) mb = max(mb, a); else ma = max(ma, a);
     }
-    uint32_t amax_a = 0u, amax_b = 0u, amax_mine = 0u;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const uint32_t r = __reduce_max_sync(0xffffffffu, g == ga ? ma : (g == gb ? mb : 0u));
-      if (g == ga) amax_a = r;
-      if (g == gb) amax_b = r;
-      if (g == lane) amax_mine = r;
+      if (lane == (u * G + g) % 32) amax_lane[(u * G + g) / 32] = r;
     }
-    const float fa = __uint_as_float(amax_a), fb = __uint_as_float(amax_b);
-    const float inv_a = fa > 0.f ? __fdiv_rn(7.f, fa) : 0.f;
-    const float inv_b = gb == ga ? inv_a : (fb > 0.f ? __fdiv_rn(7.f, fb) : 0.f);
+  }
+  float inv_lane[R], s_lane[R];
+#pragma unroll
+  for (int k = 0; k < R; ++k) {
+    const float fa = __uint_as_float(amax_lane[k]);
+    inv_lane[k] = fa > 0.f ? __fdiv_rn(7.f, fa) : 0.f;
+    s_lane[k] = __fdiv_rn(fa, 7.f);
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    if (unit0 + u >= total) break;   // uniform across the warp
+    const float inv_a = kv4_pair_value<R>(inv_lane, u * G + ga);
+    const float inv_b = kv4_pair_value<R>(inv_lane, u * G + gb);
+    const float v[4] = {__uint_as_float(raw[u].x << 16), __uint_as_float(raw[u].x & 0xFFFF0000u),
+                        __uint_as_float(raw[u].y << 16), __uint_as_float(raw[u].y & 0xFFFF0000u)};
+    // rint to even by adding 1.5 * 2^23 (exact for |x * inv| < 2^22; here
+    // |x * inv| <= 7): the low bits of the sum are the two's-complement code
     uint32_t packed = 0u;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      int q = __float2int_rn(__fmul_rn(v[j], in_b[j] ? inv_b : inv_a));
+      const float p = __fmul_rn(v[j], in_b[j] ? inv_b : inv_a);
+      int q = static_cast<int>(__float_as_uint(__fadd_rn(p, 12582912.0f)) - 0x4B400000u);
       q = q > 7 ? 7 : (q < -8 ? -8 : q);
-      packed |= (static_cast<uint32_t>(q) & 0xFu) << (4 * j);
+      packed += (static_cast<uint32_t>(q) & 0xFu) << (4 * j);
     }
     *reinterpret_cast<uint16_t*>(codes + dst[u] * (kKvDim / 2) + 2 * lane) = static_cast<uint16_t>(packed);
-    if (lane < G) scales[dst[u] * G + lane] = __fdiv_rn(__uint_as_float(amax_mine), 7.f);
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      const int p = lane + 32 * k;   // this lane's pair in round k
+      if (p >= u * G && p < u * G + G) scales[dst[u] * G + (p - u * G)] = s_lane[k];
+    }
   }
 }
 
@@ -120,47 +159,53 @@ __global__ void __launch_bounds__(kKvWarps * 32) kv4_decode_kernel(const uint8_t
                                                                    int64_t capacity, int64_t slot0, int T, int H,
                                                                    uint16_t* __restrict__ y, int64_t ldt) {
   constexpr int G = 3 * N;
+  constexpr int U = kv4_units(N);
   const int lane = threadIdx.x & 31;
   const int total = T * H;
-  const int unit0 = (blockIdx.x * kKvWarps + (threadIdx.x >> 5)) * kKvUnits;
+  const int unit0 = (blockIdx.x * kKvWarps + (threadIdx.x >> 5)) * U;
   const int ga = kv4_group_of<N>(4 * lane), gb = kv4_group_of<N>(4 * lane + 3);
   bool in_b[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) in_b[j] = kv4_group_of<N>(4 * lane + j) != ga;
-  uint32_t pk[kKvUnits];
-  float sc[kKvUnits];
-  int64_t dst[kKvUnits];   // output element offset of each unit
+  uint32_t pk[U];
+  int64_t dst[U];   // output element offset of each unit
+  constexpr int R = kv4_rounds(N);
+  float s_lane[R];   // pair u * G + g: scale of (unit u, group g)
+#pragma unroll
+  for (int k = 0; k < R; ++k) s_lane[k] = 0.f;
   {
     int tt = unit0 / H, hh = unit0 - tt * H;
 #pragma unroll
-    for (int u = 0; u < kKvUnits; ++u) {
+    for (int u = 0; u < U; ++u) {
       if (unit0 + u < total) {
         int64_t slot = slot0 + tt;               // < 2 capacity: one wrap at most
         if (slot >= capacity) slot -= capacity;
         const int64_t src = slot * H + hh;
         pk[u] = *reinterpret_cast<const uint16_t*>(codes + src * (kKvDim / 2) + 2 * lane);
-        sc[u] = lane < G ? __ldg(scales + src * G + lane) : 0.f;
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+          const int p = lane + 32 * k;
+          if (p >= u * G && p < u * G + G) s_lane[k] = __ldg(scales + src * G + (p - u * G));
+        }
         dst[u] = (int64_t)tt * ldt + (int64_t)hh * kKvDim;
       }
       if (++hh == H) { hh = 0; ++tt; }
     }
   }
 #pragma unroll
-  for (int u = 0; u < kKvUnits; ++u) {
+  for (int u = 0; u < U; ++u) {
     if (unit0 + u >= total) break;   // uniform across the warp
-    const float sa = __shfl_sync(0xffffffffu, sc[u], ga), sb = __shfl_sync(0xffffffffu, sc[u], gb);
-    uint32_t out[2];
+    const float sa = kv4_pair_value<R>(s_lane, u * G + ga), sb = kv4_pair_value<R>(s_lane, u * G + gb);
+    // q as a float without a conversion: the bits of 1.5 * 2^23 + q, minus 1.5 * 2^23 (exact)
+    float f[4];
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      uint32_t half[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int j = 2 * k + e;
-        const int q = static_cast<int>(static_cast<int32_t>(pk[u] << (28 - 4 * j)) >> 28);   // sign-extend nibble j
-        half[e] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(static_cast<float>(q), in_b[j] ? sb : sa)));
-      }
-      out[k] = half[0] | (half[1] << 16);
+    for (int j = 0; j < 4; ++j) {
+      const int q = static_cast<int>(static_cast<int32_t>(pk[u] << (28 - 4 * j)) >> 28);   // sign-extend nibble j
+      f[j] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B400000u + static_cast<uint32_t>(q)), 12582912.0f),
+                       in_b[j] ? sb : sa);
     }
+    const __nv_bfloat162 b01 = __floats2bfloat162_rn(f[0], f[1]), b23 = __floats2bfloat162_rn(f[2], f[3]);
+    const uint32_t out[2] = {*reinterpret_cast<const uint32_t*>(&b01), *reinterpret_cast<const uint32_t*>(&b23)};
     *reinterpret_cast<uint2*>(y + dst[u] + 4 * lane) = make_uint2(out[0], out[1]);
   }
 }
@@ -168,7 +213,7 @@ __global__ void __launch_bounds__(kKvWarps * 32) kv4_decode_kernel(const uint8_t
 cudaError_t launch_kv4_encode(const uint16_t* x, int T, int H, int64_t ldt, int n, uint8_t* codes, float* scales,
                               int64_t capacity, int64_t slot0, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  const int64_t per_block = (int64_t)kKvWarps * kKvUnits;
+  const int64_t per_block = (int64_t)kKvWarps * kv4_units(n);
   const dim3 grid(static_cast<unsigned>(((int64_t)T * H + per_block - 1) / per_block));
   switch (n) {
     case 1: kv4_encode_kernel<1><<<grid, kKvWarps * 32, 0, st>>>(x, T, H, ldt, codes, scales, capacity, slot0); break;
@@ -182,7 +227,7 @@ cudaError_t launch_kv4_encode(const uint16_t* x, int T, int H, int64_t ldt, int 
 cudaError_t launch_kv4_decode(const uint8_t* codes, const float* scales, int64_t capacity, int64_t slot0, int T,
                               int H, int n, uint16_t* y, int64_t ldt, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  const int64_t per_block = (int64_t)kKvWarps * kKvUnits;
+  const int64_t per_block = (int64_t)kKvWarps * kv4_units(n);
   const dim3 grid(static_cast<unsigned>(((int64_t)T * H + per_block - 1) / per_block));
   switch (n) {
     case 1: kv4_decode_kernel<1><<<grid, kKvWarps * 32, 0, st>>>(codes, scales, capacity, slot0, T, H, y, ldt); break;
