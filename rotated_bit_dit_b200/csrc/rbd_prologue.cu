@@ -24,10 +24,6 @@ namespace {
 
 constexpr int kTeam = 16;  // threads per 256-block
 
-struct QuantParams {
-  float qmax;
-};
-
 __device__ __forceinline__ int quant1(float v, float inv, float qmax) {
   const float t = __fmul_rn(v, inv);
   int q = __float2int_rn(t);
