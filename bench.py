@@ -255,22 +255,18 @@ def run_ours(args, cfg, t):
     value = whole_job_rate(world, args.steps, ops_step, t_max) / 1e12
     tokens_s = whole_job_rate(world, args.steps, M, t_max)
 
-    # ---- end to end through the public layer call with host buffers
+    # ---- end to end through the public layer call with host buffers: forward_host streams
+    # 1024-token slices through two CUDA streams so the copies overlap the kernels
     xh = torch.from_numpy(np.ascontiguousarray(t["x"]).view(np.int16)).view(torch.bfloat16).pin_memory()
     yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    xd = torch.empty_like(x)
     e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     for _ in range(2):
-        xd.copy_(xh, non_blocking=True)
-        layer(xd, out=out)
-        yh.copy_(out, non_blocking=True)
+        layer.forward_host(xh, yh)
     torch.cuda.synchronize()
     for i in range(args.steps):
         flush.zero_()
         e2e_ev[i][0].record()
-        xd.copy_(xh, non_blocking=True)
-        layer(xd, out=out)
-        yh.copy_(out, non_blocking=True)
+        layer.forward_host(xh, yh)
         e2e_ev[i][1].record()
     torch.cuda.synchronize()
     e2e_t = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / 1e3, dev)
@@ -303,7 +299,9 @@ def run_ours(args, cfg, t):
                                   "unit": "GB/s", "frac": pro_bytes / pro_s / 1e9 / peaks["hbm_gbs"],
                                   "algorithmic_bytes": pro_bytes},
             "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": int(xh.numel() * 2),
-                    "d2h_bytes_per_step": int(yh.numel() * 2)},
+                    "d2h_bytes_per_step": int(yh.numel() * 2),
+                    "call": "RotatedLowBitLinear.forward_host: pinned host X in, Y out, 1024-token slices on "
+                            "two streams (copies overlap the kernels)"},
             "gpu_launches": 2 * args.steps,   # fused prologue + GEMM per step
             "clocks": clk.summary(),
         }

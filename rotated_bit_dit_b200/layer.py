@@ -58,8 +58,11 @@ class RotatedLowBitLinear:
 
     def __call__(self, x: torch.Tensor, residual: Optional[torch.Tensor] = None,
                  out: Optional[torch.Tensor] = None, acc_debug: Optional[torch.Tensor] = None) -> torch.Tensor:
+        codes, sx, ld = self.buffers(x.shape[0], x.device)
+        return self._run(x, codes, sx, ld, residual, out, acc_debug)
+
+    def _run(self, x, codes, sx, ld, residual=None, out=None, acc_debug=None) -> torch.Tensor:
         M = x.shape[0]
-        codes, sx, ld = self.buffers(M, x.device)
         if self.rank:
             B.rbd_lowrank_fused(x, codes, sx, self.l1t, ld, self.bits, self.rot_group, self.scale_group)
         else:
@@ -71,3 +74,51 @@ class RotatedLowBitLinear:
         fn = B.rbd_w4a4_linear if self.bits == 4 else B.rbd_w8a8_linear
         fn(codes, sx, self.wq, self.sw, out, self.scale_group, epi, self.rot_group)
         return out
+
+    def forward_host(self, xh: torch.Tensor, yh: torch.Tensor, residual_h: Optional[torch.Tensor] = None,
+                     chunk: int = 1024, device=None) -> torch.Tensor:
+        """The layer on host-resident tokens: xh bf16 [M, K] and yh bf16 [M, N] in pinned host memory
+        (residual_h likewise [M, N] for the gated residual).  Tokens are independent, so the call
+        streams `chunk`-token slices through two CUDA streams: the host-to-device copy of slice i + 1
+        and the device-to-host copy of slice i - 1 run on the copy engines while slice i computes.
+        Every output element is computed exactly as by __call__ (bit-identical).  Ordered after the
+        work already queued on the current stream; the current stream waits for the result."""
+        if not (xh.is_pinned() and yh.is_pinned()) or (residual_h is not None and not residual_h.is_pinned()):
+            raise ValueError("host tensors must be pinned")
+        dev = torch.device(device) if device is not None else self.wq.device
+        M = xh.shape[0]
+        cur = torch.cuda.current_stream(dev)
+        streams = [torch.cuda.Stream(device=dev) for _ in range(2)]
+        start = torch.cuda.Event()
+        start.record(cur)
+        G = self.K // 64 if self.scale_group else 1
+        staged = []   # per stream: its own input, output, residual and intermediate buffers
+        for s in streams:
+            s.wait_event(start)
+            bufs = (torch.empty((chunk, self.K), dtype=torch.bfloat16, device=dev),
+                    torch.empty((chunk, self.N), dtype=torch.bfloat16, device=dev),
+                    torch.empty((chunk, self.N), dtype=torch.bfloat16, device=dev) if residual_h is not None else None,
+                    torch.empty((chunk, self.K), dtype=torch.int8, device=dev),
+                    torch.empty((chunk, G) if self.scale_group else (chunk,), dtype=torch.float32, device=dev),
+                    torch.empty((chunk, self.rank), dtype=torch.bfloat16, device=dev) if self.rank else None)
+            staged.append(bufs)
+        for i, m0 in enumerate(range(0, M, chunk)):
+            m = min(M, m0 + chunk) - m0
+            s = streams[i % 2]
+            xd, yd, rd, codes, sx, ld = staged[i % 2]
+            with torch.cuda.stream(s):
+                xd[:m].copy_(xh[m0:m0 + m], non_blocking=True)
+                r = None
+                if rd is not None:
+                    rd[:m].copy_(residual_h[m0:m0 + m], non_blocking=True)
+                    r = rd[:m]
+                self._run(xd[:m], codes[:m], sx[:m], ld[:m] if ld is not None else None, r, yd[:m])
+                yh[m0:m0 + m].copy_(yd[:m], non_blocking=True)
+        for s in streams:
+            cur.wait_stream(s)
+        # the staging buffers stay alive until the streams are done with them
+        for s, bufs in zip(streams, staged):
+            for t in bufs:
+                if t is not None:
+                    t.record_stream(s)
+        return yh

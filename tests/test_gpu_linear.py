@@ -137,3 +137,20 @@ def test_w4a4_qkvg_config_sampled_rows():
     ref = reference(case, rows=rows)
     stats = check_output(y[rows], ref["ref64"], ref["ref_bf16"])
     assert stats["rel64"] < 5e-3
+
+
+@pytest.mark.parametrize("bits,sg,rank,gate_mode", [(4, 64, 32, 1), (8, 0, 0, 2), (4, 0, 16, 0)])
+def test_forward_host_matches_the_device_call(bits, sg, rank, gate_mode):
+    # host-resident tokens streamed in chunks (ragged last chunk) give the device call's output bit for bit
+    case = build_case(1000, 256, 512, bits, sg, seed=60, rank=rank, bias=True, gate_mode=gate_mode,
+                      gate_cols=(128, 256))
+    y_dev, _, layer = run_layer(case)
+    xh = torch.from_numpy(np.ascontiguousarray(case["x"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty((1000, 256), dtype=torch.bfloat16).pin_memory()
+    rh = None
+    if case["residual"] is not None:
+        rh = torch.from_numpy(np.ascontiguousarray(case["residual"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+    layer.forward_host(xh, yh, rh, chunk=384)
+    torch.cuda.synchronize()
+    assert R.rbd_check() == 0
+    assert np.array_equal(yh.view(torch.int16).numpy().view(np.uint16), y_dev)
