@@ -255,7 +255,7 @@ rbd_status rbd_nvfp4_linear(const uint8_t* xq, const uint8_t* xbs, const float* 
                             int64_t M, int64_t N, int64_t K, const rbd_epilogue* epi,
                             void* y, int64_t ldy, void* stream);
 
-/* INT4 KV-cache codec ("Krea Realtime 14B on one RTX 4090" essay, Study 6:
+/* INT4 KV-cache codec ("lab", Study 6, "The cache becomes the model":
  * int4 packed two values per byte, one scale per token, per head, per rotary
  * band; the 128 channels of a head split into rotary bands of 44, 42 and 42;
  * groups subdivide the bands and never cross them; reading unpacks and scales

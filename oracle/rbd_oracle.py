@@ -37,8 +37,8 @@ What it computes (plain, slow, float64 unless a step fixes the precision):
    rotation.  Source: OrbitQuant W4A4 card, "Fused transformer" (the RMSNorm
    and modulation run in the activation quantisation prologues).
 8. INT4 KV-cache codec: packed codes with one float32 scale per token, head
-   and group, groups inside the 44 | 42 | 42 rotary bands.  Source: the Krea
-   Realtime 14B essay, Study 6 (the cache goes to four bits).
+   and group, groups inside the 44 | 42 | 42 rotary bands.  Source: "lab",
+   Study 6 (the cache goes to four bits).
 
 Readings of points the pages leave open are listed where they are used.
 """
@@ -506,7 +506,7 @@ def nvfp4_linear(x_bits, w_bits, rot_group: int = GROUP) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # 8. INT4 KV-cache codec
 # ---------------------------------------------------------------------------
-# Source: "Krea Realtime 14B on one RTX 4090" essay, Study 6: the cache stores
+# Source: "lab", Study 6 ("The cache becomes the model"): the cache stores
 # int4 packed two values per byte with one scale per token, per head, per
 # rotary band; rotary splits the 128 channels of a head into bands of 44
 # (time), 42 (height) and 42 (width); groups are subdivided inside the bands

@@ -2,7 +2,7 @@
 // key or value cache with one float32 scale per token, head and group, the
 // groups lying inside the rotary bands of the head.
 //
-// Method: "Krea Realtime 14B on one RTX 4090" essay, Study 6: the cache stores
+// Method: "lab", Study 6 ("The cache becomes the model"): the cache stores
 // int4 packed two values per byte with one scale per token, per head, per
 // rotary band; rotary splits the 128 channels of a head into bands of 44, 42
 // and 42; finer groups are cut inside the bands, never across them; reading
