@@ -6,6 +6,12 @@ W4A4 GEMM with group-64 dequant, rank-32 branch and sigmoid gate epilogue
 (the grouped Q|K|V|gate projection, M=4096 tokens, K=3072, N=4*3072).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --sweep small-m|stack|prologue|kv4   (one JSON line per case)
+
+Sweeps: small-m (K = N = 3072 layer at 1..1024 tokens, W4A4 and NVFP4, HBM
+roofline), stack (the 28-block stack of 224 linears), prologue (the
+activation prologues at the layer shapes, HBM roofline), kv4 (the INT4
+KV-cache codec, HBM roofline).
 
 Under torchrun each rank runs its own replica on its own batch (tokens are
 independent; no collective on the data path), scaling is weak and the value
