@@ -153,60 +153,65 @@ __global__ void __launch_bounds__(kKvWarps * 32) kv4_encode_kernel(const uint16_
   }
 }
 
+// Decode: a half-warp per (token, head) unit, lane i of the half owning
+// channels 8i .. 8i+7 (4 bytes of codes in, one 16-byte store out); the 8
+// channels touch at most two groups, whose scales lanes i < G of the half
+// load and shuffle.  A warp handles 2 * kKvDecSteps units.
+constexpr int kKvDecSteps = 4;
+
 template <int N>
 __global__ void __launch_bounds__(kKvWarps * 32) kv4_decode_kernel(const uint8_t* __restrict__ codes,
                                                                    const float* __restrict__ scales,
                                                                    int64_t capacity, int64_t slot0, int T, int H,
                                                                    uint16_t* __restrict__ y, int64_t ldt) {
   constexpr int G = 3 * N;
-  constexpr int U = kv4_units(N);
   const int lane = threadIdx.x & 31;
+  const int half = lane >> 4, li = lane & 15;
   const int total = T * H;
-  const int unit0 = (blockIdx.x * kKvWarps + (threadIdx.x >> 5)) * U;
-  const int ga = kv4_group_of<N>(4 * lane), gb = kv4_group_of<N>(4 * lane + 3);
-  bool in_b[4];
+  const int unit0 = (blockIdx.x * kKvWarps + (threadIdx.x >> 5)) * (2 * kKvDecSteps);
+  const int ga = kv4_group_of<N>(8 * li), gb = kv4_group_of<N>(8 * li + 7);
+  bool in_b[8];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) in_b[j] = kv4_group_of<N>(4 * lane + j) != ga;
-  uint32_t pk[U];
-  int64_t dst[U];   // output element offset of each unit
-  constexpr int R = kv4_rounds(N);
-  float s_lane[R];   // pair u * G + g: scale of (unit u, group g)
+  for (int j = 0; j < 8; ++j) in_b[j] = kv4_group_of<N>(8 * li + j) != ga;
+  uint32_t pk[kKvDecSteps];
+  float sc[kKvDecSteps];
+  int64_t dst[kKvDecSteps];
 #pragma unroll
-  for (int k = 0; k < R; ++k) s_lane[k] = 0.f;
-  {
-    int tt = unit0 / H, hh = unit0 - tt * H;
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (unit0 + u < total) {
-        int64_t slot = slot0 + tt;               // < 2 capacity: one wrap at most
-        if (slot >= capacity) slot -= capacity;
-        const int64_t src = slot * H + hh;
-        pk[u] = *reinterpret_cast<const uint16_t*>(codes + src * (kKvDim / 2) + 2 * lane);
-#pragma unroll
-        for (int k = 0; k < R; ++k) {
-          const int p = lane + 32 * k;
-          if (p >= u * G && p < u * G + G) s_lane[k] = __ldg(scales + src * G + (p - u * G));
-        }
-        dst[u] = (int64_t)tt * ldt + (int64_t)hh * kKvDim;
-      }
-      if (++hh == H) { hh = 0; ++tt; }
+  for (int k = 0; k < kKvDecSteps; ++k) {
+    const int unit = unit0 + 2 * k + half;
+    if (unit < total) {
+      const int t = unit / H, h = unit - t * H;
+      int64_t slot = slot0 + t;                  // < 2 capacity: one wrap at most
+      if (slot >= capacity) slot -= capacity;
+      const int64_t src = slot * H + h;
+      pk[k] = *reinterpret_cast<const uint32_t*>(codes + src * (kKvDim / 2) + 4 * li);
+      sc[k] = li < G ? __ldg(scales + src * G + li) : 0.f;
+      dst[k] = (int64_t)t * ldt + (int64_t)h * kKvDim;
+    } else {
+      pk[k] = 0u;
+      sc[k] = 0.f;
+      dst[k] = -1;
     }
   }
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    if (unit0 + u >= total) break;   // uniform across the warp
-    const float sa = kv4_pair_value<R>(s_lane, u * G + ga), sb = kv4_pair_value<R>(s_lane, u * G + gb);
+  for (int k = 0; k < kKvDecSteps; ++k) {
+    const float sa = __shfl_sync(0xffffffffu, sc[k], ga, 16), sb = __shfl_sync(0xffffffffu, sc[k], gb, 16);
+    if (dst[k] < 0) continue;
     // q as a float without a conversion: the bits of 1.5 * 2^23 + q, minus 1.5 * 2^23 (exact)
-    float f[4];
+    float f[8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int q = static_cast<int>(static_cast<int32_t>(pk[u] << (28 - 4 * j)) >> 28);   // sign-extend nibble j
+    for (int j = 0; j < 8; ++j) {
+      const int q = static_cast<int>(static_cast<int32_t>(pk[k] << (28 - 4 * j)) >> 28);   // sign-extend nibble j
       f[j] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B400000u + static_cast<uint32_t>(q)), 12582912.0f),
                        in_b[j] ? sb : sa);
     }
-    const __nv_bfloat162 b01 = __floats2bfloat162_rn(f[0], f[1]), b23 = __floats2bfloat162_rn(f[2], f[3]);
-    const uint32_t out[2] = {*reinterpret_cast<const uint32_t*>(&b01), *reinterpret_cast<const uint32_t*>(&b23)};
-    *reinterpret_cast<uint2*>(y + dst[u] + 4 * lane) = make_uint2(out[0], out[1]);
+    uint32_t out[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+      out[e] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+    *reinterpret_cast<uint4*>(y + dst[k] + 8 * li) = make_uint4(out[0], out[1], out[2], out[3]);
   }
 }
 
@@ -227,7 +232,7 @@ cudaError_t launch_kv4_encode(const uint16_t* x, int T, int H, int64_t ldt, int 
 cudaError_t launch_kv4_decode(const uint8_t* codes, const float* scales, int64_t capacity, int64_t slot0, int T,
                               int H, int n, uint16_t* y, int64_t ldt, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  const int64_t per_block = (int64_t)kKvWarps * kv4_units(n);
+  const int64_t per_block = (int64_t)kKvWarps * 2 * kKvDecSteps;
   const dim3 grid(static_cast<unsigned>(((int64_t)T * H + per_block - 1) / per_block));
   switch (n) {
     case 1: kv4_decode_kernel<1><<<grid, kKvWarps * 32, 0, st>>>(codes, scales, capacity, slot0, T, H, y, ldt); break;
