@@ -29,9 +29,11 @@
 //   - Row scales: TT = 256, NB = 2.  One promotion per tile.
 //   - Group scales: TT = 128, NB = 4 (4 x 128 columns fill the 512 of TMEM).
 //     Every 64-wide K block needs its own promotion, so the epilogue is the
-//     busy side: four buffers let the tensor core run three segments ahead,
-//     and the small tile keeps the epilogue's accumulators and in-flight
-//     TMEM loads in registers (see the group-scale epilogue below).
+//     busy side.  The four buffers are handed over in pairs (the two groups
+//     of one 128-wide K stage): the tensor core fills one pair while the
+//     epilogue drains the other, and the small tile keeps the epilogue's
+//     accumulators and in-flight TMEM loads in registers (see the
+//     group-scale epilogue below).
 // In group mode the epilogue adds the bit pattern of 12582912.0f (1.5 * 2^23)
 // to each int32 partial: read as float the sum is exactly 12582912 + 16*acc,
 // and fma(f, a, -12582912*a) gives the correctly rounded 16*acc*a without an
@@ -42,8 +44,8 @@
 // Warp roles (16 warps, registers redistributed per warpgroup with setmaxnreg):
 //   warpgroup 0: warps 0, 2, 3 TMA producers, warp 1 TMEM allocator + MMA issuer;
 //   warpgroup 1: INT4 -> INT8 converters (W4A4 only);
-//   warpgroups 2-3: epilogue; row scales: thread = one output feature x TT/2
-//   tokens; group scales: thread = 4 features x 16 tokens.
+//   warpgroups 2-3: epilogue; thread = one output feature (TMEM lane) x TT/2
+//   tokens (128 with row scales, 64 with group scales).
 #include "rbd_common.cuh"
 #include "rbd_internal.cuh"
 
