@@ -45,6 +45,7 @@ class RotatedLowBitLinear:
         self.gate_mode, self.gate_cols = gate_mode, gate_cols
         self.gate = gate.contiguous() if gate is not None else None
         self._bufs = {}
+        self._host_pipes = {}   # forward_host: streams and staging buffers per (device, chunk, residual)
 
     def buffers(self, M: int, device):
         key = (M, str(device))
@@ -88,20 +89,11 @@ class RotatedLowBitLinear:
         dev = torch.device(device) if device is not None else self.wq.device
         M = xh.shape[0]
         cur = torch.cuda.current_stream(dev)
-        streams = [torch.cuda.Stream(device=dev) for _ in range(2)]
+        streams, staged = self._host_pipeline(dev, chunk, residual_h is not None)
         start = torch.cuda.Event()
         start.record(cur)
-        G = self.K // 64 if self.scale_group else 1
-        staged = []   # per stream: its own input, output, residual and intermediate buffers
         for s in streams:
             s.wait_event(start)
-            bufs = (torch.empty((chunk, self.K), dtype=torch.bfloat16, device=dev),
-                    torch.empty((chunk, self.N), dtype=torch.bfloat16, device=dev),
-                    torch.empty((chunk, self.N), dtype=torch.bfloat16, device=dev) if residual_h is not None else None,
-                    torch.empty((chunk, self.K), dtype=torch.int8, device=dev),
-                    torch.empty((chunk, G) if self.scale_group else (chunk,), dtype=torch.float32, device=dev),
-                    torch.empty((chunk, self.rank), dtype=torch.bfloat16, device=dev) if self.rank else None)
-            staged.append(bufs)
         for i, m0 in enumerate(range(0, M, chunk)):
             m = min(M, m0 + chunk) - m0
             s = streams[i % 2]
@@ -116,9 +108,25 @@ class RotatedLowBitLinear:
                 yh[m0:m0 + m].copy_(yd[:m], non_blocking=True)
         for s in streams:
             cur.wait_stream(s)
-        # the staging buffers stay alive until the streams are done with them
-        for s, bufs in zip(streams, staged):
-            for t in bufs:
-                if t is not None:
-                    t.record_stream(s)
         return yh
+
+    def _host_pipeline(self, dev, chunk: int, with_residual: bool):
+        """The two streams of forward_host and, per stream, its own input, output, residual and
+        intermediate buffers; created once per (device, chunk, residual) and reused.  Reuse is
+        safe: a buffer is only touched on its own stream, every call makes its streams wait for
+        the caller's stream first, and the caller's stream waits for them at the end."""
+        key = (str(dev), chunk, with_residual)
+        if key not in self._host_pipes:
+            G = self.K // 64 if self.scale_group else 1
+            streams = [torch.cuda.Stream(device=dev) for _ in range(2)]
+            staged = []
+            for _ in streams:
+                staged.append((
+                    torch.empty((chunk, self.K), dtype=torch.bfloat16, device=dev),
+                    torch.empty((chunk, self.N), dtype=torch.bfloat16, device=dev),
+                    torch.empty((chunk, self.N), dtype=torch.bfloat16, device=dev) if with_residual else None,
+                    torch.empty((chunk, self.K), dtype=torch.int8, device=dev),
+                    torch.empty((chunk, G) if self.scale_group else (chunk,), dtype=torch.float32, device=dev),
+                    torch.empty((chunk, self.rank), dtype=torch.bfloat16, device=dev) if self.rank else None))
+            self._host_pipes[key] = (streams, staged)
+        return self._host_pipes[key]
