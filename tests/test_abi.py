@@ -184,3 +184,16 @@ def test_kv4_validation_without_gpu():
     assert enc(FAKE, 0, 2, 256, 1, null, null, 8, 0, None) == 0          # empty slice
     assert dec(FAKE, FAKE, 8, 0, 4, 0, 1, FAKE, 256, None) == 1          # no heads
     assert dec(null, FAKE, 8, 0, 4, 2, 1, FAKE, 256, None) == 1
+
+
+@pytest.mark.parametrize("lang,std", [("c", "-std=c99"), ("c++", "-std=c++17")])
+def test_header_is_plain_c_and_cxx(lang, std):
+    # the boundary header carries no torch or CUDA types: it compiles alone as C99 and as C++
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    r = subprocess.run([cc, "-fsyntax-only", "-Wall", "-Wextra", "-Werror", "-x", lang, std, HDR],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
