@@ -6,12 +6,13 @@ W4A4 GEMM with group-64 dequant, rank-32 branch and sigmoid gate epilogue
 (the grouped Q|K|V|gate projection, M=4096 tokens, K=3072, N=4*3072).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-    python bench.py --sweep small-m|stack|prologue|kv4   (one JSON line per case)
+    python bench.py --sweep small-m|stack|prologue|kv4|nvfp4   (one JSON line per case)
 
 Sweeps: small-m (K = N = 3072 layer at 1..1024 tokens, W4A4 and NVFP4, HBM
 roofline), stack (the 28-block stack of 224 linears), prologue (the
 activation prologues at the layer shapes, HBM roofline), kv4 (the INT4
-KV-cache codec, HBM roofline).
+KV-cache codec, HBM roofline), nvfp4 (the NVFP4 variant at the Q|K|V|gate
+shape against the FP4 dense peak).
 
 Under torchrun each rank runs its own replica on its own batch (tokens are
 independent; no collective on the data path), scaling is weak and the value
@@ -543,6 +544,81 @@ def run_kv4_sweep(args):
                 flush=True)
 
 
+# ----------------------------------------------------------------------------- NVFP4 at the layer shape
+def run_nvfp4_sweep(args):
+    """The NVFP4 variant at the grouped Q|K|V|gate shape (K = 3072, N = 12288, rank-32 branch, sigmoid
+    gate) and 1024 / 4096 tokens, compute-bound: the FP4 GEMM against the FP4 dense peak (measured
+    bf16 x 4, the nominal FP4:BF16 ratio), plus the whole layer (two-pass quantiser + GEMM).  Each
+    timed call follows a 256 MB L2 flush."""
+    import torch
+
+    import rotated_bit_dit_b200 as R
+    from rotated_bit_dit_b200 import _binding as B
+    from rotated_bit_dit_b200 import inputs as I
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    R.load()
+    peaks, src = load_peaks()
+    fp4_peak = 4.0 * peaks["bf16_tflops"]
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    K, N, r = 3072, 12288, 32
+    w = up(I.gaussian_bf16(1, (N, K), 0.02))
+    wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    wbs = torch.empty((B.rbd_nvfp4_scale_bytes(N, K),), dtype=torch.uint8, device=dev)
+    wgs = torch.empty((1,), dtype=torch.float32, device=dev)
+    work = torch.empty((1,), dtype=torch.int32, device=dev)
+    B.rbd_nvfp4_quant(w, wq, wbs, wgs, work, 256)
+    l1t = up(I.gaussian_bf16(2, (r, K), 0.01))
+    l2t = up(I.gaussian_bf16(3, (N, r), 0.01))
+    for M in (1024, 4096):
+        x = up(I.gaussian_bf16(4, (M, K), 1.0, 0.005, 30.0))
+        xq = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        xbs = torch.empty((B.rbd_nvfp4_scale_bytes(M, K),), dtype=torch.uint8, device=dev)
+        xgs = torch.empty((1,), dtype=torch.float32, device=dev)
+        ld = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        epi = B.make_epilogue(None, ld, l2t, 1, (3 * 3072, 4 * 3072))
+
+        def prologue():
+            B.rbd_nvfp4_quant(x, xq, xbs, xgs, work, 256)
+            B.rbd_lowrank_down(x, l1t, ld)
+
+        def gemm():
+            B.rbd_nvfp4_linear(xq, xbs, xgs, wq, wbs, wgs, y, epi)
+
+        prologue()
+        gemm()
+        torch.cuda.synchronize()
+        assert R.rbd_check() == 0
+        tg, tl = [], []
+        for i in range(max(args.warmup, 3) + args.steps):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            ev[0].record()
+            prologue()
+            ev[1].record()
+            gemm()
+            ev[2].record()
+            torch.cuda.synchronize()
+            if i >= max(args.warmup, 3):
+                tg.append(ev[1].elapsed_time(ev[2]) / 1e3)
+                tl.append(ev[0].elapsed_time(ev[2]) / 1e3)
+        assert R.rbd_check() == 0
+        g, lay = statistics.median(tg), statistics.median(tl)
+        ops = 2.0 * M * N * K
+        print(json.dumps({
+            "sweep": "nvfp4", "M": M, "K": K, "N": N, "rank": r, "gemm_us": g * 1e6, "layer_us": lay * 1e6,
+            "gemm_tflops": ops / g / 1e12, "layer_tflops": ops / lay / 1e12,
+            "frac_fp4_peak": ops / g / 1e12 / fp4_peak,
+            "peak_source": f"{src} bf16 dense {peaks['bf16_tflops']} TFLOP/s x 4 (nominal FP4:BF16 ratio)",
+            "timing": f"median of {args.steps} calls, each after a 256 MB L2 flush"}), flush=True)
+
+
 # ----------------------------------------------------------------------------- 28-block stack
 STACK_LAYERS = (("wq", 3072, 3072), ("wk", 3072, 3072), ("wv", 3072, 3072), ("gate", 3072, 3072),
                 ("wo", 3072, 3072), ("mlp.gate", 3072, 12288), ("mlp.up", 3072, 12288), ("mlp.down", 12288, 3072))
@@ -650,7 +726,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--print-gemm-hash", action="store_true", help="print the GEMM source hash and exit")
-    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4"], default=None,
+    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4", "nvfp4"], default=None,
                     help="instead of the headline line, print the small-token-count sweep (one line per case)")
     args = ap.parse_args()
     if args.print_gemm_hash:
@@ -667,6 +743,9 @@ def main():
         return
     if args.sweep == "kv4":
         run_kv4_sweep(args)
+        return
+    if args.sweep == "nvfp4":
+        run_nvfp4_sweep(args)
         return
     if args.impl == "reference" and int(os.environ.get("RANK", "0")) != 0:
         return                      # the oracle arm runs on rank 0 only; other ranks do no work
