@@ -39,6 +39,10 @@ What it computes (plain, slow, float64 unless a step fixes the precision):
 8. INT4 KV-cache codec: packed codes with one float32 scale per token, head
    and group, groups inside the 44 | 42 | 42 rotary bands.  Source: "lab",
    Study 6 (the cache goes to four bits).
+9. Offline SVDQuant fit of the low-rank branch (randomized SVD, alternating
+   refit / requantise keeping the best, optional activation weighting).
+   Source: Krea-2-SVDQuant-ComfyUI, "Low-rank refinement, and what the
+   objective actually is", "Activation-aware branch".
 
 Readings of points the pages leave open are listed where they are used.
 """
@@ -563,3 +567,80 @@ def kv4_decode(packed: np.ndarray, scales: np.ndarray, groups_per_band: int) -> 
     sizes = kv4_group_sizes(groups_per_band)
     s = np.repeat(scales, sizes, axis=2).astype(np.float32)
     return f64_to_bf16((q * s).astype(np.float32).astype(np.float64))
+
+
+# ---------------------------------------------------------------------------
+# 9. Offline SVDQuant fit of the low-rank branch
+# ---------------------------------------------------------------------------
+# Source: Krea-2-SVDQuant-ComfyUI, "Low-rank refinement, and what the
+# objective actually is" and "Activation-aware branch": the branch is fitted
+# by minimising ||W - (Q + L1 L2)||; a seeded randomized SVD gives the first
+# split; the branch is then refit against the current quantisation error and
+# the residual requantised, repeatedly, keeping the best, so refining never
+# does worse; --act-stats weights the objective by a per-input-channel
+# activation RMS d, normalised to mean 1 and floor-clamped at 0.05.
+# Readings: the residual is rounded to bf16 before it is quantised (the
+# packer's input type); the quantised residual is the layer's own rotated
+# INT4/INT8 format; the randomized SVD's Gaussian test matrices are inputs
+# (one per iteration); the rank-r product is split evenly, L1 = V sqrt(S),
+# L2 = sqrt(S) U^T, so that (x L1) L2 = x (U S V^T)^T.
+
+def dequantize_weights(q: np.ndarray, scales: np.ndarray, bits: int, rot_group: int = GROUP,
+                       scale_group: int = 0) -> np.ndarray:
+    """Codes times scales in the rotated domain, rotated back (R = H/16 is symmetric and
+    orthonormal, so R^-1 = R): the float64 weight the quantised format stands for, [N, K]."""
+    codes = (unpack_int4(q) if bits == 4 else np.asarray(q)).astype(np.float64)
+    n, k = codes.shape
+    s = np.asarray(scales, dtype=np.float64)
+    s = np.repeat(s, scale_group, axis=1) if scale_group else s[:, None]
+    wr = codes * s
+    if rot_group:
+        wr = np.matmul(wr.reshape(n, k // rot_group, rot_group), rotation_matrix(rot_group)).reshape(n, k)
+    return wr
+
+
+def randomized_svd(a: np.ndarray, rank: int, omega: np.ndarray, power_iters: int = 1):
+    """Rank-`rank` factors (U [n, r], S [r], Vt [r, k]) of a [n, k] by a Gaussian sketch:
+    Y = A Omega (Omega [k, r + p] given), `power_iters` rounds of Y = A (A^T Y) with
+    re-orthonormalisation, Q = orth(Y), B = Q^T A = U_b S V^T, U = Q U_b; truncated to r."""
+    a = np.asarray(a, dtype=np.float64)
+    y = a @ omega
+    qy, _ = np.linalg.qr(y)
+    for _ in range(power_iters):
+        z, _ = np.linalg.qr(a.T @ qy)
+        qy, _ = np.linalg.qr(a @ z)
+    ub, s, vt = np.linalg.svd(qy.T @ a, full_matrices=False)
+    return (qy @ ub)[:, :rank], s[:rank], vt[:rank]
+
+
+def act_weights(act_rms: np.ndarray) -> np.ndarray:
+    """Per-input-channel weights of the activation-aware objective: mean 1, floor 0.05."""
+    d = np.asarray(act_rms, dtype=np.float64)
+    d = d / d.mean()
+    return np.maximum(d, 0.05)
+
+
+def svdquant_fit(w_bits: np.ndarray, rank: int, bits: int, omegas, rot_group: int = GROUP,
+                 scale_group: int = 0, act_rms=None):
+    """The alternating fit.  omegas: one Gaussian test matrix [K, rank + p] per iteration (the first
+    is the single-shot split, each further one a refinement).  Returns the best iterate:
+    dict(l1 [K, r], l2 [r, N] float64, q, scales, err, errs) where err is the (weighted) Frobenius
+    error ||(W - (deq(Q) + (L1 L2)^T)) diag(d)|| and errs the error of every iterate."""
+    w = bf16_to_f64(w_bits)
+    d = np.ones(w.shape[1]) if act_rms is None else act_weights(act_rms)
+    target = w                              # what the branch approximates in this iterate
+    best, errs = None, []
+    for omega in omegas:
+        u, s, vt = randomized_svd(target * d[None, :], rank, omega)
+        low = (u * s) @ vt / d[None, :]     # the branch's part of W, [N, K]
+        q, sc = quantize_weights(f64_to_bf16(w - low), bits, rot_group, scale_group)
+        deq = dequantize_weights(q, sc, bits, rot_group, scale_group)
+        err = float(np.linalg.norm((w - (deq + low)) * d[None, :]))
+        errs.append(err)
+        if best is None or err < best["err"]:
+            root = np.sqrt(s)
+            vd = vt / d[None, :]             # undo the channel weighting on the input side
+            best = dict(l1=(vd.T * root[None, :]), l2=(root[:, None] * u.T), q=q, scales=sc, err=err)
+        target = w - deq                    # refit against the current quantisation error
+    best["errs"] = errs
+    return best

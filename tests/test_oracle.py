@@ -449,3 +449,81 @@ def test_kv4_band_isolation_and_error_bound():
         y = O.bf16_to_f64(O.kv4_decode(p0, s0, n))
         s = np.repeat(s0, sizes, axis=2)
         assert np.all(np.abs(y - O.bf16_to_f64(xb)) <= s / 2 + np.abs(y) * 2.0 ** -8 + 1e-30)
+
+
+# --------------------------------------------------------------- offline SVDQuant fit
+def _lowrank_plus_noise(seed, n=64, k=256, r=8, noise=0.01):
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal((n, r)) @ rng.standard_normal((r, k)) * 0.05 + noise * rng.standard_normal((n, k))
+    return O.f64_to_bf16(w)
+
+
+@pytest.mark.parametrize("bits,sg", [(4, 0), (4, 64), (8, 0)])
+def test_weight_dequantisation_error_bound(bits, sg):
+    wb = I.gaussian_bf16(60, (32, 512), 0.02)
+    q, s = O.quantize_weights(wb, bits, 256, sg)
+    deq = O.dequantize_weights(q, s, bits, 256, sg)
+    # R is orthonormal: the Frobenius error equals the rotated-domain error, at most half a step per element
+    step = np.repeat(s, sg, axis=1) if sg else np.repeat(s[:, None], 512, axis=1)
+    assert np.linalg.norm(O.bf16_to_f64(wb) - deq) <= np.linalg.norm(step / 2) * 1.0001 + 1e-12
+
+
+def test_randomized_svd_exact_rank_and_eckart_young():
+    rng = np.random.default_rng(61)
+    a = rng.standard_normal((80, 6)) @ rng.standard_normal((6, 200))
+    u, s, vt = O.randomized_svd(a, 6, rng.standard_normal((200, 14)))
+    assert np.linalg.norm(a - (u * s) @ vt) <= 1e-10 * np.linalg.norm(a)
+    # a spectral gap after rank 5: the sketch reaches the optimal truncation error
+    uu, _ = np.linalg.qr(rng.standard_normal((80, 80)))
+    vv, _ = np.linalg.qr(rng.standard_normal((200, 80)))
+    sig = np.concatenate([[100, 80, 60, 40, 20], 0.01 * np.ones(75)])
+    b = (uu * sig) @ vv.T
+    u, s, vt = O.randomized_svd(b, 5, rng.standard_normal((200, 15)))
+    optimal = np.sqrt((sig[5:] ** 2).sum())
+    assert abs(np.linalg.norm(b - (u * s) @ vt) - optimal) <= 1e-6 * optimal
+    assert np.allclose(s, sig[:5], rtol=1e-9)
+
+
+def test_svdquant_fit_keeps_the_best_and_never_does_worse_than_the_single_shot():
+    wb = _lowrank_plus_noise(62)
+    rng = np.random.default_rng(63)
+    omegas = [rng.standard_normal((256, 16)) for _ in range(4)]
+    single = O.svdquant_fit(wb, 8, 4, omegas[:1])
+    refined = O.svdquant_fit(wb, 8, 4, omegas)
+    assert single["err"] == refined["errs"][0]          # iteration one is the single-shot split
+    assert refined["err"] == min(refined["errs"]) <= single["err"]
+    # the kept factors and codes reproduce the kept error
+    w = O.bf16_to_f64(wb)
+    deq = O.dequantize_weights(refined["q"], refined["scales"], 4)
+    assert np.isclose(np.linalg.norm(w - (deq + (refined["l1"] @ refined["l2"]).T)), refined["err"], rtol=1e-9)
+    # the branch carries the low-rank part: far below quantising W alone
+    q, s = O.quantize_weights(wb, 4)
+    assert refined["err"] < 0.2 * np.linalg.norm(w - O.dequantize_weights(q, s, 4))
+
+
+def test_svdquant_activation_weights():
+    # mean-1 normalisation, then the 0.05 floor for a dead channel
+    d = O.act_weights(np.r_[0.0, np.ones(255)])
+    assert d[0] == 0.05 and np.allclose(d[1:], 256 / 255)
+    wb = _lowrank_plus_noise(64)
+    rng = np.random.default_rng(65)
+    omegas = [rng.standard_normal((256, 16)) for _ in range(2)]
+    plain = O.svdquant_fit(wb, 8, 4, omegas)
+    const = O.svdquant_fit(wb, 8, 4, omegas, act_rms=np.full(256, 2.0))   # constant RMS: weights exactly 1
+    assert plain["errs"] == const["errs"] and np.array_equal(plain["q"], const["q"])
+    # competing structure: a rank-4 part in channels 0-31 and a larger rank-4 part in the others.
+    # With a rank-4 budget the plain fit's branch takes the larger part; weighting channels 0-31
+    # by 8 moves the branch onto them.  (The total error there need not drop: the residual's
+    # per-row scale then carries the large part, which a weighting of the branch cannot change.)
+    r4 = np.random.default_rng(66)
+    w = np.zeros((64, 256))
+    w[:, :32] = r4.standard_normal((64, 4)) @ r4.standard_normal((4, 32)) * 0.03
+    w[:, 32:] = r4.standard_normal((64, 4)) @ r4.standard_normal((4, 224)) * 0.06
+    cb = O.f64_to_bf16(w + 1e-3 * r4.standard_normal((64, 256)))
+    rms = np.ones(256)
+    rms[:32] = 8.0
+    om4 = [r4.standard_normal((256, 12)) for _ in range(2)]
+    wc = O.bf16_to_f64(cb)
+    def branch_miss(fit):           # how far the branch is from the heavy channels' structure
+        return np.linalg.norm(wc[:, :32] - (fit["l1"] @ fit["l2"]).T[:, :32])
+    assert branch_miss(O.svdquant_fit(cb, 4, 4, om4, act_rms=rms)) < 0.5 * branch_miss(O.svdquant_fit(cb, 4, 4, om4))
