@@ -31,4 +31,5 @@ from ._binding import (  # noqa: F401
     rbd_kv4_encode,
     rbd_kv4_decode,
 )
+from .kvcache import Int4KVCache  # noqa: F401
 from .layer import RotatedLowBitLinear  # noqa: F401

@@ -1,0 +1,68 @@
+"""Int4KVCache: a ring of INT4 key (or value) slots driven by rbd_kv4_encode / rbd_kv4_decode.
+
+The cache offers the three operations a serving loop performs on a KV cache -- a slice
+write, a rolling eviction and a slice read -- ("lab", Study 6: the int4 cache presents itself
+to the runtime as an ordinary tensor across exactly those operations).  Only the ring's
+bookkeeping lives here; encoding and decoding run in librbd.so.  Token 0 of the cache is the
+oldest one held; slots are reused in ring order, so a write never moves existing codes.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _binding as B
+
+
+class Int4KVCache:
+    def __init__(self, capacity: int, heads: int, groups_per_band: int = 1, device=None):
+        """capacity: token slots; heads: heads of 128 channels per token; groups_per_band 1, 2
+        or 4 (3, 6 or 12 scale groups per head)."""
+        if capacity <= 0 or heads <= 0:
+            raise ValueError("capacity and heads must be positive")
+        if groups_per_band not in (1, 2, 4):
+            raise ValueError("groups_per_band must be 1, 2 or 4")
+        self.capacity, self.heads, self.groups_per_band = capacity, heads, groups_per_band
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.codes = torch.zeros((capacity, heads, 64), dtype=torch.uint8, device=dev)
+        self.scales = torch.zeros((capacity, heads, 3 * groups_per_band), dtype=torch.float32, device=dev)
+        self.start = 0   # slot of the oldest token held
+        self.size = 0    # tokens held
+
+    def write(self, x: torch.Tensor) -> None:
+        """Append the tokens of x (bf16 [T, heads * 128], row stride may be larger).  When the
+        ring is full the oldest tokens are evicted first (rolling)."""
+        if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != self.heads * 128:
+            raise ValueError("x must be bf16 [T, heads * 128]")
+        t = x.shape[0]
+        if t > self.capacity:
+            raise ValueError("slice longer than the cache")
+        overflow = self.size + t - self.capacity
+        if overflow > 0:
+            self.evict(overflow)
+        slot0 = (self.start + self.size) % self.capacity
+        B.rbd_kv4_encode(x, self.codes, self.scales, self.groups_per_band, slot0)
+        self.size += t
+
+    def evict(self, n: int) -> None:
+        """Drop the n oldest tokens (their slots are reused by later writes)."""
+        if n < 0 or n > self.size:
+            raise ValueError("cannot evict more tokens than the cache holds")
+        self.start = (self.start + n) % self.capacity
+        self.size -= n
+
+    def read(self, first: int = 0, count: Optional[int] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Decode tokens first .. first + count - 1 (0 = the oldest held) into out (bf16
+        [count, heads * 128]; allocated when not given)."""
+        count = self.size - first if count is None else count
+        if first < 0 or count < 0 or first + count > self.size:
+            raise ValueError("read outside the tokens held")
+        if out is None:
+            out = torch.empty((count, self.heads * 128), dtype=torch.bfloat16, device=self.codes.device)
+        elif out.dtype != torch.bfloat16 or out.dim() != 2 or out.shape[0] < count or out.shape[1] != self.heads * 128:
+            raise ValueError("out must be bf16 [>= count, heads * 128]")
+        if count:
+            slot0 = (self.start + first) % self.capacity
+            B.rbd_kv4_decode(self.codes, self.scales, out[:count], self.groups_per_band, slot0)
+        return out
