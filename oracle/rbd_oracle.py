@@ -43,6 +43,10 @@ What it computes (plain, slow, float64 unless a step fixes the precision):
    refit / requantise keeping the best, optional activation weighting).
    Source: Krea-2-SVDQuant-ComfyUI, "Low-rank refinement, and what the
    objective actually is", "Activation-aware branch".
+10. Q/K RMSNorm + RoPE over the 44 | 42 | 42 rotary bands, and attention with
+   INT8 Q.K^T (smoothed keys, one scale per token and head) and FP16 P.V.
+   Source: OrbitQuant W4A4 card, "Fused transformer" (the SageAttention v1
+   scheme); "lab", Study 6 (the rotary bands).
 
 Readings of points the pages leave open are listed where they are used.
 """
@@ -644,3 +648,103 @@ def svdquant_fit(w_bits: np.ndarray, rank: int, bits: int, omegas, rot_group: in
         target = w - deq                    # refit against the current quantisation error
     best["errs"] = errs
     return best
+
+
+# ---------------------------------------------------------------------------
+# 10. Q/K RMSNorm + RoPE and quantized attention (SageAttention-v1 scheme)
+# ---------------------------------------------------------------------------
+# Source: OrbitQuant W4A4 card, "Fused transformer": each block runs a Q/K
+# RMSNorm + RoPE kernel after the Q|K|V|gate GEMM, and attention takes Q.K^T in
+# INT8 and P.V in FP16 (the SageAttention v1 scheme); "lab", Study 6: rotary
+# embedding splits the 128 channels of a head into bands of 44 (time), 42
+# (height) and 42 (width).
+# Readings (the pages name the scheme, not its steps):
+#   - RoPE turns channel pairs (2i, 2i+1) of a head; pair i belongs to the band
+#     holding channels 2i and 2i+1 and turns by pos[band] * base**(-2j / w),
+#     j its index inside the band of width w, base 10000; the angles reach the
+#     kernel as float32 cos / sin tables [T, 64], inputs like the activations;
+#   - Q/K RMSNorm is per token and head over the 128 channels with a bf16
+#     gamma [128] shared by the heads, computed with the RoPE turn in float64
+#     and rounded once to bf16;
+#   - keys are smoothed before quantisation by subtracting their mean over the
+#     tokens (per head and channel; softmax is unchanged by it in exact
+#     arithmetic), the mean in float64 and the smoothed key rounded once to
+#     float32;
+#   - Q and the smoothed K are quantised per token and head to INT8 with the
+#     activation quantiser's float32 steps (qmax 127); the score is the exact
+#     integer dot product times s_q s_k / sqrt(128);
+#   - softmax over the keys, then P.V with V converted from bf16 to fp16 (exact
+#     inside fp16's range).  The oracle keeps P in float64; a kernel that rounds
+#     the unnormalised P to fp16 for its MMA stays within the output tolerance.
+
+ATTN_HEAD_DIM = 128
+ROPE_BANDS = KV_BANDS
+ROPE_BASE = 10000.0
+
+
+def rope_tables(pos: np.ndarray, base: float = ROPE_BASE):
+    """pos int [T, 3] (time, height, width) -> (cos, sin) float64 [T, 64], one angle per pair."""
+    pos = np.asarray(pos, dtype=np.float64)
+    ang = np.zeros((pos.shape[0], ATTN_HEAD_DIM // 2))
+    p0 = 0
+    for axis, w in enumerate(ROPE_BANDS):
+        for j in range(w // 2):
+            ang[:, p0 + j] = pos[:, axis] * base ** (-2.0 * j / w)
+        p0 += w // 2
+    return np.cos(ang), np.sin(ang)
+
+
+def qk_norm_rope(x_bits: np.ndarray, gamma_bits, cos: np.ndarray, sin: np.ndarray, eps: float) -> np.ndarray:
+    """bf16 [T, H, 128] -> bf16 [T, H, 128]: x / sqrt(mean(x^2) + eps) * gamma, then pair i of
+    token t turned by the angle whose cosine and sine are cos[t, i], sin[t, i]."""
+    x = bf16_to_f64(x_bits)
+    r = 1.0 / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps)
+    u = x * r
+    if gamma_bits is not None:
+        u = u * bf16_to_f64(gamma_bits)[None, None, :]
+    c = np.asarray(cos, np.float64)[:, None, :]
+    s = np.asarray(sin, np.float64)[:, None, :]
+    a, b = u[..., 0::2], u[..., 1::2]
+    out = np.empty_like(u)
+    out[..., 0::2] = a * c - b * s
+    out[..., 1::2] = a * s + b * c
+    return f64_to_bf16(out)
+
+
+def smooth_keys(k: np.ndarray) -> np.ndarray:
+    """float [T, H, D] -> float32 keys minus their float64 mean over the tokens."""
+    k = np.asarray(k, np.float64)
+    return (k - k.mean(axis=0, keepdims=True)).astype(np.float32)
+
+
+def quantize_heads_int8(x: np.ndarray):
+    """float32 [T, H, D] -> (codes int8 [T, H, D], scales float32 [T, H]), one scale per token and head."""
+    t, h, d = x.shape
+    q, s = quantize(np.asarray(x, np.float32).reshape(t * h, d), 8, 0)
+    return q.reshape(t, h, d), s.reshape(t, h)
+
+
+def attention_scores(q_bits: np.ndarray, k_bits: np.ndarray, smooth: bool = True, quant: bool = True):
+    """Scores S [H, Tq, Tk] float64.  quant: the INT8 scheme; otherwise the plain q.k / sqrt(D)."""
+    q = bf16_to_f64(q_bits).astype(np.float32)
+    k = bf16_to_f64(k_bits).astype(np.float32)
+    if smooth:
+        k = smooth_keys(k)
+    d = q.shape[-1]
+    if not quant:
+        return np.einsum("qhd,khd->hqk", q.astype(np.float64), k.astype(np.float64)) / math.sqrt(d)
+    qq, sq = quantize_heads_int8(q)
+    kq, sk = quantize_heads_int8(k)
+    acc = np.einsum("qhd,khd->hqk", qq.astype(np.int64), kq.astype(np.int64))
+    return acc * (sq.T.astype(np.float64)[:, :, None] * sk.T.astype(np.float64)[:, None, :]) / math.sqrt(d)
+
+
+def sage_attention(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, smooth: bool = True,
+                   quant: bool = True) -> np.ndarray:
+    """bf16 q [Tq, H, D], k / v [Tk, H, D] -> float64 output [Tq, H, D]."""
+    s = attention_scores(q_bits, k_bits, smooth, quant)
+    s = s - s.max(axis=-1, keepdims=True)
+    p = np.exp(s)
+    p /= p.sum(axis=-1, keepdims=True)
+    v16 = bf16_to_f64(v_bits).astype(np.float16).astype(np.float64)
+    return np.einsum("hqk,khd->qhd", p, v16)

@@ -527,3 +527,132 @@ def test_svdquant_activation_weights():
     def branch_miss(fit):           # how far the branch is from the heavy channels' structure
         return np.linalg.norm(wc[:, :32] - (fit["l1"] @ fit["l2"]).T[:, :32])
     assert branch_miss(O.svdquant_fit(cb, 4, 4, om4, act_rms=rms)) < 0.5 * branch_miss(O.svdquant_fit(cb, 4, 4, om4))
+
+
+# --------------------------------------------------------------- Q/K RMSNorm + RoPE, quantized attention
+def _rope_apply(u, cos, sin):
+    """Turn pairs of a float64 [T, D] by complex multiplication (an independent form of the rotation)."""
+    z = (u[:, 0::2] + 1j * u[:, 1::2]) * (cos + 1j * sin)
+    out = np.empty_like(u)
+    out[:, 0::2], out[:, 1::2] = z.real, z.imag
+    return out
+
+
+def test_rope_tables_bands_and_first_pairs():
+    cos, sin = O.rope_tables(np.array([[0, 0, 0], [1, 0, 0], [0, 2, 0], [0, 0, 3]]))
+    assert np.array_equal(cos[0], np.ones(64)) and np.array_equal(sin[0], np.zeros(64))
+    # position 1 on the time axis turns only the 22 pairs of the 44-channel band, its first pair by 1 rad
+    assert np.all(sin[1, :22] > 0) and not sin[1, 22:].any()
+    assert cos[1, 0] == np.cos(1.0) and sin[1, 0] == np.sin(1.0)
+    # the height band holds pairs 22..42, the width band pairs 43..63; their first pairs turn by pos rad
+    assert not sin[2, :22].any() and np.all(sin[2, 22:43] != 0) and not sin[2, 43:].any()
+    assert sin[2, 22] == np.sin(2.0) and sin[3, 43] == np.sin(3.0) and not sin[3, :43].any()
+    # inside each band the frequencies form a geometric sequence spanning a factor of the base: the
+    # ratio of neighbouring pairs, raised to the band's pair count, is 1 / base
+    c, s = O.rope_tables(np.array([[1, 1, 1]]))
+    ang = np.arctan2(s[0], c[0])
+    p0 = 0
+    for w in (44, 42, 42):
+        a = ang[p0:p0 + w // 2]
+        ratio = a[1:] / a[:-1]
+        assert np.allclose(ratio, ratio[0], rtol=1e-12, atol=0)
+        assert abs(ratio[0] ** (w // 2) * O.ROPE_BASE - 1.0) < 1e-10
+        p0 += w // 2
+
+
+def test_rope_relative_position():
+    rng = np.random.default_rng(5)
+    q, k = rng.standard_normal((1, 128)), rng.standard_normal((1, 128))
+    base = np.array([[3, 5, 7], [1, 2, 9]])
+    for shift in ([4, 0, 0], [0, 6, 0], [0, 0, 11], [2, 3, 1]):
+        c, s = O.rope_tables(base + np.array(shift))
+        c0, s0 = O.rope_tables(base)
+        d0 = _rope_apply(q, c0[:1], s0[:1]) @ _rope_apply(k, c0[1:], s0[1:]).T
+        d1 = _rope_apply(q, c[:1], s[:1]) @ _rope_apply(k, c[1:], s[1:]).T
+        assert abs(d0 - d1) < 1e-12
+
+
+def test_qk_norm_rope_reduces_to_rms_norm_at_position_zero():
+    g = I.gaussian_bf16(1001, (128,), 0.1)
+    g = I.f32_to_bf16_bits((O.bf16_to_f64(g) + 1.0).astype(np.float32))
+    cos, sin = np.ones((5, 64)), np.zeros((5, 64))
+    for std, eps in ((2.0, 1e-6), (1e-3, 1e-6)):     # the second case: eps comparable to the mean square
+        x = I.gaussian_bf16(1000, (5, 3, 128), std, 0.02, 20.0)
+        got = O.qk_norm_rope(x, g, cos, sin, eps)
+        xt = torch.from_numpy(O.bf16_to_f64(x))
+        want = torch.nn.functional.rms_norm(xt, (128,), torch.from_numpy(O.bf16_to_f64(g)), eps).numpy()
+        assert np.array_equal(got, O.f64_to_bf16(want))
+
+
+def test_qk_norm_rope_quarter_turn_and_pair_norms():
+    x = I.gaussian_bf16(1002, (4, 2, 128), 1.0)
+    u = O.bf16_to_f64(O.qk_norm_rope(x, None, np.ones((4, 64)), np.zeros((4, 64)), 0.0))
+    turned = O.bf16_to_f64(O.qk_norm_rope(x, None, np.zeros((4, 64)), np.ones((4, 64)), 0.0))
+    assert np.array_equal(turned[..., 0::2], -u[..., 1::2]) and np.array_equal(turned[..., 1::2], u[..., 0::2])
+    cos, sin = O.rope_tables(np.array([[7, 3, 1], [0, 40, 2], [9, 9, 9], [1, 1, 60]]))
+    y = O.bf16_to_f64(O.qk_norm_rope(x, None, cos, sin, 0.0))
+    # each pair keeps its length up to the final bf16 rounding; the whole head keeps unit mean square
+    n0 = np.hypot(u[..., 0::2], u[..., 1::2])
+    n1 = np.hypot(y[..., 0::2], y[..., 1::2])
+    assert np.all(np.abs(n1 - n0) <= 2 ** -7 * n0 + 1e-30)
+    assert np.allclose((y * y).mean(axis=-1), 1.0, rtol=1e-2)
+    # the complex-multiplication form of the turn agrees
+    xs = O.bf16_to_f64(x)
+    xs = xs / np.sqrt((xs * xs).mean(axis=-1, keepdims=True))
+    ref = np.stack([_rope_apply(xs[:, h], cos, sin) for h in range(2)], axis=1)
+    assert np.array_equal(O.f64_to_bf16(ref), O.f64_to_bf16(y))
+
+
+def _sdpa64(q, k, v):
+    qt, kt, vt = (torch.from_numpy(np.ascontiguousarray(a.transpose(1, 0, 2))) for a in (q, k, v))
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt).numpy().transpose(1, 0, 2)
+
+
+def test_attention_without_quantisation_is_textbook_sdpa():
+    q = I.gaussian_bf16(1003, (7, 2, 128), 1.0)
+    k = I.gaussian_bf16(1004, (9, 2, 128), 1.0)
+    v = I.gaussian_bf16(1005, (9, 2, 128), 1.0)
+    want = _sdpa64(O.bf16_to_f64(q), O.bf16_to_f64(k), O.bf16_to_f64(v))
+    assert np.abs(O.sage_attention(q, k, v, smooth=False, quant=False) - want).max() < 1e-12
+    # smoothing shifts every score of a query row equally; only the float32 rounding of the
+    # smoothed keys (relative 2^-24 per element) remains
+    assert np.abs(O.sage_attention(q, k, v, smooth=True, quant=False) - want).max() < 1e-6
+
+
+def test_attention_lossless_int8_codes():
+    """Q and K that are exactly INT8 codes times a power of two, with a code of 127 in every (token,
+    head) and keys in +- pairs (zero mean): quantisation is exact, so the scheme equals SDPA."""
+    rng = np.random.default_rng(9)
+
+    def coded(t, sign_pairs):
+        c = rng.integers(-127, 128, (t, 2, 128)).astype(np.float64)
+        c[..., 5] = 127
+        if sign_pairs:
+            c = np.concatenate([c, -c])
+        e = rng.integers(-6, 3, (c.shape[0], 2, 1)).astype(np.float64)
+        return I.f32_to_bf16_bits((c * 2.0 ** e).astype(np.float32))
+
+    q, k = coded(6, False), coded(5, True)
+    v = I.gaussian_bf16(1006, (10, 2, 128), 1.0)
+    qc, sq = O.quantize_heads_int8(O.bf16_to_f64(q).astype(np.float32))
+    assert np.all(np.abs(qc).max(axis=-1) == 127)
+    assert np.array_equal(qc.astype(np.float64) * sq[..., None], O.bf16_to_f64(q))
+    got = O.sage_attention(q, k, v)
+    want = _sdpa64(O.bf16_to_f64(q), O.bf16_to_f64(k), O.bf16_to_f64(v))
+    assert np.abs(got - want).max() < 1e-12
+
+
+def test_attention_smoothing_removes_a_common_key_offset():
+    """A large per-channel key offset wastes the INT8 range; smoothing removes it and the error to the
+    exact attention drops.  The output stays inside the convex hull of the value rows."""
+    q = I.gaussian_bf16(1007, (16, 2, 128), 1.0)
+    k64 = O.bf16_to_f64(I.gaussian_bf16(1008, (32, 2, 128), 1.0)) + 40.0 * np.sin(np.arange(128))
+    k = I.f32_to_bf16_bits(k64.astype(np.float32))
+    v = I.gaussian_bf16(1009, (32, 2, 128), 1.0)
+    exact = O.sage_attention(q, k, v, smooth=False, quant=False)
+    e_plain = np.abs(O.sage_attention(q, k, v, smooth=False) - exact).max()
+    e_smooth = np.abs(O.sage_attention(q, k, v, smooth=True) - exact).max()
+    assert e_smooth < 0.25 * e_plain
+    out = O.sage_attention(q, k, v)
+    vv = O.bf16_to_f64(v)
+    assert np.all(out <= vv.max(axis=0)[None] + 1e-12) and np.all(out >= vv.min(axis=0)[None] - 1e-12)
