@@ -6,13 +6,13 @@ W4A4 GEMM with group-64 dequant, rank-32 branch and sigmoid gate epilogue
 (the grouped Q|K|V|gate projection, M=4096 tokens, K=3072, N=4*3072).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-    python bench.py --sweep small-m|stack|prologue|kv4|nvfp4   (one JSON line per case)
+    python bench.py --sweep small-m|stack|prologue|kv4|nvfp4|qknorm   (one JSON line per case)
 
 Sweeps: small-m (K = N = 3072 layer at 1..1024 tokens, W4A4 and NVFP4, HBM
 roofline), stack (the 28-block stack of 224 linears), prologue (the
 activation prologues at the layer shapes, HBM roofline), kv4 (the INT4
 KV-cache codec, HBM roofline), nvfp4 (the NVFP4 variant at the Q|K|V|gate
-shape against the FP4 dense peak).
+shape against the FP4 dense peak), qknorm (Q/K RMSNorm + RoPE, HBM roofline).
 
 Under torchrun each rank runs its own replica on its own batch (tokens are
 independent; no collective on the data path), scaling is weak and the value
@@ -544,6 +544,64 @@ def run_kv4_sweep(args):
                 flush=True)
 
 
+# ----------------------------------------------------------------------------- Q/K RMSNorm + RoPE
+def run_qknorm_sweep(args):
+    """Q/K RMSNorm + RoPE at 16384 tokens x 24 heads x 128 channels (a 2048 x 2048 image's latent
+    with the 3072-wide model): a contiguous Q [T, 3072], and Q turned in place inside the fused
+    Q|K|V|gate GEMM output [T, 12288].  The rotary tables are built once, outside the timed calls.
+    Each timed call follows a 256 MB L2 flush; bytes = heads read + written, cos / sin tables, gamma."""
+    import torch
+
+    import rotated_bit_dit_b200 as R
+    from rotated_bit_dit_b200 import _binding as B
+    from rotated_bit_dit_b200 import inputs as I
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    R.load()
+    peaks, src = load_peaks()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    T, H = 16384, 24
+    pos = torch.from_numpy(I.video_positions(1, 128, 128)).to(dev)
+    cos = torch.empty((T, 64), dtype=torch.float32, device=dev)
+    sin = torch.empty((T, 64), dtype=torch.float32, device=dev)
+    B.rbd_rope_tables(pos, cos, sin)
+    gamma = torch.from_numpy(I.f32_to_bf16_bits((1.0 + 0.1 * I.normal(12, 128)).astype(np.float32)).view(np.int16))
+    gamma = gamma.view(torch.bfloat16).to(dev)
+    q = torch.from_numpy(np.ascontiguousarray(I.gaussian_bf16(10, (T, H * 128), 1.0, 0.01, 20.0)).view(np.int16))
+    q = q.view(torch.bfloat16).to(dev)
+    fused = torch.zeros((T, 4 * H * 128), dtype=torch.bfloat16, device=dev)   # Q | K | V | gate
+    fused[:, :H * 128] = q
+    qo = torch.empty_like(q)
+    nbytes = T * H * 512 + T * 512 + 256
+    for case, fn in (("contiguous", lambda: B.rbd_qk_norm_rope(q, cos, sin, qo, gamma, 1e-6)),
+                     ("in place, fused GEMM output", lambda: B.rbd_qk_norm_rope(fused[:, :H * 128], cos, sin,
+                                                                                 fused[:, :H * 128], gamma, 1e-6))):
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        assert R.rbd_check() == 0
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) / 1e3)
+        assert R.rbd_check() == 0
+        t = statistics.median(ts)
+        gbs = nbytes / t / 1e9
+        print(json.dumps({
+            "sweep": "qknorm", "case": case, "tokens": T, "heads": H, "us": t * 1e6,
+            "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "peak_source": f"{src} copy {peaks['hbm_gbs']} GB/s",
+            "algorithmic_bytes": nbytes, "timing": f"median of {args.steps} calls, each after a 256 MB L2 flush"}),
+            flush=True)
+
+
 # ----------------------------------------------------------------------------- NVFP4 at the layer shape
 def run_nvfp4_sweep(args):
     """The NVFP4 variant at the grouped Q|K|V|gate shape (K = 3072, N = 12288, rank-32 branch, sigmoid
@@ -726,7 +784,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--print-gemm-hash", action="store_true", help="print the GEMM source hash and exit")
-    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4", "nvfp4"], default=None,
+    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4", "nvfp4", "qknorm"], default=None,
                     help="instead of the headline line, print the small-token-count sweep (one line per case)")
     args = ap.parse_args()
     if args.print_gemm_hash:
@@ -746,6 +804,9 @@ def main():
         return
     if args.sweep == "nvfp4":
         run_nvfp4_sweep(args)
+        return
+    if args.sweep == "qknorm":
+        run_qknorm_sweep(args)
         return
     if args.impl == "reference" and int(os.environ.get("RANK", "0")) != 0:
         return                      # the oracle arm runs on rank 0 only; other ranks do no work

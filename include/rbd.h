@@ -280,6 +280,36 @@ rbd_status rbd_kv4_decode(const uint8_t* codes, const float* scales, int64_t cap
                           int64_t T, int64_t H, int32_t groups_per_band, void* y, int64_t ldt,
                           void* stream);
 
+/* Q/K RMSNorm + RoPE ("Krea 2 Turbo OrbitQuant W4A4", "Fused transformer":
+ * a Q/K RMSNorm + RoPE kernel follows the Q|K|V|gate GEMM in every block;
+ * "lab", Study 6: rotary bands of 44 (time), 42 (height), 42 (width) channels).
+ * Per token t and head h of 128 channels:
+ *   r = 1 / sqrt(sum(x^2) / 128 + eps) in float64, rounded to float32
+ *   (r = 0 when that radicand is 0); then in float32 u = x r gamma,
+ *   (y[2i], y[2i+1]) = (u[2i] c - u[2i+1] s, u[2i] s + u[2i+1] c),
+ *   c = cos_t[t][i], s = sin_t[t][i]; y rounded once to bf16.
+ *   x, y    bf16 [T, ldx] / [T, ldy] row-major, H heads of 128 channels per
+ *           row (head h at h * 128); ld >= 128 H, ld % 8 == 0, 16-byte
+ *           aligned; y == x (in place) is allowed.
+ *   gamma   bf16 [128] shared by the heads, 16-byte aligned, or NULL (ones).
+ *   cos_t, sin_t  float32 [T, 64], 16-byte aligned (rbd_rope_tables).
+ *   eps     finite, >= 0.
+ * Returns RBD_ERR_INVALID_ARG / RBD_ERR_ALIGNMENT for bad arguments, and
+ * RBD_ERR_UNSUPPORTED when T * H exceeds 2^30.                               */
+rbd_status rbd_qk_norm_rope(const void* x, int64_t T, int64_t H, int64_t ldx, const void* gamma,
+                            const float* cos_t, const float* sin_t, float eps, void* y, int64_t ldy,
+                            void* stream);
+
+/* Rotary angle tables for rbd_qk_norm_rope.  pos int32 [T, 3] (time, height,
+ * width) on the device, 4-byte aligned.  Pair i of a head lies in the band
+ * holding channels 2i and 2i + 1 (pairs 0-21 time, 22-42 height, 43-63
+ * width); with j its index inside a band of w channels it turns by
+ * pos[t][band] * base^(-2j / w), formed in float64; cos_t / sin_t float32
+ * [T, 64] (16-byte aligned) receive the rounded cosine and sine.  base > 0,
+ * finite (10000 is the usual value).                                         */
+rbd_status rbd_rope_tables(const int32_t* pos, int64_t T, double base, float* cos_t, float* sin_t,
+                           void* stream);
+
 /* Synchronises `stream`, then reports the first device-side error recorded
  * since the last rbd_check (RBD_ERR_DEVICE_TIMEOUT) or a CUDA error, and
  * clears the device status word.                                              */

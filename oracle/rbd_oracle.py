@@ -664,8 +664,8 @@ def svdquant_fit(w_bits: np.ndarray, rank: int, bits: int, omegas, rot_group: in
 #     j its index inside the band of width w, base 10000; the angles reach the
 #     kernel as float32 cos / sin tables [T, 64], inputs like the activations;
 #   - Q/K RMSNorm is per token and head over the 128 channels with a bf16
-#     gamma [128] shared by the heads, computed with the RoPE turn in float64
-#     and rounded once to bf16;
+#     gamma [128] shared by the heads (r = 0 when mean(x^2) + eps is 0),
+#     computed with the RoPE turn in float64 and rounded once to bf16;
 #   - keys are smoothed before quantisation by subtracting their mean over the
 #     tokens (per head and channel; softmax is unchanged by it in exact
 #     arithmetic), the mean in float64 and the smoothed key rounded once to
@@ -694,11 +694,14 @@ def rope_tables(pos: np.ndarray, base: float = ROPE_BASE):
     return np.cos(ang), np.sin(ang)
 
 
-def qk_norm_rope(x_bits: np.ndarray, gamma_bits, cos: np.ndarray, sin: np.ndarray, eps: float) -> np.ndarray:
-    """bf16 [T, H, 128] -> bf16 [T, H, 128]: x / sqrt(mean(x^2) + eps) * gamma, then pair i of
-    token t turned by the angle whose cosine and sine are cos[t, i], sin[t, i]."""
+def qk_norm_rope_f64(x_bits: np.ndarray, gamma_bits, cos: np.ndarray, sin: np.ndarray, eps: float) -> np.ndarray:
+    """bf16 [T, H, 128] -> float64 [T, H, 128]: x / sqrt(mean(x^2) + eps) * gamma (r = 0 for a head whose
+    radicand is 0, as in the normalising prologue), then pair i of token t turned by the angle whose
+    cosine and sine are cos[t, i], sin[t, i]."""
     x = bf16_to_f64(x_bits)
-    r = 1.0 / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps)
+    rad = (x * x).mean(axis=-1, keepdims=True) + eps
+    with np.errstate(divide="ignore"):
+        r = np.where(rad > 0, 1.0 / np.sqrt(rad), 0.0)
     u = x * r
     if gamma_bits is not None:
         u = u * bf16_to_f64(gamma_bits)[None, None, :]
@@ -708,7 +711,12 @@ def qk_norm_rope(x_bits: np.ndarray, gamma_bits, cos: np.ndarray, sin: np.ndarra
     out = np.empty_like(u)
     out[..., 0::2] = a * c - b * s
     out[..., 1::2] = a * s + b * c
-    return f64_to_bf16(out)
+    return out
+
+
+def qk_norm_rope(x_bits: np.ndarray, gamma_bits, cos: np.ndarray, sin: np.ndarray, eps: float) -> np.ndarray:
+    """qk_norm_rope_f64 rounded once to bf16."""
+    return f64_to_bf16(qk_norm_rope_f64(x_bits, gamma_bits, cos, sin, eps))
 
 
 def smooth_keys(k: np.ndarray) -> np.ndarray:

@@ -30,6 +30,8 @@ from ._binding import (  # noqa: F401
     rbd_nvfp4_linear,
     rbd_kv4_encode,
     rbd_kv4_decode,
+    rbd_qk_norm_rope,
+    rbd_rope_tables,
 )
 from .kvcache import Int4KVCache  # noqa: F401
 from .layer import RotatedLowBitLinear  # noqa: F401

@@ -20,7 +20,7 @@ STATUS_NAMES = {0: "RBD_OK", 1: "RBD_ERR_INVALID_ARG", 2: "RBD_ERR_UNSUPPORTED",
 
 EXPORTED = ("rbd_rot_quant_act", "rbd_norm_rot_quant_act", "rbd_lowrank_fused", "rbd_lowrank_down", "rbd_pack_weights_int4", "rbd_pack_weights_int8",
             "rbd_w4a4_linear", "rbd_w8a8_linear", "rbd_nvfp4_scale_bytes", "rbd_nvfp4_quant",
-            "rbd_nvfp4_quant_noalloc", "rbd_nvfp4_linear", "rbd_kv4_encode", "rbd_kv4_decode", "rbd_check", "rbd_debug_timeout_probe", "rbd_status_string", "rbd_version")
+            "rbd_nvfp4_quant_noalloc", "rbd_nvfp4_linear", "rbd_kv4_encode", "rbd_kv4_decode", "rbd_qk_norm_rope", "rbd_rope_tables", "rbd_check", "rbd_debug_timeout_probe", "rbd_status_string", "rbd_version")
 
 
 class RbdError(RuntimeError):
@@ -73,6 +73,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "rbd_nvfp4_linear": [vp, vp, vp, vp, vp, vp, i64, i64, i64, ctypes.POINTER(Epilogue), vp, i64, vp],
         "rbd_kv4_encode": [vp, i64, i64, i64, i32, vp, vp, i64, i64, vp],
         "rbd_kv4_decode": [vp, vp, i64, i64, i64, i64, i32, vp, i64, vp],
+        "rbd_qk_norm_rope": [vp, i64, i64, i64, vp, vp, vp, ctypes.c_float, vp, i64, vp],
+        "rbd_rope_tables": [vp, i64, ctypes.c_double, vp, vp, vp],
         "rbd_check": [vp],
         "rbd_debug_timeout_probe": [i64, vp],
     }
@@ -290,3 +292,27 @@ def rbd_kv4_decode(codes: torch.Tensor, scales: torch.Tensor, y: torch.Tensor, g
     capacity, H = codes.shape[0], codes.shape[1]
     _ok(load().rbd_kv4_decode(_ptr(codes), _ptr(scales), capacity, slot0, T, H, groups_per_band, _ptr(y),
                               _rowstride(y), _stream(stream)), "rbd_kv4_decode")
+
+
+def rbd_qk_norm_rope(x: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor, y: torch.Tensor,
+                     gamma: Optional[torch.Tensor] = None, eps: float = 1e-6, stream=None) -> None:
+    """x bf16 [T, H*128] (row stride may be larger) -> y bf16 [T, H*128] (y may be x): per-head
+    RMSNorm times gamma (bf16 [128] or None), then the RoPE turn by cos / sin float32 [T, 64]."""
+    T = x.shape[0]
+    if x.shape[1] % 128 or y.shape[0] != T or y.shape[1] != x.shape[1]:
+        raise ValueError("x and y must be [T, H*128]")
+    if cos.shape != (T, 64) or sin.shape != (T, 64) or not (cos.is_contiguous() and sin.is_contiguous()):
+        raise ValueError("cos and sin must be contiguous [T, 64]")
+    _ok(load().rbd_qk_norm_rope(_ptr(x), T, x.shape[1] // 128, _rowstride(x), _ptr(gamma), _ptr(cos), _ptr(sin),
+                                eps, _ptr(y), _rowstride(y), _stream(stream)), "rbd_qk_norm_rope")
+
+
+def rbd_rope_tables(pos: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor, base: float = 10000.0,
+                    stream=None) -> None:
+    """pos int32 [T, 3] (time, height, width) -> cos, sin float32 [T, 64]."""
+    T = pos.shape[0]
+    if pos.dtype != torch.int32 or pos.shape != (T, 3) or not pos.is_contiguous():
+        raise ValueError("pos must be contiguous int32 [T, 3]")
+    if cos.shape != (T, 64) or sin.shape != (T, 64) or not (cos.is_contiguous() and sin.is_contiguous()):
+        raise ValueError("cos and sin must be contiguous [T, 64]")
+    _ok(load().rbd_rope_tables(_ptr(pos), T, base, _ptr(cos), _ptr(sin), _stream(stream)), "rbd_rope_tables")

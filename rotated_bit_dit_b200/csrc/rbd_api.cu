@@ -318,6 +318,33 @@ rbd_status rbd_kv4_decode(const uint8_t* codes, const float* scales, int64_t cap
                                             as_stream(stream)));
 }
 
+rbd_status rbd_qk_norm_rope(const void* x, int64_t T, int64_t H, int64_t ldx, const void* gamma,
+                            const float* cos_t, const float* sin_t, float eps, void* y, int64_t ldy,
+                            void* stream) {
+  if (T < 0 || H <= 0) return RBD_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !(eps < INFINITY)) return RBD_ERR_INVALID_ARG;   // rejects NaN too
+  if (H > 65536 || T > ((int64_t)INT32_MAX / 2) / H) return RBD_ERR_UNSUPPORTED;   // 32-bit unit indices
+  if (T == 0) return RBD_OK;
+  if (!x || !y || !cos_t || !sin_t) return RBD_ERR_INVALID_ARG;
+  if (ldx < H * 128 || ldy < H * 128) return RBD_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(cos_t) || !aligned16(sin_t) || (gamma && !aligned16(gamma)) ||
+      (ldx % 8) != 0 || (ldy % 8) != 0)
+    return RBD_ERR_ALIGNMENT;
+  return cuda_status(rbd::launch_qk_norm_rope(static_cast<const uint16_t*>(x), ldx, static_cast<int>(T),
+                                              static_cast<int>(H), static_cast<const uint16_t*>(gamma), cos_t,
+                                              sin_t, eps, static_cast<uint16_t*>(y), ldy, as_stream(stream)));
+}
+
+rbd_status rbd_rope_tables(const int32_t* pos, int64_t T, double base, float* cos_t, float* sin_t,
+                           void* stream) {
+  if (T < 0 || !(base > 0.0) || !(base < INFINITY)) return RBD_ERR_INVALID_ARG;
+  if (T > (int64_t)INT32_MAX / 64) return RBD_ERR_UNSUPPORTED;
+  if (T == 0) return RBD_OK;
+  if (!pos || !cos_t || !sin_t) return RBD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(pos) & 3u) || !aligned16(cos_t) || !aligned16(sin_t)) return RBD_ERR_ALIGNMENT;
+  return cuda_status(rbd::launch_rope_tables(pos, static_cast<int>(T), base, cos_t, sin_t, as_stream(stream)));
+}
+
 rbd_status rbd_pack_weights_int4(const void* w, int64_t N, int64_t K, rbd_qcfg cfg, uint8_t* packed, float* scales,
                                  void* stream) {
   if (cfg.bits != 4) return RBD_ERR_INVALID_ARG;

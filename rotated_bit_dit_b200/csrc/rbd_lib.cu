@@ -6,3 +6,4 @@
 #include "rbd_gemm.cu"
 #include "rbd_nvfp4.cu"
 #include "rbd_kv4.cu"
+#include "rbd_rope.cu"

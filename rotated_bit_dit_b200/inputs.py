@@ -106,6 +106,13 @@ CONFIGS = {
 }
 
 
+def video_positions(frames: int, height: int, width: int, t0: int = 0) -> np.ndarray:
+    """int32 [frames * height * width, 3] (time, row, column) of a patch grid, frame-major, times
+    starting at t0: the token positions of a video (or, with one frame, an image) latent."""
+    t, h, w = np.meshgrid(np.arange(frames) + t0, np.arange(height), np.arange(width), indexing="ij")
+    return np.stack([t.ravel(), h.ravel(), w.ravel()], axis=1).astype(np.int32)
+
+
 def make_layer_inputs(cfg: dict, seed: int = 0, M: int | None = None) -> dict:
     """All bf16 inputs of one layer call as uint16 bit-pattern arrays.
 

@@ -197,3 +197,30 @@ def test_header_is_plain_c_and_cxx(lang, std):
     r = subprocess.run([cc, "-fsyntax-only", "-Wall", "-Wextra", "-Werror", "-x", lang, std, HDR],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_qk_norm_rope_validation_without_gpu():
+    lib = R.load()
+    null = ctypes.c_void_p(0)
+    f = lib.rbd_qk_norm_rope
+    assert f(FAKE, 0, 2, 256, null, null, null, 1e-6, null, 256, null) == 0        # empty: nothing to do
+    assert f(FAKE, -1, 2, 256, null, FAKE, FAKE, 1e-6, FAKE, 256, null) == 1
+    assert f(FAKE, 4, 0, 256, null, FAKE, FAKE, 1e-6, FAKE, 256, null) == 1
+    assert f(FAKE, 4, 2, 256, null, FAKE, FAKE, float("nan"), FAKE, 256, null) == 1
+    assert f(FAKE, 4, 2, 256, null, FAKE, FAKE, -1.0, FAKE, 256, null) == 1
+    assert f(FAKE, 4, 2, 256, null, null, FAKE, 1e-6, FAKE, 256, null) == 1
+    assert f(FAKE, 4, 2, 200, null, FAKE, FAKE, 1e-6, FAKE, 256, null) == 1        # row shorter than the heads
+    assert f(FAKE, 4, 2, 256, null, FAKE, FAKE, 1e-6, FAKE, 100, null) == 1
+    assert f(FAKE_MIS, 4, 2, 256, null, FAKE, FAKE, 1e-6, FAKE, 256, null) == 3
+    assert f(FAKE, 4, 2, 256, FAKE_MIS, FAKE, FAKE, 1e-6, FAKE, 256, null) == 3
+    assert f(FAKE, 4, 2, 260, null, FAKE, FAKE, 1e-6, FAKE, 256, null) == 3        # stride not a multiple of 8
+    assert f(FAKE, 1 << 30, 4, 512, null, FAKE, FAKE, 1e-6, FAKE, 512, null) == 2  # T * H beyond 2^30
+    t = lib.rbd_rope_tables
+    assert t(FAKE, 0, 10000.0, null, null, null) == 0
+    assert t(FAKE, -1, 10000.0, FAKE, FAKE, null) == 1
+    assert t(FAKE, 4, 0.0, FAKE, FAKE, null) == 1
+    assert t(FAKE, 4, float("inf"), FAKE, FAKE, null) == 1
+    assert t(null, 4, 10000.0, FAKE, FAKE, null) == 1
+    assert t(ctypes.c_void_p(0x10002), 4, 10000.0, FAKE, FAKE, null) == 3
+    assert t(FAKE, 4, 10000.0, FAKE_MIS, FAKE, null) == 3
+    assert t(FAKE, 1 << 26, 10000.0, FAKE, FAKE, null) == 2
