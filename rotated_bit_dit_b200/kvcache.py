@@ -4,7 +4,9 @@ The cache offers the three operations a serving loop performs on a KV cache -- a
 write, a rolling eviction and a slice read -- ("lab", Study 6: the int4 cache presents itself
 to the runtime as an ordinary tensor across exactly those operations).  Only the ring's
 bookkeeping lives here; encoding and decoding run in librbd.so.  Token 0 of the cache is the
-oldest one held; slots are reused in ring order, so a write never moves existing codes.
+oldest one held; slots are reused in ring order, so a write never moves existing codes.  Token
+slices index it like a tensor: cache[a:b] reads, cache[a:b] = x overwrites, cache[len(cache):] = x
+appends.
 """
 from __future__ import annotations
 
@@ -44,6 +46,41 @@ class Int4KVCache:
         slot0 = (self.start + self.size) % self.capacity
         B.rbd_kv4_encode(x, self.codes, self.scales, self.groups_per_band, slot0)
         self.size += t
+
+    def overwrite(self, first: int, x: torch.Tensor) -> None:
+        """Re-encode held tokens first .. first + T - 1 (0 = the oldest held) from x (bf16
+        [T, heads * 128]); the ring's start and size do not change."""
+        if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != self.heads * 128:
+            raise ValueError("x must be bf16 [T, heads * 128]")
+        if first < 0 or first + x.shape[0] > self.size:
+            raise ValueError("overwrite outside the tokens held")
+        B.rbd_kv4_encode(x, self.codes, self.scales, self.groups_per_band, (self.start + first) % self.capacity)
+
+    def __len__(self) -> int:
+        return self.size
+
+    def _span(self, key) -> tuple:
+        if not isinstance(key, slice):
+            raise TypeError("the cache is indexed by token slices")
+        a, b, step = key.indices(self.size)
+        if step != 1:
+            raise ValueError("slices of the cache have step 1")
+        return a, max(b - a, 0)
+
+    def __getitem__(self, key) -> torch.Tensor:
+        """cache[a:b] decodes tokens a .. b - 1 (Python slice rules, 0 = the oldest held)."""
+        a, n = self._span(key)
+        return self.read(a, n)
+
+    def __setitem__(self, key, x: torch.Tensor) -> None:
+        """cache[a:b] = x re-encodes held tokens a .. b - 1; cache[len(cache):] = x appends (rolling)."""
+        if isinstance(key, slice) and key.start == self.size and key.stop is None and key.step is None:
+            self.write(x)
+            return
+        a, n = self._span(key)
+        if n != x.shape[0]:
+            raise ValueError("slice and x differ in token count")
+        self.overwrite(a, x)
 
     def evict(self, n: int) -> None:
         """Drop the n oldest tokens (their slots are reused by later writes)."""

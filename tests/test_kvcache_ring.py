@@ -101,6 +101,38 @@ def test_ring_rolling_eviction_slots(oracle_codec):
     assert oracle_codec[-1] == ("decode", 4, 5)
 
 
+def test_ring_slices_and_overwrite(oracle_codec):
+    n = 2
+    cache = R.Int4KVCache(8, 2, n, device="cpu")
+    xa = I.gaussian_bf16(960, (6, 2, 128), 1.0, 0.02, 12.0)
+    xb = I.gaussian_bf16(961, (5, 2, 128), 1.0, 0.02, 12.0)
+    xc = I.gaussian_bf16(962, (3, 2, 128), 1.0, 0.02, 12.0)
+    cache[len(cache):] = _bf16(xa.reshape(6, 256), "cpu")
+    cache[len(cache):] = _bf16(xb.reshape(5, 256), "cpu")     # rolls: 3 oldest evicted, the ring wraps
+    held = list(xa[3:]) + list(xb)
+    assert len(cache) == 8 and cache.start == 3
+    cache[2:5] = _bf16(xc.reshape(3, 256), "cpu")               # held tokens 2..4 re-encoded in place
+    held[2:5] = list(xc)
+    assert (len(cache), cache.start) == (8, 3)
+
+    def want(lo, hi):
+        p, s = O.kv4_encode(np.stack(held[lo:hi]), n)
+        return O.kv4_decode(p, s, n)
+
+    for lo, hi, key in ((0, 8, slice(None)), (1, 7, slice(1, 7)), (5, 8, slice(-3, None)), (4, 6, slice(4, 6))):
+        got = cache[key]
+        assert np.array_equal(_bits(got).reshape(hi - lo, 2, 128), want(lo, hi)), key
+    assert cache[6:2].shape[0] == 0
+    with pytest.raises(ValueError):
+        cache[::2]
+    with pytest.raises(TypeError):
+        cache[3]
+    with pytest.raises(ValueError):
+        cache[0:2] = _bf16(xc.reshape(3, 256), "cpu")
+    with pytest.raises(ValueError):
+        cache.overwrite(6, _bf16(xc.reshape(3, 256), "cpu"))
+
+
 def test_ring_argument_errors(oracle_codec):
     cache = R.Int4KVCache(4, 1, 2, device="cpu")
     with pytest.raises(ValueError):
