@@ -656,3 +656,34 @@ def test_attention_smoothing_removes_a_common_key_offset():
     out = O.sage_attention(q, k, v)
     vv = O.bf16_to_f64(v)
     assert np.all(out <= vv.max(axis=0)[None] + 1e-12) and np.all(out >= vv.min(axis=0)[None] - 1e-12)
+
+
+def test_attention_tiled_fp16_p_stays_within_the_output_tolerance():
+    """Reading of the FP16 P.V step: a flash-style evaluation over 128-key tiles (running max and sum,
+    the unnormalised P rounded to fp16 for the product, float32 accumulation, a ragged last tile)
+    stays within the output tolerance of the oracle's float64 softmax."""
+    from tests.helpers import check_output
+
+    Tq, Tk, H = 256, 1000, 2
+    q = I.gaussian_bf16(1010, (Tq, H, 128), 1.0, 0.02, 10.0)
+    k = I.gaussian_bf16(1011, (Tk, H, 128), 1.0, 0.02, 10.0)
+    v = I.gaussian_bf16(1012, (Tk, H, 128), 1.0)
+    ref64 = O.sage_attention(q, k, v)
+    s2 = O.attention_scores(q, k).astype(np.float32) * np.float32(np.log2(np.e))   # [H, Tq, Tk]
+    v16 = O.bf16_to_f64(v).astype(np.float16).astype(np.float32)
+    out = np.zeros((Tq, H, 128))
+    for h in range(H):
+        m = np.full(Tq, -np.inf, np.float32)
+        l = np.zeros(Tq, np.float32)
+        acc = np.zeros((Tq, 128), np.float32)
+        for j0 in range(0, Tk, 128):
+            st = s2[h, :, j0:j0 + 128]
+            m_new = np.maximum(m, st.max(axis=1))
+            alpha = np.where(np.isinf(m), 0.0, np.exp2(m - m_new)).astype(np.float32)
+            p = np.exp2(st - m_new[:, None]).astype(np.float32)
+            l = l * alpha + p.sum(axis=1, dtype=np.float32)
+            acc = acc * alpha[:, None] + p.astype(np.float16).astype(np.float32) @ v16[j0:j0 + 128, h]
+            m = m_new
+        out[:, h] = acc / l[:, None]
+    got = O.f64_to_bf16(out)
+    check_output(got.reshape(Tq, -1), ref64.reshape(Tq, -1), O.f64_to_bf16(ref64).reshape(Tq, -1))
