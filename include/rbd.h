@@ -256,10 +256,10 @@ rbd_status rbd_nvfp4_linear(const uint8_t* xq, const uint8_t* xbs, const float* 
                             void* y, int64_t ldy, void* stream);
 
 /* INT4 KV-cache codec ("lab", Study 6, "The cache becomes the model":
- * int4 packed two values per byte, one scale per token, per head, per rotary
- * band; the 128 channels of a head split into rotary bands of 44, 42 and 42;
- * groups subdivide the bands and never cross them; reading unpacks and scales
- * in one pass).
+ * four-bit codes, two to a byte, with a scale for each (token, head, rotary
+ * band); the rotary bands of a head are channels 0-43, 44-85 and 86-127;
+ * finer scale groups stay inside one band; a read unpacks and rescales in a
+ * single pass).
  *   groups_per_band n in {1, 2, 4}: 3, 6 or 12 groups per head; a band of b
  *           channels is cut into n contiguous runs whose sizes differ by at
  *           most one, longer runs first.

@@ -310,7 +310,7 @@ def norm_rot_quant(x_bits: np.ndarray, bits: int, rot_group: int = GROUP, scale_
 def pack_int4(q: np.ndarray) -> np.ndarray:
     """Two's-complement nibbles, row-major, even k in the low nibble -> uint8 [rows, K/2].
 
-    Reading: the pages say only "packed signed INT4" / "two values per byte".
+    Reading: the pages fix only that the codes are signed four-bit values stored two to a byte.
     """
     q = np.asarray(q, dtype=np.int64)
     if q.min(initial=0) < -8 or q.max(initial=0) > 7:
@@ -514,12 +514,11 @@ def nvfp4_linear(x_bits, w_bits, rot_group: int = GROUP) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # 8. INT4 KV-cache codec
 # ---------------------------------------------------------------------------
-# Source: "lab", Study 6 ("The cache becomes the model"): the cache stores
-# int4 packed two values per byte with one scale per token, per head, per
-# rotary band; rotary splits the 128 channels of a head into bands of 44
-# (time), 42 (height) and 42 (width); groups are subdivided inside the bands
-# and never across them (three, six or twelve groups per head); reading
-# unpacks and scales in one pass.
+# Source: "lab", Study 6 ("The cache becomes the model"): four-bit codes, two
+# to a byte, with a scale for each (token, head, rotary band); a head's 128
+# channels form three rotary bands -- channels 0-43 carry time, 44-85 height,
+# 86-127 width; finer scale groups stay inside one band (3, 6 or 12 groups
+# per head); a read unpacks and rescales in a single pass.
 # Readings (the pages give the structure, not the arithmetic):
 #   - a band of b channels split into n groups is cut into contiguous runs whose
 #     sizes differ by at most one, the longer runs first;
@@ -655,9 +654,9 @@ def svdquant_fit(w_bits: np.ndarray, rank: int, bits: int, omegas, rot_group: in
 # ---------------------------------------------------------------------------
 # Source: OrbitQuant W4A4 card, "Fused transformer": each block runs a Q/K
 # RMSNorm + RoPE kernel after the Q|K|V|gate GEMM, and attention takes Q.K^T in
-# INT8 and P.V in FP16 (the SageAttention v1 scheme); "lab", Study 6: rotary
-# embedding splits the 128 channels of a head into bands of 44 (time), 42
-# (height) and 42 (width).
+# INT8 and P.V in FP16 (the SageAttention v1 scheme); "lab", Study 6: the
+# rotary bands of a head are channels 0-43 (time), 44-85 (height) and 86-127
+# (width).
 # Readings (the pages name the scheme, not its steps):
 #   - RoPE turns channel pairs (2i, 2i+1) of a head; pair i belongs to the band
 #     holding channels 2i and 2i+1 and turns by pos[band] * base**(-2j / w),

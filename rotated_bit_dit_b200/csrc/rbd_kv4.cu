@@ -2,11 +2,10 @@
 // key or value cache with one float32 scale per token, head and group, the
 // groups lying inside the rotary bands of the head.
 //
-// Method: "lab", Study 6 ("The cache becomes the model"): the cache stores
-// int4 packed two values per byte with one scale per token, per head, per
-// rotary band; rotary splits the 128 channels of a head into bands of 44, 42
-// and 42; finer groups are cut inside the bands, never across them; reading
-// unpacks and scales in one pass per token and head.
+// Method: "lab", Study 6 ("The cache becomes the model"): four-bit codes, two
+// to a byte, with a scale for each (token, head, rotary band); the bands of a
+// head are channels 0-43, 44-85 and 86-127; finer scale groups stay inside one
+// band; a read unpacks and rescales in a single pass per token and head.
 //
 // Arithmetic per group (the same IEEE float32 steps as the activation
 // quantiser): amax, s = amax / 7, inv = 7 / amax, q = clamp(rint(x * inv), -8, 7);

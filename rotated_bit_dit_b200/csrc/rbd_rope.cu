@@ -3,8 +3,8 @@
 //
 // Method: "Krea 2 Turbo OrbitQuant W4A4", "Fused transformer" (each block runs
 // a Q/K RMSNorm + RoPE kernel after the grouped Q|K|V|gate GEMM); "lab",
-// Study 6 (rotary embedding splits the 128 channels of a head into bands of 44
-// for time and 42 each for height and width).
+// Study 6 (a head's rotary bands: channels 0-43 time, 44-85 height, 86-127
+// width).
 //
 // Per token t and head h (128 channels):
 //   r = 1 / sqrt(sum(x^2) / 128 + eps)          (float64, rounded to float32;
