@@ -64,7 +64,8 @@ typedef struct rbd_qcfg {
 } rbd_qcfg;
 
 /* Online activation rotate + dynamic quantise (INT4 tensorwise card, header:
- * "activations rotated online and dynamically quantized inside the kernel").
+ * the activation rotation happens at run time and the quantisation scales are
+ * computed by the kernel itself).
  *   x       bf16 [M, ldx], first K columns used.  ldx >= K, ldx % 8 == 0,
  *           x 16-byte aligned.
  *   M       >= 0 (M == 0 is a no-op).   K: multiple of 256 (rotation) or of 64,
@@ -80,8 +81,8 @@ rbd_status rbd_rot_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, r
                              int8_t* codes, float* scales, void* stream);
 
 /* RMSNorm and adaLN-style modulation fused ahead of rbd_rot_quant_act
- * (Krea 2 Turbo OrbitQuant W4A4, "Fused transformer": the RMSNorm and the
- * modulation run in the activation quantisation prologues).  Per row:
+ * (Krea 2 Turbo OrbitQuant W4A4, "Fused transformer": the norm and the
+ * modulation are folded into the kernels that quantise activations).  Per row:
  *   r = 1 / sqrt(sum_k x_k^2 / K + eps), float64 IEEE operations on the exact
  *       squares, rounded once to float32 (r = 0 when the radicand is 0);
  *   per element, single float32 operations in this order:
@@ -125,7 +126,7 @@ rbd_status rbd_lowrank_down(const void* x, int64_t M, int64_t K, int64_t ldx, co
                             int32_t r, void* ld, void* stream);
 
 /* Offline weight rotate + quantise + pack to signed INT4 (INT4 tensorwise card,
- * header: "packed signed INT4 weights with group-256 ... rotation").
+ * header: the weights are signed four-bit codes, rotated in groups of 256).
  * Each output row of W is rotated and quantised exactly like a token.
  *   w       bf16 [N, K] row-major, 16-byte aligned.    cfg.bits must be 4.
  *   packed  uint8 [N, K/2]: byte k/2 of row n holds code k (even k) in the low
@@ -135,13 +136,15 @@ rbd_status rbd_pack_weights_int4(const void* w, int64_t N, int64_t K, rbd_qcfg c
                                  uint8_t* packed, float* scales, void* stream);
 
 /* Offline per-row INT8 weights for the protected ff.down layers (OrbitQuant
- * card, "What is quantized": per-row INT8 weights for a W8A8 GEMM).
+ * card, "What is quantized": those 28 projections keep eight-bit weights with
+ * one scale per output row and run as W8A8).
  *   w8      int8 [N, K].  cfg.bits must be 8.                                  */
 rbd_status rbd_pack_weights_int8(const void* w, int64_t N, int64_t K, rbd_qcfg cfg,
                                  int8_t* w8, float* scales, void* stream);
 
-/* Epilogue options of the linear calls ("Fused transformer": sigmoid gate in
- * the Q|K|V|gate GEMM epilogue, gated residual updates in the GEMM epilogues;
+/* Epilogue options of the linear calls ("Fused transformer": the Q|K|V|gate
+ * GEMM applies the sigmoid gate on its way out, and the residual adds with
+ * their gates are done by the GEMMs' epilogues as well;
  * "What is quantized": biases are not 4-bit tensors).
  *   bias      bf16 [N] or NULL.
  *   ld, l2t   low-rank branch: ld bf16 [M, r] (from rbd_lowrank_fused) and the

@@ -10,32 +10,34 @@ What it computes (plain, slow, float64 unless a step fixes the precision):
 1. Rotation.  Every 256-wide block of the K axis is multiplied by R = H/16, H
    the regular Hadamard matrix (J4 - 2 I4) Kronecker-powered four times.
    Source: Krea-2 Turbo -- INT4 tensorwise W4A4 (+ConvRot, mixed int8 fallback),
-   header ("group-256 regular-Hadamard ConvRot rotation, activations rotated
-   online"); Krea-2-SVDQuant-ComfyUI, "Why this exists" (the group-wise
-   Hadamard rotation spreads outliers analytically).  The rotated value is
+   header (a regular Hadamard rotation over groups of 256 channels, applied
+   to activations at run time); Krea-2-SVDQuant-ComfyUI, "Why this exists"
+   (rotating by Hadamard blocks spreads outlier channels in closed form, with
+   no calibration).  The rotated value is
    the exact sum rounded once to float32.
 2. Dynamic symmetric quantisation per token (or per 64-wide group) to signed
    INT4 (qmax 7) or INT8 (qmax 127), round half to even, clamp.
-   Source: the INT4 tensorwise model card header ("dynamically quantized
-   inside the kernel"); Krea 2 Turbo OrbitQuant W4A4, "What is quantized"
+   Source: the INT4 tensorwise model card header (the kernel computes the
+   activation scales itself, at run time); Krea 2 Turbo OrbitQuant W4A4, "What is quantized"
    (per-row INT8 ff.down weights with INT8 activations); Krea 2 Turbo Nunchaku
    Lite INT4 r32, header (group size 64, rank 32).
 3. Packed signed INT4 weights, two codes per byte (even k in the low nibble).
-   Source: INT4 tensorwise model card header ("packed signed INT4 weights").
+   Source: INT4 tensorwise model card header (signed four-bit weight codes, packed).
 4. Integer GEMM, exact (int64 here), one partial per 64-group in group mode.
 5. Epilogue in float64: dequant scales, + bias, + low-rank branch
    (X L1) L2 on the unrotated input, then a sigmoid on the gate columns or a
    gated residual out = R + g * y, then one round to bf16.
-   Source: OrbitQuant W4A4 card, "Fused transformer" (sigmoid gate in the
-   Q|K|V|gate GEMM epilogue, gated residual updates in the GEMM epilogues);
-   Krea-2-SVDQuant-ComfyUI, "LoRA" ((W + BA)x == Wx + B(Ax)) and "Why this
-   exists" (low-rank correction branch on top of the W4A4 kernel).
+   Source: OrbitQuant W4A4 card, "Fused transformer" (the Q|K|V|gate GEMM
+   applies the sigmoid gate on its way out; residual adds with their gates are
+   also done in GEMM epilogues); Krea-2-SVDQuant-ComfyUI, "LoRA" (a low-rank
+   term distributes over the product: (W + BA)x = Wx + B(Ax)) and "Why this
+   exists" (the W4A4 kernel carries an extra low-rank term beside it).
 6. NVFP4 variant: E2M1 codes with an E4M3 scale per 16 elements and a float32
    tensor scale.  Source: Nunchaku Lite INT4 r32 card, "Benchmark" (NVFP4 build
    on native FP4 tensor cores).
 7. Normalising prologue: RMSNorm and adaLN-style modulation ahead of the
-   rotation.  Source: OrbitQuant W4A4 card, "Fused transformer" (the RMSNorm
-   and modulation run in the activation quantisation prologues).
+   rotation.  Source: OrbitQuant W4A4 card, "Fused transformer" (the norm and
+   the modulation are folded into the kernels that quantise activations).
 8. INT4 KV-cache codec: packed codes with one float32 scale per token, head
    and group, groups inside the 44 | 42 | 42 rotary bands.  Source: "lab",
    Study 6 (the cache goes to four bits).
@@ -267,8 +269,8 @@ def norm_modulate(x_bits: np.ndarray, gamma_bits=None, shift_bits=None, scale_bi
                   eps: float = 1e-6) -> np.ndarray:
     """RMSNorm and adaLN-style modulation of bf16 rows, returned as bf16 patterns.
 
-    Source: Krea 2 Turbo OrbitQuant W4A4, "Fused transformer": the RMSNorm and
-    the modulation run in the activation quantisation prologues.  The pages
+    Source: Krea 2 Turbo OrbitQuant W4A4, "Fused transformer": the norm and the
+    modulation are folded into the kernels that quantise activations.  The pages
     print no formula; the readings (plainest ones) are:
       - RMS over the whole row: S = sum_k x_k^2 (exact, rounded once to
         float64), ms = S / K, d = ms + eps, r = 1 / sqrt(d), all float64 IEEE
@@ -576,12 +578,13 @@ def kv4_decode(packed: np.ndarray, scales: np.ndarray, groups_per_band: int) -> 
 # 9. Offline SVDQuant fit of the low-rank branch
 # ---------------------------------------------------------------------------
 # Source: Krea-2-SVDQuant-ComfyUI, "Low-rank refinement, and what the
-# objective actually is" and "Activation-aware branch": the branch is fitted
-# by minimising ||W - (Q + L1 L2)||; a seeded randomized SVD gives the first
-# split; the branch is then refit against the current quantisation error and
-# the residual requantised, repeatedly, keeping the best, so refining never
-# does worse; --act-stats weights the objective by a per-input-channel
-# activation RMS d, normalised to mean 1 and floor-clamped at 0.05.
+# objective actually is" and "Activation-aware branch": the objective is the
+# Frobenius distance between W and the quantised part plus the branch; the
+# first split comes from a seeded randomized SVD; after that the branch is
+# re-fitted to what quantisation currently misses and the remainder is
+# quantised again, several times, and the best iterate wins, so extra
+# iterations cannot hurt; with activation statistics each input channel's
+# error counts by that channel's RMS d (scaled to mean 1, never below 0.05).
 # Readings: the residual is rounded to bf16 before it is quantised (the
 # packer's input type); the quantised residual is the layer's own rotated
 # INT4/INT8 format; the randomized SVD's Gaussian test matrices are inputs
@@ -644,7 +647,7 @@ def svdquant_fit(w_bits: np.ndarray, rank: int, bits: int, omegas, rot_group: in
             root = np.sqrt(s)
             vd = vt / d[None, :]             # undo the channel weighting on the input side
             best = dict(l1=(vd.T * root[None, :]), l2=(root[:, None] * u.T), q=q, scales=sc, err=err)
-        target = w - deq                    # refit against the current quantisation error
+        target = w - deq                    # next branch: what the current quantisation misses
     best["errs"] = errs
     return best
 
@@ -654,7 +657,7 @@ def svdquant_fit(w_bits: np.ndarray, rank: int, bits: int, omegas, rot_group: in
 # ---------------------------------------------------------------------------
 # Source: OrbitQuant W4A4 card, "Fused transformer": each block runs a Q/K
 # RMSNorm + RoPE kernel after the Q|K|V|gate GEMM, and attention takes Q.K^T in
-# INT8 and P.V in FP16 (the SageAttention v1 scheme); "lab", Study 6: the
+# INT8 with P.V in FP16, as SageAttention v1 does; "lab", Study 6: the
 # rotary bands of a head are channels 0-43 (time), 44-85 (height) and 86-127
 # (width).
 # Readings (the pages name the scheme, not its steps):

@@ -76,12 +76,6 @@ cudaError_t launch_kv4_encode(const uint16_t* x, int T, int H, int64_t ldt, int 
 cudaError_t launch_kv4_decode(const uint8_t* codes, const float* scales, int64_t capacity, int64_t slot0, int T,
                               int H, int n, uint16_t* y, int64_t ldt, cudaStream_t st);
 
-cudaError_t launch_qk_norm_rope(const uint16_t* x, int64_t ldx, int T, int H, const uint16_t* gamma,
-                                const float* cos_t, const float* sin_t, float eps, uint16_t* y, int64_t ldy,
-                                cudaStream_t st);
-cudaError_t launch_rope_tables(const int32_t* pos, int T, double base, float* cos_t, float* sin_t,
-                               cudaStream_t st);
-
 uint32_t gemm_smem_bytes(bool g64, int r, int G);   // dynamic shared memory of one GEMM CTA
 int gemm_tile_tokens(bool g64);                     // tokens per GEMM tile
 

@@ -48,8 +48,8 @@ struct NormArgs {
 // team `tm` of a row processes 256-blocks g = tm, tm + teams, ... (at most CMAX).
 // OUT_PACKED: write packed INT4 bytes instead of one code per byte.
 // NORM: the row (all of it is in registers) is first normalised and modulated
-// -- "Krea 2 Turbo OrbitQuant W4A4", section "Fused transformer": the RMSNorm
-// and modulation run in the activation quantisation prologues.  The sum of the
+// -- "Krea 2 Turbo OrbitQuant W4A4", section "Fused transformer": the norm and
+// the modulation are folded into the kernels that quantise activations.  The sum of the
 // exact squares is accumulated in float64 and reduced across the row's
 // threads; r = 1 / sqrt(sum / K + eps) (float64 IEEE operations) is rounded
 // once to float32; then per element, as single float32 operations,

@@ -25,6 +25,7 @@
 
 #include "rbd_common.cuh"
 #include "rbd_internal.cuh"
+#include "rbd_rope.cuh"
 
 namespace rbd {
 

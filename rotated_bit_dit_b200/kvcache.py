@@ -1,7 +1,7 @@
 """Int4KVCache: a ring of INT4 key (or value) slots driven by rbd_kv4_encode / rbd_kv4_decode.
 
-The cache offers the three operations a serving loop performs on a KV cache -- a slice
-write, a rolling eviction and a slice read -- ("lab", Study 6: the serving loop touches the
+The cache offers the three operations a serving loop performs on a KV cache -- appending a
+slice, evicting the oldest tokens, reading a slice back -- ("lab", Study 6: the serving loop touches the
 four-bit cache only through these, so it can stand where a bf16 cache tensor stood).  Only the ring's
 bookkeeping lives here; encoding and decoding run in librbd.so.  Token 0 of the cache is the
 oldest one held; slots are reused in ring order, so a write never moves existing codes.  Token
