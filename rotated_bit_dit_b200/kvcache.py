@@ -35,8 +35,7 @@ class Int4KVCache:
     def write(self, x: torch.Tensor) -> None:
         """Append the tokens of x (bf16 [T, heads * 128], row stride may be larger).  When the
         ring is full the oldest tokens are evicted first (rolling)."""
-        if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != self.heads * 128:
-            raise ValueError("x must be bf16 [T, heads * 128]")
+        self._check_slice(x)
         t = x.shape[0]
         if t > self.capacity:
             raise ValueError("slice longer than the cache")
@@ -50,11 +49,16 @@ class Int4KVCache:
     def overwrite(self, first: int, x: torch.Tensor) -> None:
         """Re-encode held tokens first .. first + T - 1 (0 = the oldest held) from x (bf16
         [T, heads * 128]); the ring's start and size do not change."""
-        if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != self.heads * 128:
-            raise ValueError("x must be bf16 [T, heads * 128]")
+        self._check_slice(x)
         if first < 0 or first + x.shape[0] > self.size:
             raise ValueError("overwrite outside the tokens held")
         B.rbd_kv4_encode(x, self.codes, self.scales, self.groups_per_band, (self.start + first) % self.capacity)
+
+    def _check_slice(self, x: torch.Tensor) -> None:
+        if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != self.heads * 128:
+            raise ValueError("x must be bf16 [T, heads * 128]")
+        if x.device != self.codes.device:
+            raise ValueError(f"x is on {x.device}, the cache on {self.codes.device}")
 
     def __len__(self) -> int:
         return self.size
@@ -99,6 +103,8 @@ class Int4KVCache:
             out = torch.empty((count, self.heads * 128), dtype=torch.bfloat16, device=self.codes.device)
         elif out.dtype != torch.bfloat16 or out.dim() != 2 or out.shape[0] < count or out.shape[1] != self.heads * 128:
             raise ValueError("out must be bf16 [>= count, heads * 128]")
+        elif out.device != self.codes.device:
+            raise ValueError(f"out is on {out.device}, the cache on {self.codes.device}")
         if count:
             slot0 = (self.start + first) % self.capacity
             B.rbd_kv4_decode(self.codes, self.scales, out[:count], self.groups_per_band, slot0)

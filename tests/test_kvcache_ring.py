@@ -148,6 +148,8 @@ def test_ring_argument_errors(oracle_codec):
         cache.read(2, 2)
     with pytest.raises(ValueError):
         cache.read(0, 3, out=torch.empty((2, 128), dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        cache.write(torch.zeros((1, 128), dtype=torch.bfloat16, device="meta"))      # another device
     for bad in [dict(capacity=0, heads=1), dict(capacity=4, heads=0), dict(capacity=4, heads=1, groups_per_band=3)]:
         with pytest.raises(ValueError):
             R.Int4KVCache(device="cpu", **bad)
