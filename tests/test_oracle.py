@@ -4,6 +4,7 @@ Each test is chosen so that a plausible slip in the oracle (a wrong Hadamard
 construction, a transposed operand, a dropped 1/16, a wrong tie rule, a lost
 scale, a wrong nibble order, a sign error in the epilogue) fails at least one.
 """
+import math
 from fractions import Fraction
 
 import numpy as np
@@ -268,6 +269,31 @@ def test_epilogue_special_cases():
     assert np.all(out[:, 4:] == 0.5) and np.all(out[:, :4] == 0.0)
 
 
+def test_epilogue_sigmoid_values_symmetry_and_sign():
+    # closed forms: sigmoid(ln 3) = 3/4, sigmoid(-ln 3) = 1/4; a sign slip inside the
+    # exponential swaps them, which the value at 0 alone cannot show
+    y = np.array([[math.log(3.0), -math.log(3.0), 0.0, math.log(9.0)]])
+    out = O.epilogue(y, gate_mode=1, gate_cols=(0, 4))
+    assert np.allclose(out, [[0.75, 0.25, 0.5, 0.9]], rtol=0, atol=1e-15)
+    rng = np.random.default_rng(41)
+    v = rng.standard_normal((6, 40)) * 4.0
+    s_pos = O.epilogue(v, gate_mode=1, gate_cols=(0, 40))
+    s_neg = O.epilogue(-v, gate_mode=1, gate_cols=(0, 40))
+    # sigmoid(-y) = 1 - sigmoid(y)
+    assert np.allclose(s_neg, 1.0 - s_pos, rtol=0, atol=1e-15)
+    # strictly increasing in y, inside (0, 1), above 1/2 exactly where y > 0
+    order = np.argsort(v.ravel())
+    assert np.all(np.diff(s_pos.ravel()[order]) >= 0)
+    assert np.all((s_pos > 0) & (s_pos < 1))
+    assert np.array_equal(s_pos > 0.5, v > 0)
+    # the gate applies to the gate columns only, after bias is added
+    b = I.f32_to_bf16_bits(np.full(8, 2.0, np.float32))
+    z = np.zeros((1, 8))
+    g = O.epilogue(z, bias=b, gate_mode=1, gate_cols=(6, 8))
+    assert np.allclose(g[0, 6:], 1.0 / (1.0 + math.exp(-2.0)), rtol=0, atol=1e-15)
+    assert np.array_equal(g[0, :6], np.full(6, 2.0))
+
+
 def test_lowrank_branch_is_parallel_linear():
     # (W + L1 L2)-style branch: X L1 L2 added once, on the unrotated input
     x = I.gaussian_bf16(6, (3, 256))
@@ -343,6 +369,55 @@ def test_nvfp4_block_error_bound_and_scale_range():
     assert np.all(np.abs(xr - deq) <= step / 2 * 1.0001 + 1e-30)
     rel = np.linalg.norm(xr - deq) / np.linalg.norm(xr)
     assert rel < 0.12
+
+
+def _nvfp4_exact_operand(seed, rows, k, tensor_scale):
+    """bf16 rows whose 16-blocks are E2M1 grid values times one E4M3 block scale times a
+    power-of-two tensor scale; every block holds a +-6 and one block has scale 448, so the
+    two-level quantiser reproduces them exactly."""
+    rng = np.random.default_rng(seed)
+    grid = np.concatenate([-O.E2M1_GRID[1:], O.E2M1_GRID])
+    e4m3 = np.array([0.125, 0.25, 0.375, 0.5, 0.75, 1.0, 1.25, 2.5, 3.0, 6.5, 13.0, 24.0, 104.0, 448.0])
+    q = rng.choice(grid, (rows, k // 16, 16))
+    q[:, :, 0] = rng.choice([-6.0, 6.0], (rows, k // 16))
+    bs = rng.choice(e4m3, (rows, k // 16))
+    bs[0, 0] = 448.0
+    v = (q * bs[..., None] * tensor_scale).reshape(rows, k)
+    bits = I.f32_to_bf16_bits(v.astype(np.float32))
+    assert np.array_equal(O.bf16_to_f64(bits), v)            # exactly representable
+    return bits
+
+
+def test_nvfp4_linear_exact_on_representable_operands():
+    # unrotated, operands already on the two-level NVFP4 grid: the layer must return the
+    # plain float64 product exactly (catches a tensor scale applied once instead of twice,
+    # a block scale repeated wrongly, or a transposed operand)
+    x = _nvfp4_exact_operand(50, 5, 64, 2.0 ** -3)
+    w = _nvfp4_exact_operand(51, 7, 64, 2.0 ** -9)
+    got = O.nvfp4_linear(x, w, rot_group=0)
+    want = O.bf16_to_f64(x) @ O.bf16_to_f64(w).T
+    assert np.array_equal(got, want)
+
+
+def test_nvfp4_linear_rotated_within_the_quantisation_bound():
+    # with rotation both operands are rotated: X W^T = (XR)(WR)^T, so the result stays within the
+    # per-element half-step bound of the unrotated float64 product.  W holds X's own rows, so the
+    # diagonal is the large |x|^2; forgetting to rotate W would leave (XR) W^T, outside the bound
+    x = I.gaussian_bf16(52, (6, 512), 1.0, 0.01, 30.0)
+    w = np.concatenate([x, I.gaussian_bf16(53, (3, 512), 0.02)])
+    got = O.nvfp4_linear(x, w)
+    xr, wr = O.rotate(O.bf16_to_f64(x)), O.rotate(O.bf16_to_f64(w))
+    qx, bsx, gsx = O.nvfp4_quantize(xr)
+    qw, bsw, gsw = O.nvfp4_quantize(wr)
+    hx = np.repeat(bsx, 16, axis=1) * float(gsx)       # half of the largest grid step, per element
+    hw = np.repeat(bsw, 16, axis=1) * float(gsw)
+    bound = hx @ (np.abs(wr) + hw).T + np.abs(xr) @ hw.T
+    exact = O.bf16_to_f64(x) @ O.bf16_to_f64(w).T
+    assert np.all(np.abs(got - exact) <= bound * (1 + 1e-9) + 1e-12)
+    # the test has the power to see the slip: W quantised unrotated breaks the bound
+    qu, bsu, gsu = O.nvfp4_quantize(O.bf16_to_f64(w))
+    slip = (qx * hx) @ (qu * np.repeat(bsu, 16, axis=1) * float(gsu)).T
+    assert np.any(np.abs(slip - exact) > bound)
 
 
 # --------------------------------------------------------------- normalising prologue
@@ -582,6 +657,19 @@ def test_qk_norm_rope_reduces_to_rms_norm_at_position_zero():
         xt = torch.from_numpy(O.bf16_to_f64(x))
         want = torch.nn.functional.rms_norm(xt, (128,), torch.from_numpy(O.bf16_to_f64(g)), eps).numpy()
         assert np.array_equal(got, O.f64_to_bf16(want))
+
+
+def test_qk_norm_rope_zero_head_gives_zero():
+    # a head whose radicand mean(x^2) + eps is 0 (all zero, eps = 0) normalises to 0, not NaN;
+    # with eps > 0 the same head is 0 too, and a nonzero head next to it is unaffected
+    x = np.zeros((3, 2, 128), np.uint16)
+    x[:, 1] = I.gaussian_bf16(1003, (3, 128), 1.0)
+    cos, sin = O.rope_tables(np.array([[1, 2, 3], [4, 5, 6], [0, 0, 0]]))
+    for eps in (0.0, 1e-6):
+        out = O.qk_norm_rope_f64(x, None, cos, sin, eps)
+        assert np.all(np.isfinite(out))
+        assert np.all(out[:, 0] == 0.0)
+        assert np.allclose((out[:, 1] ** 2).mean(axis=-1), 1.0, rtol=1e-5)
 
 
 def test_qk_norm_rope_quarter_turn_and_pair_norms():
