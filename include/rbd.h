@@ -236,6 +236,10 @@ rbd_status rbd_nvfp4_quant(const void* x, int64_t M, int64_t K, int64_t ldx, int
  * stream capture).  The word is cleared at the start of every call.  All calls
  * on a device share the array, so calls that overlap in time (other streams,
  * other host threads) race and give wrong results.  Allocates nothing.
+ * The looked-up address is kept for the life of the process: a device reset
+ * (cudaDeviceReset, or another library resetting the primary context) after
+ * the first call on that device is not supported, since the kept address then
+ * points into freed memory.
  * Arguments and results as rbd_nvfp4_quant.                                   */
 rbd_status rbd_nvfp4_quant_noalloc(const void* x, int64_t M, int64_t K, int64_t ldx, int32_t rot_group,
                                    uint8_t* codes, uint8_t* block_scales, float* tensor_scale,

@@ -2,7 +2,8 @@
 
 Argument marshalling only.  Every computation runs in the library's CUDA
 kernels; there is no Python or CPU fallback.  Tensors must be CUDA tensors on
-the current device; the current torch stream is used unless `stream` is given.
+the current device (others are refused before any launch); the current torch
+stream is used unless `stream` is given.
 """
 from __future__ import annotations
 
@@ -93,10 +94,17 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
 
 
 def _ptr(t: Optional[torch.Tensor]):
+    """Device address of t.  Every kernel launches on the current device, so a tensor that
+    lives on another device is refused here, before any launch (its address would be
+    dereferenced by the wrong GPU)."""
     if t is None:
         return None
     if not t.is_cuda:
         raise ValueError("expected a CUDA tensor")
+    cur = torch.cuda.current_device()
+    if t.device.index is not None and t.device.index != cur:
+        raise ValueError(f"tensor on {t.device} while cuda:{cur} is current; "
+                         f"call under torch.cuda.device({t.device})")
     return ctypes.c_void_p(t.data_ptr())
 
 

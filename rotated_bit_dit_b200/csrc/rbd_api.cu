@@ -87,7 +87,8 @@ static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoallocScratchWords
 
 // Device address of the scratch array for the current device.  The first call
 // on a device resolves it with cudaGetSymbolAddress (a runtime call that should
-// happen before any stream capture); later calls reuse the cached address.
+// happen before any stream capture); later calls reuse the cached address, so
+// a device reset after the first call on a device is not supported.
 rbd_status noalloc_scratch(uint32_t** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RBD_ERR_CUDA;

@@ -39,12 +39,14 @@ class Int4KVCache:
         t = x.shape[0]
         if t > self.capacity:
             raise ValueError("slice longer than the cache")
-        overflow = self.size + t - self.capacity
-        if overflow > 0:
-            self.evict(overflow)
-        slot0 = (self.start + self.size) % self.capacity
+        # the ring's bookkeeping moves only once the encode has been accepted: a refused call
+        # (bad stride, alignment, device) leaves the held tokens as they were
+        overflow = max(self.size + t - self.capacity, 0)
+        start = (self.start + overflow) % self.capacity
+        size = self.size - overflow
+        slot0 = (start + size) % self.capacity
         B.rbd_kv4_encode(x, self.codes, self.scales, self.groups_per_band, slot0)
-        self.size += t
+        self.start, self.size = start, size + t
 
     def overwrite(self, first: int, x: torch.Tensor) -> None:
         """Re-encode held tokens first .. first + T - 1 (0 = the oldest held) from x (bf16

@@ -48,7 +48,10 @@ class RotatedLowBitLinear:
         self._host_pipes = {}   # forward_host: streams and staging buffers per (device, chunk, residual)
 
     def buffers(self, M: int, device):
-        key = (M, str(device))
+        """The call's intermediates (codes, scales, low-rank Ld) for M tokens, kept per
+        (M, device, current stream): calls queued on different streams never share them, so
+        one stream's prologue cannot overwrite codes another stream's GEMM has yet to read."""
+        key = (M, str(device), torch.cuda.current_stream(device).cuda_stream)
         if key not in self._bufs:
             G = self.K // 64 if self.scale_group else 1
             codes = torch.empty((M, self.K), dtype=torch.int8, device=device)

@@ -60,3 +60,29 @@ def test_package_fails_loudly_without_the_library(tmp_path, monkeypatch):
     monkeypatch.setattr(B, "load", missing)
     with pytest.raises(RuntimeError):
         B.rbd_version()
+
+
+def test_tensor_on_another_device_is_refused_before_any_launch(monkeypatch):
+    """Every kernel runs on the current device, so a pointer to another GPU's memory must be
+    refused on the host (it would otherwise be dereferenced by the wrong GPU).  Host-side
+    only: a stand-in tensor and a stand-in current device, no launch."""
+    import torch
+    from rotated_bit_dit_b200 import _binding as B
+
+    class FakeCudaTensor:
+        is_cuda = True
+
+        def __init__(self, index):
+            self.device = torch.device("cuda", index)
+
+        def data_ptr(self):
+            return 0x1000
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    assert B._ptr(FakeCudaTensor(0)).value == 0x1000
+    with pytest.raises(ValueError, match="cuda:1"):
+        B._ptr(FakeCudaTensor(1))
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 1)
+    assert B._ptr(FakeCudaTensor(1)).value == 0x1000
+    with pytest.raises(ValueError):
+        B._ptr(FakeCudaTensor(0))

@@ -154,3 +154,18 @@ def test_forward_host_matches_the_device_call(bits, sg, rank, gate_mode):
     torch.cuda.synchronize()
     assert R.rbd_check() == 0
     assert np.array_equal(yh.view(torch.int16).numpy().view(np.uint16), y_dev)
+
+
+def test_intermediates_are_kept_per_stream():
+    # calls queued on two streams must not share codes / scales / Ld buffers
+    case = build_case(64, 256, 256, 4, 64, seed=70, rank=16)
+    _, _, layer = run_layer(case)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    with torch.cuda.stream(s1):
+        b1 = layer.buffers(64, torch.device("cuda"))
+    with torch.cuda.stream(s2):
+        b2 = layer.buffers(64, torch.device("cuda"))
+    with torch.cuda.stream(s1):
+        b1b = layer.buffers(64, torch.device("cuda"))
+    assert b1[0].data_ptr() != b2[0].data_ptr() and b1[1].data_ptr() != b2[1].data_ptr()
+    assert b1[0].data_ptr() == b1b[0].data_ptr()

@@ -156,6 +156,30 @@ def test_ring_argument_errors(oracle_codec):
     assert not [c for c in oracle_codec if c[1] > 4]
 
 
+def test_refused_write_leaves_the_ring_unchanged(oracle_codec, monkeypatch):
+    # a write that would roll the ring but whose encode is refused (here: the stand-in raises the
+    # library's error for any slice of 3 tokens) must not evict anything or move the ring
+    cache = R.Int4KVCache(6, 1, 1, device="cpu")
+    xb = I.gaussian_bf16(970, (5, 1, 128), 1.0, 0.02, 12.0)
+    cache.write(_bf16(xb.reshape(5, 128), "cpu"))
+    good = K.B.rbd_kv4_encode
+
+    def refusing(x, codes, scales, n=1, slot0=0, stream=None):
+        if x.shape[0] == 3:
+            raise K.B.RbdError(3, "rbd_kv4_encode")
+        return good(x, codes, scales, n, slot0, stream)
+
+    monkeypatch.setattr(K.B, "rbd_kv4_encode", refusing)
+    with pytest.raises(K.B.RbdError):
+        cache.write(_bf16(I.gaussian_bf16(971, (3, 128)), "cpu"))
+    assert (cache.start, len(cache)) == (0, 5)
+    p, s = O.kv4_encode(xb, 1)
+    assert np.array_equal(_bits(cache[:]).reshape(5, 1, 128), O.kv4_decode(p, s, 1))
+    # an accepted write afterwards rolls as usual
+    cache.write(_bf16(I.gaussian_bf16(972, (2, 128)), "cpu"))
+    assert (cache.start, len(cache)) == (1, 6)
+
+
 @pytest.mark.gpu
 @pytest.mark.parametrize("n", [1, 2, 4])
 def test_gpu_ring_script_against_the_oracle(n):
