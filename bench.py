@@ -322,7 +322,7 @@ def run_ours(args, cfg, t):
 
 GEMM_SOURCES = [os.path.join(ROOT, "rotated_bit_dit_b200", "csrc", f)
                 for f in ("rbd_gemm.cu", "rbd_common.cuh", "rbd_internal.cuh")]
-TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "lowbit_gemm_w4a4_qkvg.md")
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "lowbit_gemm_w4a4_qkvg.json")
 
 
 def gemm_source_hash():
@@ -333,6 +333,73 @@ def gemm_source_hash():
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------- tensor ceilings
+PEAKS_FILE = os.path.join(ROOT, "profiles", "peaks.json")
+
+
+def run_peaks(args):
+    """Dense tensor-core ceilings of library GEMMs on this GPU, for the roofline denominators:
+    INT8 (torch._int_mm, int32 out) and FP8 E4M3 (torch._scaled_mm, bf16 out) at 8192^3, each the
+    best of 10 single calls (burst) and the mean over a 4 s back-to-back loop (sustained), with
+    the SM clocks sampled during the loops.  Prints one JSON line (kept as profiles/peaks.json)."""
+    import torch
+    dev = torch.device("cuda", 0)
+    n = 8192
+    ops = 2.0 * n ** 3
+    out = {"what": "dense GEMM ceilings, 8192^3, CUDA events", "gpu": torch.cuda.get_device_name(dev),
+           "torch": torch.__version__}
+
+    def measure(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            best = min(best, a.elapsed_time(b) / 1e3)
+        with ClockSampler(0) as clk:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            calls = max(8, int(4.0 / best))
+            a.record()
+            for _ in range(calls):
+                fn()
+            b.record()
+            b.synchronize()
+        sus = a.elapsed_time(b) / 1e3 / calls
+        return {"burst_tops": ops / best / 1e12, "sustained_tops": ops / sus / 1e12, "clocks": clk.summary()}
+
+    g = torch.Generator(device=dev).manual_seed(0)
+    a8 = torch.randint(-128, 128, (n, n), dtype=torch.int8, device=dev, generator=g)
+    b8 = torch.randint(-128, 128, (n, n), dtype=torch.int8, device=dev, generator=g).t()
+    try:
+        out["int8"] = measure(lambda: torch._int_mm(a8, b8))
+        out["int8"]["call"] = "torch._int_mm int8 x int8 -> int32"
+    except RuntimeError as e:
+        out["int8"] = {"unavailable": str(e).splitlines()[0]}
+    del a8, b8
+    af = torch.randn((n, n), device=dev, generator=g).to(torch.float8_e4m3fn)
+    bf = torch.randn((n, n), device=dev, generator=g).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), dtype=torch.float32, device=dev)
+    try:
+        out["fp8_e4m3"] = measure(lambda: torch._scaled_mm(af, bf, one, one, out_dtype=torch.bfloat16))
+        out["fp8_e4m3"]["call"] = "torch._scaled_mm e4m3 x e4m3 -> bf16, tensor scales"
+    except RuntimeError as e:
+        out["fp8_e4m3"] = {"unavailable": str(e).splitlines()[0]}
+    print(json.dumps(out), flush=True)
+
+
+def load_tensor_peaks():
+    """Measured INT8 / FP8 dense ceilings (profiles/peaks.json) or None when not measured."""
+    if not os.path.exists(PEAKS_FILE):
+        return None
+    with open(PEAKS_FILE) as f:
+        return json.load(f)
 
 
 # ----------------------------------------------------------------------------- small-M sweep
@@ -757,23 +824,17 @@ def run_stack(args):
 
 
 def _profile_traffic():
-    """DRAM bytes per GEMM launch from the committed ncu summary.  The summary
-    records the hash of the GEMM source it was captured from; a summary of an
-    older kernel gives no figure (null)."""
-    if not os.path.exists(TRAFFIC_SUMMARY):
+    """DRAM bytes per GEMM launch from the committed ncu record (a small JSON beside the
+    summary).  The record carries the hash of the GEMM source it was captured from; a record
+    of an older kernel gives no figure (null)."""
+    if not os.path.exists(TRAFFIC_RECORD):
         return None
-    fields = {}
-    with open(TRAFFIC_SUMMARY) as f:
-        for ln in f:
-            if ln.startswith("- ") and ":" in ln:
-                k, v = ln[2:].split(":", 1)
-                fields[k.strip()] = v.strip().strip("`")
-    if fields.get("source_sha256_16") != gemm_source_hash():
+    with open(TRAFFIC_RECORD) as f:
+        rec = json.load(f)
+    if rec.get("source_sha256_16") != gemm_source_hash():
         return None
-    try:
-        return int(fields["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+    v = rec.get("dram_bytes_per_launch")
+    return int(v) if isinstance(v, (int, float)) else None
 
 
 def main():
@@ -784,11 +845,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--print-gemm-hash", action="store_true", help="print the GEMM source hash and exit")
-    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4", "nvfp4", "qknorm"], default=None,
+    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4", "nvfp4", "qknorm", "peaks"], default=None,
                     help="instead of the headline line, print the small-token-count sweep (one line per case)")
     args = ap.parse_args()
     if args.print_gemm_hash:
         print(gemm_source_hash())
+        return
+    if args.sweep == "peaks":
+        run_peaks(args)
         return
     if args.sweep == "small-m":
         run_small_m_sweep(args)

@@ -102,6 +102,22 @@ def test_long_k_group_scales_two_stage_pipeline(bits, rank):
     check_output(y, ref["ref64"], ref["ref_bf16"])
 
 
+@pytest.mark.parametrize("M,N,K,bits,sg,rank", [
+    (2048, 2560, 512, 4, 64, 32),     # group scales: 320 tiles of 128 x 128 over 148 CTAs
+    (4096, 2048, 1024, 8, 0, 0),      # row scales: 256 tiles of 128 x 256
+    (4096, 2048, 512, 4, 0, 16),      # INT4 row scales, 256 tiles
+    (1500, 2304, 256, 8, 64, 0),      # INT8 group scales, 216 tiles, ragged last token tile
+])
+def test_persistent_grid_exact_accumulators(M, N, K, bits, sg, rank):
+    # more tiles than CTAs: every CTA walks several tiles, so the accumulator buffers' phases wrap
+    # across tiles and the per-tile scale tables are restaged; every int32 accumulator is checked
+    case = build_case(M, N, K, bits, sg, seed=80 + M % 97, rank=rank, bias=True)
+    y, acc, _ = run_layer(case, acc_debug=True)
+    ref = reference(case)
+    assert np.array_equal(acc.astype(np.int64), exact_acc(case, ref))
+    check_output(y, ref["ref64"], ref["ref_bf16"])
+
+
 def test_deterministic_run_to_run():
     case = build_case(300, 512, 1024, 4, 64, seed=30, rank=32, bias=True, gate_mode=1, gate_cols=(0, 128))
     y1, _, layer = run_layer(case)

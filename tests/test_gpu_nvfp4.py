@@ -147,6 +147,28 @@ def test_nvfp4_linear_small_m_sweep_shape():
     assert stats["rel64"] < 5e-3
 
 
+def test_nvfp4_linear_qkvg_shape_sampled_rows():
+    # the Q|K|V|gate layer shape the NVFP4 sweep times (M = 4096, K = 3072, N = 12288, rank-32
+    # branch, sigmoid on the last quarter), checked on sampled token rows.  The activation tensor
+    # scale depends on every row, so both operands are quantised whole and only the product is
+    # restricted to the sampled rows.
+    cfg = I.CONFIGS["w4a4_qkvg"]
+    t = I.make_layer_inputs(cfg, seed=0)
+    M, N = cfg["M"], cfg["N"]
+    kw = dict(l1=t["l1"], l2=t["l2"], gate_mode=1, gate_cols=cfg["gate_cols"])
+    y = run_linear(t["x"], t["w"], **kw)
+    rng = np.random.default_rng(7)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 40, replace=False)]))
+    xq, xbs, xgs = O.nvfp4_quantize(O.rotate(O.bf16_to_f64(t["x"])))
+    wq, wbs, wgs = O.nvfp4_quantize(O.rotate(O.bf16_to_f64(t["w"])))
+    xd = xq[rows] * np.repeat(xbs[rows], 16, axis=1) * float(xgs)
+    wd = wq * np.repeat(wbs, 16, axis=1) * float(wgs)
+    ld = O.bf16_to_f64(O.f64_to_bf16(O.lowrank_down(t["x"][rows], t["l1"])))
+    ref64 = O.epilogue(xd @ wd.T, None, ld, t["l2"], 1, cfg["gate_cols"])
+    stats = check_output(y[rows], ref64, O.f64_to_bf16(ref64))
+    assert stats["rel64"] < 5e-3
+
+
 def test_nvfp4_linear_low_rank_branch_is_added():
     # the branch must change the output by exactly its own contribution (within tolerance):
     # the same layer with L2 = 0 gives the plain result
