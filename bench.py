@@ -228,10 +228,10 @@ def run_ours(args, cfg, t):
     def step(ev=None):
         if ev:
             ev[0].record()
-        B.rbd_lowrank_fused(x, codes, sx, layer.l1t, ld, 4, 256, 64)
+        B.rbd_lowrank_fused(x, codes, sx, layer.l1t, ld, 4, 256, 64, code_format=layer.code_format)
         if ev:
             ev[1].record()
-        B.rbd_w4a4_linear(codes, sx, layer.wq, layer.sw, out, 64, epi)
+        B.rbd_w4a4_linear(codes, sx, layer.wq, layer.sw, out, 64, epi, code_format=layer.code_format)
         if ev:
             ev[2].record()
 
@@ -540,11 +540,14 @@ def run_prologue_sweep(args):
         l1t = up(I.gaussian_bf16(7, (r, K), 0.01))
         ld = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
         base = M * K * 2 + M * K + (M * (K // 64) if sg else M) * 4
-        cases = [("rot_quant", lambda: B.rbd_rot_quant_act(x, codes, sx, bits, 256, sg), base),
+        cf = B.CODES_E4M3 if (bits == 4 and sg == 64) else B.CODES_INT8   # as the layer stores them
+        cases = [("rot_quant", lambda: B.rbd_rot_quant_act(x, codes, sx, bits, 256, sg, code_format=cf), base),
                  ("norm_rot_quant", lambda: B.rbd_norm_rot_quant_act(x, codes, sx, gamma, shift, scale, 1e-6,
-                                                                     bits, 256, sg), base + 3 * K * 2)]
+                                                                     bits, 256, sg, code_format=cf),
+                  base + 3 * K * 2)]
         if sg == 64:
-            cases.append(("rot_quant_lowrank", lambda: B.rbd_lowrank_fused(x, codes, sx, l1t, ld, bits, 256, sg),
+            cases.append(("rot_quant_lowrank", lambda: B.rbd_lowrank_fused(x, codes, sx, l1t, ld, bits, 256, sg,
+                                                                           code_format=cf),
                           base + M * r * 2 + r * K * 2))
         for cname, fn, nbytes in cases:
             for _ in range(max(args.warmup, 3)):

@@ -48,6 +48,19 @@ typedef enum rbd_status {
   RBD_ERR_DEVICE_TIMEOUT = 5  /* a device-side bounded wait expired              */
 } rbd_status;
 
+/* How activation codes are stored, one code per byte either way.  The codes
+ * themselves (the integers) are the same; only the byte that holds one differs.
+ *   RBD_CODES_INT8  the code as a two's-complement int8.
+ *   RBD_CODES_E4M3  the code as the E4M3 (8-bit float, 4 exponent and 3
+ *                   mantissa bits, bias 7) value equal to it; every INT4 code
+ *                   is exact in E4M3.  4-bit codes only.  rbd_w4a4_linear
+ *                   with group-64 scales runs these on the FP8 tensor-core
+ *                   path (fp32 group partials, exact for 64-wide groups).    */
+typedef enum rbd_code_format {
+  RBD_CODES_INT8 = 0,
+  RBD_CODES_E4M3 = 1
+} rbd_code_format;
+
 /* Quantisation configuration.
  *   bits        4 (signed INT4, codes in [-8,7], produced range [-7,7]) or
  *               8 (signed INT8, produced range [-127,127]).
@@ -56,11 +69,17 @@ typedef enum rbd_status {
  *               0: no rotation.
  *   scale_group 0: one scale per row (per token for activations, per output
  *               channel for weights); 64: one scale per 64-wide K block of a
- *               row (group-64 scales).                                        */
+ *               row (group-64 scales).
+ *   code_format an rbd_code_format: how activation codes are stored (written
+ *               by the quantisers, read by the linears).  Weight packers take
+ *               RBD_CODES_INT8 only.  RBD_CODES_E4M3 needs bits == 4 (else
+ *               RBD_ERR_UNSUPPORTED); the linears take it with group-64 scales
+ *               only.  Zero-initialising the struct selects RBD_CODES_INT8.  */
 typedef struct rbd_qcfg {
   int32_t bits;
   int32_t rot_group;
   int32_t scale_group;
+  int32_t code_format;
 } rbd_qcfg;
 
 /* Online activation rotate + dynamic quantise (INT4 tensorwise card, header:
@@ -70,7 +89,8 @@ typedef struct rbd_qcfg {
  *           x 16-byte aligned.
  *   M       >= 0 (M == 0 is a no-op).   K: multiple of 256 (rotation) or of 64,
  *           K <= 16384.
- *   codes   int8 [M, K] (one code per byte), 16-byte aligned.
+ *   codes   [M, K], one code per byte in cfg.code_format (two's-complement
+ *           int8, or the equal E4M3 value for 4-bit codes), 16-byte aligned.
  *   scales  float32 [M] (scale_group 0) or [M, K/64] (scale_group 64);
  *           dequantised value = code * scale.
  * Per row (or per 64 block): amax = max |xr|, scale = amax/qmax,
@@ -172,10 +192,17 @@ typedef struct rbd_epilogue {
   int32_t* acc_debug;
 } rbd_epilogue;
 
-/* W4A4 linear: INT4 activation codes (int8 containers, from rbd_rot_quant_act
- * with bits 4) times packed INT4 weights (rbd_pack_weights_int4), int32
- * accumulation on the tcgen05 INT8 tensor path, then the epilogue.
- *   codes   int8 [M, K], sx float32 [M] or [M, K/64].
+/* W4A4 linear: INT4 activation codes (from rbd_rot_quant_act with bits 4)
+ * times packed INT4 weights (rbd_pack_weights_int4), then the epilogue.
+ *   cfg.code_format RBD_CODES_INT8: int32 accumulation on the tcgen05 INT8
+ *           tensor path.  RBD_CODES_E4M3 (group-64 scales only): the weight
+ *           nibbles are widened to E4M3 and each 64-wide group partial is
+ *           accumulated in float32 on the FP8 tensor path, exactly (every
+ *           partial is an integer of magnitude <= 4096).  Both give the same
+ *           integer partials; the E4M3 path promotes them with two float32
+ *           operations per element and group instead of three.
+ *   codes   [M, K] one code per byte in cfg.code_format, sx float32 [M] or
+ *           [M, K/64].
  *   w_packed uint8 [N, K/2], sw float32 [N] or [N, K/64].
  *   K % 128 == 0, N % 128 == 0, M >= 1 (ragged M is handled).  A shape whose
  *   per-tile scale table does not fit in shared memory (group scales with a

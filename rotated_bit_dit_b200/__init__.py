@@ -6,6 +6,8 @@ Importing the package does not load the library; the first call does, and it
 raises if the library cannot be loaded (there is no CPU fallback).
 """
 from ._binding import (  # noqa: F401
+    CODES_E4M3,
+    CODES_INT8,
     EXPORTED,
     Epilogue,
     QCfg,

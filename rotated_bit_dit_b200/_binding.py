@@ -30,8 +30,13 @@ class RbdError(RuntimeError):
         self.status = status
 
 
+CODES_INT8 = 0   # activation code stored as a two's-complement int8
+CODES_E4M3 = 1   # activation code stored as the E4M3 byte of the same value (4-bit codes)
+
+
 class QCfg(ctypes.Structure):
-    _fields_ = [("bits", ctypes.c_int32), ("rot_group", ctypes.c_int32), ("scale_group", ctypes.c_int32)]
+    _fields_ = [("bits", ctypes.c_int32), ("rot_group", ctypes.c_int32), ("scale_group", ctypes.c_int32),
+                ("code_format", ctypes.c_int32)]
 
 
 class Epilogue(ctypes.Structure):
@@ -121,8 +126,8 @@ def _ok(status: int, where: str):
         raise RbdError(status, where)
 
 
-def _qcfg(bits: int, rot_group: int, scale_group: int) -> QCfg:
-    return QCfg(bits, rot_group, scale_group)
+def _qcfg(bits: int, rot_group: int, scale_group: int, code_format: int = CODES_INT8) -> QCfg:
+    return QCfg(bits, rot_group, scale_group, code_format)
 
 
 def _rowstride(t: torch.Tensor) -> int:
@@ -133,17 +138,18 @@ def _rowstride(t: torch.Tensor) -> int:
 
 # ---------------------------------------------------------------- entry points
 def rbd_rot_quant_act(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, bits: int = 4,
-                      rot_group: int = 256, scale_group: int = 0, stream=None) -> None:
-    """x bf16 [M, K] -> codes int8 [M, K], scales float32 [M] or [M, K/64]."""
+                      rot_group: int = 256, scale_group: int = 0, stream=None, code_format: int = CODES_INT8) -> None:
+    """x bf16 [M, K] -> codes [M, K] (one byte each, in code_format), scales float32 [M] or [M, K/64]."""
     M, K = x.shape
-    _ok(load().rbd_rot_quant_act(_ptr(x), M, K, _rowstride(x), _qcfg(bits, rot_group, scale_group),
+    _ok(load().rbd_rot_quant_act(_ptr(x), M, K, _rowstride(x), _qcfg(bits, rot_group, scale_group, code_format),
                                  _ptr(codes), _ptr(scales), _stream(stream)), "rbd_rot_quant_act")
 
 
 def rbd_norm_rot_quant_act(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
                            gamma: Optional[torch.Tensor] = None, shift: Optional[torch.Tensor] = None,
                            scale: Optional[torch.Tensor] = None, eps: float = 1e-6, bits: int = 4,
-                           rot_group: int = 256, scale_group: int = 0, stream=None) -> None:
+                           rot_group: int = 256, scale_group: int = 0, stream=None,
+                           code_format: int = CODES_INT8) -> None:
     """RMSNorm (optional gamma) and modulation x*(1 + scale) + shift, then rbd_rot_quant_act.
     gamma, shift, scale: bf16 [K] or None."""
     M, K = x.shape
@@ -151,19 +157,19 @@ def rbd_norm_rot_quant_act(x: torch.Tensor, codes: torch.Tensor, scales: torch.T
         if v is not None and (v.numel() != K or not v.is_contiguous()):
             raise ValueError(f"{name} must be a contiguous bf16 vector of length K")
     _ok(load().rbd_norm_rot_quant_act(_ptr(x), M, K, _rowstride(x), _ptr(gamma), _ptr(shift), _ptr(scale),
-                                      float(eps), _qcfg(bits, rot_group, scale_group), _ptr(codes),
+                                      float(eps), _qcfg(bits, rot_group, scale_group, code_format), _ptr(codes),
                                       _ptr(scales), _stream(stream)), "rbd_norm_rot_quant_act")
 
 
 def rbd_lowrank_fused(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, l1t: torch.Tensor,
                       ld: torch.Tensor, bits: int = 4, rot_group: int = 256, scale_group: int = 0,
-                      stream=None) -> None:
+                      stream=None, code_format: int = CODES_INT8) -> None:
     """rbd_rot_quant_act plus ld = X @ L1 (l1t = L1^T bf16 [r, K], ld bf16 [M, r])."""
     M, K = x.shape
     r = l1t.shape[0]
     if _rowstride(l1t) != K:
         raise ValueError("l1t must be a contiguous [r, K] tensor")
-    _ok(load().rbd_lowrank_fused(_ptr(x), M, K, _rowstride(x), _qcfg(bits, rot_group, scale_group),
+    _ok(load().rbd_lowrank_fused(_ptr(x), M, K, _rowstride(x), _qcfg(bits, rot_group, scale_group, code_format),
                                  _ptr(codes), _ptr(scales), _ptr(l1t), r, _ptr(ld), _stream(stream)),
         "rbd_lowrank_fused")
 
@@ -210,20 +216,21 @@ def make_epilogue(bias=None, ld=None, l2t=None, gate_mode: int = 0, gate_cols=(0
     return e
 
 
-def _linear(fn, where, codes, sx, w, sw, y, bits, rot_group, scale_group, epi, stream):
+def _linear(fn, where, codes, sx, w, sw, y, bits, rot_group, scale_group, epi, stream, code_format=CODES_INT8):
     M, K = codes.shape
     N = y.shape[1]
     e = epi if epi is not None else Epilogue()
-    _ok(fn(_ptr(codes), _ptr(sx), _ptr(w), _ptr(sw), M, N, K, _qcfg(bits, rot_group, scale_group),
+    _ok(fn(_ptr(codes), _ptr(sx), _ptr(w), _ptr(sw), M, N, K, _qcfg(bits, rot_group, scale_group, code_format),
            ctypes.byref(e), _ptr(y), _rowstride(y), _stream(stream)), where)
 
 
 def rbd_w4a4_linear(codes: torch.Tensor, sx: torch.Tensor, w_packed: torch.Tensor, sw: torch.Tensor,
                     y: torch.Tensor, scale_group: int = 0, epi: Optional[Epilogue] = None,
-                    rot_group: int = 256, stream=None) -> None:
-    """y bf16 [M, N] = epilogue(dequant(codes @ unpack(w_packed)^T))."""
+                    rot_group: int = 256, stream=None, code_format: int = CODES_INT8) -> None:
+    """y bf16 [M, N] = epilogue(dequant(codes @ unpack(w_packed)^T)); codes in code_format (E4M3
+    codes take the FP8 tensor-core path, group-64 scales only)."""
     _linear(load().rbd_w4a4_linear, "rbd_w4a4_linear", codes, sx, w_packed, sw, y, 4, rot_group,
-            scale_group, epi, stream)
+            scale_group, epi, stream, code_format)
 
 
 def rbd_w8a8_linear(codes: torch.Tensor, sx: torch.Tensor, w8: torch.Tensor, sw: torch.Tensor,

@@ -26,6 +26,8 @@ rbd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RBD_OK : RBD_E
 
 rbd_status check_qcfg(const rbd_qcfg& c, int64_t K) {
   if (c.bits != 4 && c.bits != 8) return RBD_ERR_INVALID_ARG;
+  if (c.code_format != RBD_CODES_INT8 && c.code_format != RBD_CODES_E4M3) return RBD_ERR_INVALID_ARG;
+  if (c.code_format == RBD_CODES_E4M3 && c.bits != 4) return RBD_ERR_UNSUPPORTED;
   if (c.rot_group != 0 && c.rot_group != 256) return RBD_ERR_UNSUPPORTED;
   if (c.scale_group != 0 && c.scale_group != 64) return RBD_ERR_UNSUPPORTED;
   if (K <= 0 || K % 256 != 0 || K > 16384) return RBD_ERR_UNSUPPORTED;
@@ -135,8 +137,8 @@ rbd_status quant_common(const void* x, int64_t M, int64_t K, int64_t ld, rbd_qcf
   rbd_status s = quant_validate(x, M, K, ld, cfg, out, scales);
   if (s != RBD_OK || M == 0) return s;
   return cuda_status(rbd::launch_rot_quant(static_cast<const uint16_t*>(x), M, K, ld, cfg.bits, cfg.rot_group != 0,
-                                           cfg.scale_group == 64, packed, static_cast<int8_t*>(out), scales,
-                                           as_stream(stream)));
+                                           cfg.scale_group == 64, packed, cfg.code_format == RBD_CODES_E4M3,
+                                           static_cast<int8_t*>(out), scales, as_stream(stream)));
 }
 
 template <bool W4>
@@ -145,6 +147,10 @@ rbd_status linear_common(const int8_t* codes, const float* sx, const void* w, co
                          void* stream) {
   if (cfg.bits != (W4 ? 4 : 8)) return RBD_ERR_INVALID_ARG;
   if (cfg.scale_group != 0 && cfg.scale_group != 64) return RBD_ERR_UNSUPPORTED;
+  if (cfg.code_format != RBD_CODES_INT8 && cfg.code_format != RBD_CODES_E4M3) return RBD_ERR_INVALID_ARG;
+  // E4M3 codes: 4-bit codes with group-64 scales (a float32 partial per 64-wide group is exact)
+  const bool f8 = cfg.code_format == RBD_CODES_E4M3;
+  if (f8 && !(W4 && cfg.scale_group == 64)) return RBD_ERR_UNSUPPORTED;
   if (M < 0 || N <= 0 || K <= 0) return RBD_ERR_INVALID_ARG;
   if (K % 128 != 0 || N % 128 != 0) return RBD_ERR_UNSUPPORTED;
   if (M > (int64_t)INT32_MAX / 2 || N > (1 << 24) || K > (1 << 20)) return RBD_ERR_UNSUPPORTED;
@@ -209,12 +215,12 @@ rbd_status linear_common(const int8_t* codes, const float* sx, const void* w, co
   a.y = static_cast<uint16_t*>(y);
   a.ldy = ldy;
   a.acc_debug = e.acc_debug;
-  a.acc_scale = W4 ? 1.0f / 16.0f : 1.0f;
+  a.acc_scale = (W4 && !f8) ? 1.0f / 16.0f : 1.0f;   // the INT8 path widens a nibble q to the byte 16 q
   a.num_m_tiles = static_cast<int>((M + tt - 1) / tt);
   a.num_tiles = a.num_m_tiles * static_cast<int>(N / 128);
   const int sms = num_sms_current();
   if (sms <= 0) return RBD_ERR_CUDA;
-  return cuda_status(rbd::launch_lowbit_gemm(W4, cfg.scale_group == 64, tm_x, tm_w, tm_ld, tm_l2, tm_y, a, sms,
+  return cuda_status(rbd::launch_lowbit_gemm(W4, cfg.scale_group == 64, f8, tm_x, tm_w, tm_ld, tm_l2, tm_y, a, sms,
                                              as_stream(stream)));
 }
 
@@ -264,7 +270,7 @@ rbd_status rbd_norm_rot_quant_act(const void* x, int64_t M, int64_t K, int64_t l
   if (s != RBD_OK || M == 0) return s;
   return cuda_status(rbd::launch_norm_rot_quant(
       static_cast<const uint16_t*>(x), M, K, ldx, cfg.bits, cfg.rot_group != 0, cfg.scale_group == 64,
-      static_cast<const uint16_t*>(gamma), static_cast<const uint16_t*>(shift),
+      cfg.code_format == RBD_CODES_E4M3, static_cast<const uint16_t*>(gamma), static_cast<const uint16_t*>(shift),
       static_cast<const uint16_t*>(scale), eps, codes, scales, as_stream(stream)));
 }
 
@@ -278,8 +284,9 @@ rbd_status rbd_lowrank_fused(const void* x, int64_t M, int64_t K, int64_t ldx, r
   if (cfg.scale_group == 64) {
     // group scales: one pass over X yields codes, scales and the down product
     return cuda_status(rbd::launch_rot_quant_lowrank(static_cast<const uint16_t*>(x), M, K, ldx, cfg.bits,
-                                                     cfg.rot_group != 0, static_cast<const uint16_t*>(l1t), r,
-                                                     codes, scales, static_cast<uint16_t*>(ld), as_stream(stream)));
+                                                     cfg.rot_group != 0, cfg.code_format == RBD_CODES_E4M3,
+                                                     static_cast<const uint16_t*>(l1t), r, codes, scales,
+                                                     static_cast<uint16_t*>(ld), as_stream(stream)));
   }
   s = quant_common(x, M, K, ldx, cfg, codes, scales, false, stream);
   if (s != RBD_OK) return s;
@@ -350,12 +357,14 @@ rbd_status rbd_rope_tables(const int32_t* pos, int64_t T, double base, float* co
 rbd_status rbd_pack_weights_int4(const void* w, int64_t N, int64_t K, rbd_qcfg cfg, uint8_t* packed, float* scales,
                                  void* stream) {
   if (cfg.bits != 4) return RBD_ERR_INVALID_ARG;
+  if (cfg.code_format != RBD_CODES_INT8) return RBD_ERR_UNSUPPORTED;   // packed nibbles are two's complement
   return quant_common(w, N, K, K, cfg, packed, scales, true, stream);
 }
 
 rbd_status rbd_pack_weights_int8(const void* w, int64_t N, int64_t K, rbd_qcfg cfg, int8_t* w8, float* scales,
                                  void* stream) {
   if (cfg.bits != 8) return RBD_ERR_INVALID_ARG;
+  if (cfg.code_format != RBD_CODES_INT8) return RBD_ERR_UNSUPPORTED;
   return quant_common(w, N, K, K, cfg, w8, scales, false, stream);
 }
 

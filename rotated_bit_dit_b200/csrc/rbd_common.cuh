@@ -190,6 +190,16 @@ __device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem]^T, 8-bit float inputs (kind::f8f6f4, formats
+// given by the instruction descriptor), fp32 accumulation, K = 32 per instruction.
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulation.
 __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
@@ -263,6 +273,11 @@ __host__ __device__ constexpr uint32_t idesc_i8(uint32_t m, uint32_t n, bool a_s
          | ((a_signed ? 1u : 0u) << 7)       // A: s8 / u8
          | ((b_signed ? 1u : 0u) << 10)      // B: s8 / u8
          | ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+// Instruction descriptor of kind::f8f6f4: E4M3 x E4M3 (format 0) -> F32, both
+// K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_e4m3(uint32_t m, uint32_t n) {
+  return (1u << 4) | ((n >> 3) << 17) | ((m >> 4) << 24);
 }
 // Instruction descriptor: BF16 x BF16 -> F32, both K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t m, uint32_t n) {

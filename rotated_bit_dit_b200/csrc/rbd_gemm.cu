@@ -41,6 +41,15 @@
 // so that 12582912*a is exact; the relative change of the scale is below
 // 2^-22).
 //
+// E4M3 path (F8, W4A4 with group-64 scales and E4M3 activation codes).  Every
+// INT4 code in [-8, 7] is an exact E4M3 value, and a 64-wide group partial of
+// such products (|sum| <= 4096) is exact in the float32 accumulator, so the
+// contraction can run as tcgen05.mma kind::f8f6f4 at the INT8 rate and hand
+// the epilogue float32 partials: promotion is then y += (p * a) * b, two
+// float32 operations per element and group, with no int -> float step.  The
+// converter warps widen each packed nibble into its E4M3 byte through a
+// 16-entry byte-permute lookup (three permutes and one select per 4 codes).
+//
 // Warp roles (16 warps, registers redistributed per warpgroup with setmaxnreg):
 //   warpgroup 0: warps 0, 2, 3 TMA producers, warp 1 TMEM allocator + MMA issuer;
 //   warpgroup 1: INT4 -> INT8 converters (W4A4 only);
@@ -81,6 +90,31 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Eight packed two's-complement nibbles (code k in bits 4k..4k+3) -> their eight
+// E4M3 bytes, codes 0-3 in o0 and 4-7 in o1, in order.  Two byte-permute
+// tables give the E4M3 byte of every non-negative nibble value (0..7) and of
+// every negative one (-8..-1) from the nibble's low three bits; a third permute
+// replicates each nibble's sign bit into a byte mask that selects between them.
+constexpr uint32_t kE4Pos0 = 0x44403800u;   // E4M3 of 0, 1, 2, 3
+constexpr uint32_t kE4Pos1 = 0x4E4C4A48u;   // E4M3 of 4, 5, 6, 7
+constexpr uint32_t kE4Neg0 = 0xCACCCED0u;   // E4M3 of -8, -7, -6, -5
+constexpr uint32_t kE4Neg1 = 0xB8C0C4C8u;   // E4M3 of -4, -3, -2, -1
+__device__ __forceinline__ void nibbles_to_e4m3(uint32_t pw, uint32_t& o0, uint32_t& o1) {
+  const uint32_t sel = pw & 0x77777777u;   // low three bits of every nibble
+  const uint32_t sh4 = pw << 4;            // sign bits of the even nibbles at byte msbs
+  const uint32_t selh = sel >> 16;
+  const uint32_t m0 = prmt(sh4, pw, 0xD9C8u);   // 0xFF where codes 0..3 are negative
+  const uint32_t m1 = prmt(sh4, pw, 0xFBEAu);   // likewise codes 4..7
+  o0 = (prmt(kE4Pos0, kE4Pos1, sel) & ~m0) | (prmt(kE4Neg0, kE4Neg1, sel) & m0);
+  o1 = (prmt(kE4Pos0, kE4Pos1, selh) & ~m1) | (prmt(kE4Neg0, kE4Neg1, selh) & m1);
 }
 
 }  // namespace
@@ -159,8 +193,10 @@ __device__ __forceinline__ void tmem_reg_fence32(uint32_t (&v)[32]) {
 }
 
 // y[16 P + j2] += (16*acc*a) * b for the 32 columns of phase P; b4 points at the
-// scales of the phase's first column (broadcast reads).
-template <int P, bool W4, bool DBG>
+// scales of the phase's first column (broadcast reads).  F8: the partials are
+// float32 already and y += (p * a) * b, two paired float32 operations per two
+// columns.
+template <int P, bool W4, bool DBG, bool F8>
 __device__ __forceinline__ void g64_promote_phase(float2 (&y)[32], const uint32_t (&v)[32], const float4* b4,
                                                   float a, float c, int32_t* dbg, int64_t dbg_m0, int64_t M,
                                                   int64_t N) {
@@ -173,11 +209,17 @@ __device__ __forceinline__ void g64_promote_phase(float2 (&y)[32], const uint32_
       const uint32_t u0 = v[j], u1 = v[j + 1];
       if (DBG) {
         const int64_t m = dbg_m0 + 32 * P + j;
-        if (m < M) dbg[m * N] = W4 ? ((int32_t)u0 >> 4) : (int32_t)u0;
-        if (m + 1 < M) dbg[(m + 1) * N] = W4 ? ((int32_t)u1 >> 4) : (int32_t)u1;
+        if (F8) {
+          if (m < M) dbg[m * N] = __float2int_rn(__uint_as_float(u0));
+          if (m + 1 < M) dbg[(m + 1) * N] = __float2int_rn(__uint_as_float(u1));
+        } else {
+          if (m < M) dbg[m * N] = W4 ? ((int32_t)u0 >> 4) : (int32_t)u0;
+          if (m + 1 < M) dbg[(m + 1) * N] = W4 ? ((int32_t)u1 >> 4) : (int32_t)u1;
+        }
       }
-      const float2 t = make_float2(fmaf(__uint_as_float(u0 + kMagicBits), a, c),
-                                   fmaf(__uint_as_float(u1 + kMagicBits), a, c));
+      const float2 t = F8 ? __fmul2_rn(make_float2(__uint_as_float(u0), __uint_as_float(u1)), make_float2(a, a))
+                          : make_float2(fmaf(__uint_as_float(u0 + kMagicBits), a, c),
+                                        fmaf(__uint_as_float(u1 + kMagicBits), a, c));
       const float2 b = hh ? make_float2(bq.z, bq.w) : make_float2(bq.x, bq.y);
       float2& yy = y[16 * P + j / 2];
       yy = __ffma2_rn(t, b, yy);
@@ -203,7 +245,7 @@ __device__ __forceinline__ void g64_add_phase(float2 (&y)[32], const uint32_t (&
 // 2 pb + 1): the two groups of one 128-wide K stage share a pair, the low-rank
 // segment takes a pair of its own.  Returns false if a wait timed out (nothing
 // is stored then).
-template <bool W4, bool LR, bool DBG>
+template <bool W4, bool LR, bool DBG, bool F8>
 __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, uint64_t* pfull, uint64_t* pempty,
                                          int& pb, uint32_t& pbits, const float* sxc, int sx_stride, int m0, int n,
                                          int col0, uint32_t lane, const CUtensorMap* tm_y, uint16_t* sout) {
@@ -250,8 +292,10 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
   for (int g = 0; g < G; ++g) {
     const int odd = g & 1;
     const uint32_t tA = tcol + (2 * pb + odd) * TT;
-    const float a = __uint_as_float((__float_as_uint(swn * args.acc_scale) + 2u) & ~3u);   // 22 significant bits
-    const float c = -kMagicF * a;                                                           // exact
+    // integer partials: weight scale rounded to 22 significant bits so that c is exact;
+    // float32 partials (F8): the weight scale itself
+    const float a = F8 ? swn * args.acc_scale : __uint_as_float((__float_as_uint(swn * args.acc_scale) + 2u) & ~3u);
+    const float c = -kMagicF * a;
     if (g + 1 < G) swn = __ldg(swp + g + 1);
     const float4* b4 = reinterpret_cast<const float4*>(sxc + (int64_t)g * sx_stride);
     int32_t* dg = DBG ? dbg + (int64_t)g * args.M * args.N : nullptr;
@@ -259,7 +303,7 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
     tmem_wait_ld();
     tmem_reg_fence32(vX);
     g64_load_phase<1>(tA, vY);
-    g64_promote_phase<0, W4, DBG>(y, vX, b4, a, c, dg, dbg_m0, args.M, args.N);
+    g64_promote_phase<0, W4, DBG, F8>(y, vX, b4, a, c, dg, dbg_m0, args.M, args.N);
     // phase 1 (columns 32-63) while the next segment's phase 0 is in flight;
     // a pair is free as soon as the last load of its second buffer has landed
     tmem_wait_ld();
@@ -274,7 +318,7 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
         else g64_load_phase<0>(tcol + 2 * pb * TT, vX);
       }
     }
-    g64_promote_phase<1, W4, DBG>(y, vY, b4 + 8, a, c, dg, dbg_m0, args.M, args.N);
+    g64_promote_phase<1, W4, DBG, F8>(y, vY, b4 + 8, a, c, dg, dbg_m0, args.M, args.N);
     if (!ok) return false;
   }
 
@@ -321,7 +365,7 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
   return true;
 }
 
-template <bool W4, bool G64, bool LR, bool DBG>
+template <bool W4, bool G64, bool LR, bool DBG, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w8,
                        const __grid_constant__ CUtensorMap tm_ld, const __grid_constant__ CUtensorMap tm_l2,
@@ -434,7 +478,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // division and dynamic indexing (segment boundaries are compile-time:
       // one per tile with row scales, two per stage with group scales).
       if (elect_one()) {
-        const uint32_t idesc = idesc_i8(kTileF, TT);
+        static_assert(!F8 || (W4 && G64), "the E4M3 path is the W4A4 group-scale path");
+        const uint32_t idesc = F8 ? idesc_e4m3(kTileF, TT) : idesc_i8(kTileF, TT);
         const uint32_t idesc_lr = idesc_bf16(kTileF, TT);
         // descriptor address fields are byte offsets >> 4; stage s adds s * stage bytes >> 4
         const uint64_t bdesc0 = smem_desc_kmajor(smem_u32(smem + L.x_off), 128);
@@ -480,8 +525,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int hg = 0; hg < 2; ++hg) {
                 const uint32_t d = tmem + (2 * pb + hg) * TT;
-                mma_i8_ss(d, adesc + 4 * hg, bdesc + 4 * hg, idesc, 0u);   // overwrite: a new group
-                mma_i8_ss(d, adesc + 4 * hg + 2, bdesc + 4 * hg + 2, idesc, 1u);
+                if constexpr (F8) {
+                  mma_f8_ss(d, adesc + 4 * hg, bdesc + 4 * hg, idesc, 0u);   // overwrite: a new group
+                  mma_f8_ss(d, adesc + 4 * hg + 2, bdesc + 4 * hg + 2, idesc, 1u);
+                } else {
+                  mma_i8_ss(d, adesc + 4 * hg, bdesc + 4 * hg, idesc, 0u);   // overwrite: a new group
+                  mma_i8_ss(d, adesc + 4 * hg + 2, bdesc + 4 * hg + 2, idesc, 1u);
+                }
               }
               tc_commit(&pfull[pb]);
               pb ^= 1;
@@ -551,10 +601,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t o[8];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const uint32_t lo = (pw[j] << 4) & 0xF0F0F0F0u;  // even k, as 16*q
-              const uint32_t hi = pw[j] & 0xF0F0F0F0u;         // odd k, as 16*q
-              o[2 * j] = __byte_perm(lo, hi, 0x5140);
-              o[2 * j + 1] = __byte_perm(lo, hi, 0x7362);
+              if constexpr (F8) {
+                nibbles_to_e4m3(pw[j], o[2 * j], o[2 * j + 1]);   // E4M3 bytes of q
+              } else {
+                const uint32_t lo = (pw[j] << 4) & 0xF0F0F0F0u;  // even k, as 16*q
+                const uint32_t hi = pw[j] & 0xF0F0F0F0u;         // odd k, as 16*q
+                o[2 * j] = __byte_perm(lo, hi, 0x5140);
+                o[2 * j + 1] = __byte_perm(lo, hi, 0x7362);
+              }
             }
             const uint32_t ch0 = (2u * i) ^ (fr & 7u), ch1 = (2u * i + 1u) ^ (fr & 7u);
             *reinterpret_cast<uint4*>(arow + ch0 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -622,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar_epi();
       if constexpr (G64) {
         if (ok)
-          ok = g64_tile<W4, LR, DBG>(args, tmem + lane_base + col0, pfull, pempty, pb, pbits, sx_s + col0,
+          ok = g64_tile<W4, LR, DBG, F8>(args, tmem + lane_base + col0, pfull, pempty, pb, pbits, sx_s + col0,
                                      L.sx_stride, m0, n0 + fr, (int)col0, lane, &tm_y,
                                      reinterpret_cast<uint16_t*>(smem + L.out_off) +
                                          (warp - kWarpEpi0) * (kOutWarpBytes / 2));
@@ -785,7 +839,7 @@ static bool regs_ok(const void* kern) {
   return fa.numRegs == 128;
 }
 
-cudaError_t launch_lowbit_gemm(bool w4, bool g64, const CUtensorMap& tm_x, const CUtensorMap& tm_w8,
+cudaError_t launch_lowbit_gemm(bool w4, bool g64, bool f8, const CUtensorMap& tm_x, const CUtensorMap& tm_w8,
                                const CUtensorMap& tm_ld, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
                                const GemmArgs& a, int num_sms, cudaStream_t st) {
   const bool lr = a.r > 0;
@@ -793,16 +847,21 @@ cudaError_t launch_lowbit_gemm(bool w4, bool g64, const CUtensorMap& tm_x, const
   if (smem > 227u * 1024u) return cudaErrorInvalidConfiguration;
   const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
   const bool dbg = a.acc_debug != nullptr;
-#define RBD_GEMM_CASE(W, G, R, D)                                                                     \
-  if (w4 == W && g64 == G && lr == R && dbg == D) {                                                  \
-    auto kern = lowbit_gemm_kernel<W, G, R, D>;                                                      \
+  if (f8 && !(w4 && g64)) return cudaErrorInvalidValue;
+#define RBD_GEMM_CASE(W, G, R, D, F)                                                                  \
+  if (w4 == W && g64 == G && lr == R && dbg == D && f8 == F) {                                       \
+    auto kern = lowbit_gemm_kernel<W, G, R, D, F>;                                                   \
     if (!regs_ok(reinterpret_cast<const void*>(kern))) return cudaErrorInvalidConfiguration;         \
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);    \
     if (e != cudaSuccess) return e;                                                                  \
     kern<<<grid, kThreads, smem, st>>>(tm_x, tm_w8, tm_ld, tm_l2, tm_y, a);                               \
     return cudaGetLastError();                                                                       \
   }
-#define RBD_GEMM_CASES(W, G, R) RBD_GEMM_CASE(W, G, R, false) RBD_GEMM_CASE(W, G, R, true)
+#define RBD_GEMM_CASES(W, G, R) RBD_GEMM_CASE(W, G, R, false, false) RBD_GEMM_CASE(W, G, R, true, false)
+  RBD_GEMM_CASE(true, true, true, false, true)
+  RBD_GEMM_CASE(true, true, true, true, true)
+  RBD_GEMM_CASE(true, true, false, false, true)
+  RBD_GEMM_CASE(true, true, false, true, true)
   RBD_GEMM_CASES(true, true, true)
   RBD_GEMM_CASES(true, true, false)
   RBD_GEMM_CASES(true, false, true)

@@ -29,20 +29,22 @@ struct GemmArgs {
   int num_m_tiles, num_tiles;
 };
 
+// e4m3: write each (4-bit) code as the E4M3 byte of equal value instead of an int8.
 cudaError_t launch_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot, bool g64,
-                             bool packed, int8_t* codes, float* scales, cudaStream_t st);
+                             bool packed, bool e4m3, int8_t* codes, float* scales, cudaStream_t st);
 // RMSNorm + modulation, then rotate/quantise (activation codes, one byte each).
 cudaError_t launch_norm_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot,
-                                  bool g64, const uint16_t* gamma, const uint16_t* shift, const uint16_t* scale,
-                                  float eps, int8_t* codes, float* scales, cudaStream_t st);
+                                  bool g64, bool e4m3, const uint16_t* gamma, const uint16_t* shift,
+                                  const uint16_t* scale, float eps, int8_t* codes, float* scales, cudaStream_t st);
 // Group-scale prologue and low-rank down product in one pass over X.
 cudaError_t launch_rot_quant_lowrank(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot,
-                                     const uint16_t* l1t, int r, int8_t* codes, float* scales, uint16_t* ld,
-                                     cudaStream_t st);
+                                     bool e4m3, const uint16_t* l1t, int r, int8_t* codes, float* scales,
+                                     uint16_t* ld, cudaStream_t st);
 cudaError_t launch_lowrank_down(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const uint16_t* l1t, int r,
                                 uint16_t* ld, cudaStream_t st);
 // tm_y: unswizzled map of Y with 32-feature x 64-token boxes (group-scale tiles store through it)
-cudaError_t launch_lowbit_gemm(bool w4, bool g64, const CUtensorMap& tm_x, const CUtensorMap& tm_w8,
+// f8: E4M3 activation codes and the kind::f8f6f4 contraction (W4A4 with group scales only).
+cudaError_t launch_lowbit_gemm(bool w4, bool g64, bool f8, const CUtensorMap& tm_x, const CUtensorMap& tm_w8,
                                const CUtensorMap& tm_ld, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
                                const GemmArgs& a, int num_sms, cudaStream_t st);
 

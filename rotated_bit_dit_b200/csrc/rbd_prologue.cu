@@ -14,6 +14,8 @@
 // that it holds positions tau + 16*i (digits j2, j3 in registers), transforms
 // those, and quantises.  Codes go back through shared memory so each thread
 // stores 16 contiguous bytes.
+#include <cuda_fp8.h>
+
 #include "rbd_common.cuh"
 #include "rbd_internal.cuh"
 #include "rbd_rotate.cuh"
@@ -33,6 +35,17 @@ __device__ __forceinline__ int quant1(float v, float inv, float qmax) {
   return q;
 }
 
+// The byte that holds one activation code: the two's-complement int8, or (E4)
+// the E4M3 byte of the same value, exact for every INT4 code.
+template <bool E4>
+__device__ __forceinline__ uint32_t code_byte(int q) {
+  if constexpr (E4) {
+    return static_cast<uint32_t>(__nv_cvt_float_to_fp8(static_cast<float>(q), __NV_SATFINITE, __NV_E4M3));
+  } else {
+    return static_cast<uint32_t>(q) & 0xFFu;
+  }
+}
+
 }  // namespace
 
 // RMSNorm + modulation ahead of the rotation (NORM variant).  gamma, shift and
@@ -47,6 +60,7 @@ struct NormArgs {
 // One CTA handles `rows` rows; each row is handled by T = 16 * teams threads;
 // team `tm` of a row processes 256-blocks g = tm, tm + teams, ... (at most CMAX).
 // OUT_PACKED: write packed INT4 bytes instead of one code per byte.
+// E4: each code byte is the E4M3 byte of the code's value (4-bit codes only).
 // NORM: the row (all of it is in registers) is first normalised and modulated
 // -- "Krea 2 Turbo OrbitQuant W4A4", section "Fused transformer": the norm and
 // the modulation are folded into the kernels that quantise activations.  The sum of the
@@ -55,7 +69,7 @@ struct NormArgs {
 // once to float32; then per element, as single float32 operations,
 // u = x * r, u *= gamma, u *= (1 + scale), u += shift, rounded once to bf16.
 // A row whose mean square plus eps is zero gets r = 0.
-template <bool ROT, bool G64, bool OUT_PACKED, int CMAX, bool NORM = false>
+template <bool ROT, bool G64, bool OUT_PACKED, int CMAX, bool NORM = false, bool E4 = false>
 __global__ void __launch_bounds__(256) rot_quant_kernel(const uint16_t* __restrict__ x, int64_t M, int K,
                                                         int64_t ldx, float qmax, int teams, int rows,
                                                         int8_t* __restrict__ codes, float* __restrict__ scales,
@@ -231,7 +245,7 @@ __global__ void __launch_bounds__(256) rot_quant_kernel(const uint16_t* __restri
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float inv = G64 ? inv_g[c][i >> 2] : inv_row;
-        cb[tau + 16 * i] = static_cast<unsigned char>(static_cast<int8_t>(quant1(xr[c][i], inv, qmax)));
+        cb[tau + 16 * i] = static_cast<unsigned char>(code_byte<E4>(quant1(xr[c][i], inv, qmax)));
       }
       __syncwarp();
       const uint4 q4 = *reinterpret_cast<const uint4*>(cb + 16 * tau);
@@ -245,7 +259,7 @@ __global__ void __launch_bounds__(256) rot_quant_kernel(const uint16_t* __restri
         for (int b = 0; b < 4; ++b) {
           const int i = 4 * wv + b;
           const float inv = G64 ? inv_g[c][tau >> 2] : inv_row;
-          word |= (static_cast<uint32_t>(quant1(xr[c][i], inv, qmax)) & 0xFFu) << (8 * b);
+          word |= code_byte<E4>(quant1(xr[c][i], inv, qmax)) << (8 * b);
         }
         packed_words[wv] = word;
       }
@@ -388,7 +402,7 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <bool ROT, int R>
+template <bool ROT, int R, bool E4 = false>
 __global__ void __launch_bounds__(kLrWarps * 32, R <= 32 ? 3 : 2)
     rot_quant_lowrank_kernel(const uint16_t* __restrict__ x, int64_t M, int K, int64_t ldx, float qmax,
                              const uint16_t* __restrict__ l1t, int8_t* __restrict__ codes,
@@ -461,7 +475,7 @@ __global__ void __launch_bounds__(kLrWarps * 32, R <= 32 ? 3 : 2)
       unsigned char* cb = reinterpret_cast<unsigned char*>(tb);
 #pragma unroll
       for (int i = 0; i < 16; ++i)
-        cb[tau + 16 * i] = static_cast<unsigned char>(static_cast<int8_t>(quant1(xr[i], inv_g[i >> 2], qmax)));
+        cb[tau + 16 * i] = static_cast<unsigned char>(code_byte<E4>(quant1(xr[i], inv_g[i >> 2], qmax)));
       __syncwarp();
       const uint4 q4 = *reinterpret_cast<const uint4*>(cb + 16 * tau);
       __syncwarp();
@@ -472,7 +486,7 @@ __global__ void __launch_bounds__(kLrWarps * 32, R <= 32 ? 3 : 2)
         uint32_t word = 0;
 #pragma unroll
         for (int b = 0; b < 4; ++b)
-          word |= (static_cast<uint32_t>(quant1(xr[4 * wv + b], inv_g[tau >> 2], qmax)) & 0xFFu) << (8 * b);
+          word |= code_byte<E4>(quant1(xr[4 * wv + b], inv_g[tau >> 2], qmax)) << (8 * b);
         w[wv] = word;
       }
     }
@@ -544,14 +558,14 @@ Geometry geometry(int64_t K) {
   return gm;
 }
 
-template <bool ROT, bool G64, bool PK, bool NORM = false>
+template <bool ROT, bool G64, bool PK, bool NORM = false, bool E4 = false>
 cudaError_t launch_rq_c(int cmax, dim3 grid, int threads, size_t smem, cudaStream_t st, const uint16_t* x,
                         int64_t M, int K, int64_t ldx, float qmax, int teams, int rows, int8_t* codes,
                         float* scales, NormArgs norm = NormArgs{}) {
   switch (cmax) {
 #define RBD_RQ_CASE(C)                                                                                    \
   case C: {                                                                                               \
-    auto kern = rot_quant_kernel<ROT, G64, PK, C, NORM>;                                                  \
+    auto kern = rot_quant_kernel<ROT, G64, PK, C, NORM, E4>;                                              \
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
     if (e != cudaSuccess) return e;                                                                       \
     kern<<<grid, threads, smem, st>>>(x, M, K, ldx, qmax, teams, rows, codes, scales, norm);             \
@@ -569,12 +583,24 @@ cudaError_t launch_rq_c(int cmax, dim3 grid, int threads, size_t smem, cudaStrea
 }  // namespace
 
 cudaError_t launch_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot, bool g64,
-                             bool packed, int8_t* codes, float* scales, cudaStream_t st) {
+                             bool packed, bool e4m3, int8_t* codes, float* scales, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   const Geometry gm = geometry(K);
   const float qmax = bits == 4 ? 7.f : 127.f;
   const dim3 grid(static_cast<unsigned>((M + gm.rows - 1) / gm.rows));
   const int Ki = static_cast<int>(K);
+  if (e4m3) {
+    if (packed || bits != 4) return cudaErrorInvalidValue;
+#define RBD_RQ_E4(R_, G_)                                                                                \
+  return launch_rq_c<R_, G_, false, false, true>(gm.cmax, grid, gm.threads, gm.smem, st, x, M, Ki, ldx, qmax, \
+                                                 gm.teams, gm.rows, codes, scales)
+    if (rot) {
+      if (g64) RBD_RQ_E4(true, true); else RBD_RQ_E4(true, false);
+    } else {
+      if (g64) RBD_RQ_E4(false, true); else RBD_RQ_E4(false, false);
+    }
+#undef RBD_RQ_E4
+  }
 #define RBD_RQ_DISPATCH(R_, G_, P_)                                                                      \
   return launch_rq_c<R_, G_, P_>(gm.cmax, grid, gm.threads, gm.smem, st, x, M, Ki, ldx, qmax, gm.teams, \
                                  gm.rows, codes, scales)
@@ -595,17 +621,20 @@ cudaError_t launch_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ld
 }
 
 cudaError_t launch_norm_rot_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot,
-                                  bool g64, const uint16_t* gamma, const uint16_t* shift, const uint16_t* scale,
-                                  float eps, int8_t* codes, float* scales, cudaStream_t st) {
+                                  bool g64, bool e4m3, const uint16_t* gamma, const uint16_t* shift,
+                                  const uint16_t* scale, float eps, int8_t* codes, float* scales, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   const Geometry gm = geometry(K);
   const float qmax = bits == 4 ? 7.f : 127.f;
   const dim3 grid(static_cast<unsigned>((M + gm.rows - 1) / gm.rows));
   const int Ki = static_cast<int>(K);
   const NormArgs norm{gamma, shift, scale, eps};
-#define RBD_NRQ(R_, G_)                                                                                \
-  return launch_rq_c<R_, G_, false, true>(gm.cmax, grid, gm.threads, gm.smem, st, x, M, Ki, ldx, qmax, \
-                                          gm.teams, gm.rows, codes, scales, norm)
+  if (e4m3 && bits != 4) return cudaErrorInvalidValue;
+#define RBD_NRQ(R_, G_)                                                                                      \
+  return e4m3 ? launch_rq_c<R_, G_, false, true, true>(gm.cmax, grid, gm.threads, gm.smem, st, x, M, Ki, ldx,  \
+                                                       qmax, gm.teams, gm.rows, codes, scales, norm)           \
+              : launch_rq_c<R_, G_, false, true, false>(gm.cmax, grid, gm.threads, gm.smem, st, x, M, Ki, ldx, \
+                                                        qmax, gm.teams, gm.rows, codes, scales, norm)
   if (rot) {
     if (g64) RBD_NRQ(true, true); else RBD_NRQ(true, false);
   } else {
@@ -630,15 +659,16 @@ cudaError_t launch_lowrank_down(const uint16_t* x, int64_t M, int64_t K, int64_t
 }
 
 cudaError_t launch_rot_quant_lowrank(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int bits, bool rot,
-                                     const uint16_t* l1t, int r, int8_t* codes, float* scales, uint16_t* ld,
-                                     cudaStream_t st) {
+                                     bool e4m3, const uint16_t* l1t, int r, int8_t* codes, float* scales,
+                                     uint16_t* ld, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   const dim3 grid(static_cast<unsigned>((M + kFuseTok - 1) / kFuseTok));
   const float qmax = bits == 4 ? 7.f : 127.f;
   const int Ki = static_cast<int>(K);
+  if (e4m3 && bits != 4) return cudaErrorInvalidValue;
 #define RBD_RQL_CASE(ROT_, R_)                                                                          \
   {                                                                                                     \
-    auto kern = rot_quant_lowrank_kernel<ROT_, R_>;                                                     \
+    auto kern = e4m3 ? rot_quant_lowrank_kernel<ROT_, R_, true> : rot_quant_lowrank_kernel<ROT_, R_, false>; \
     const size_t smem = fuse_smem_bytes(R_);                                                            \
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
     if (e != cudaSuccess) return e;                                                                     \

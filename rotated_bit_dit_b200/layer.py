@@ -20,12 +20,17 @@ class RotatedLowBitLinear:
     def __init__(self, weight: torch.Tensor, bits: int = 4, scale_group: int = 0, rot_group: int = 256,
                  bias: Optional[torch.Tensor] = None, l1: Optional[torch.Tensor] = None,
                  l2: Optional[torch.Tensor] = None, gate_mode: int = 0, gate_cols=(0, 0),
-                 gate: Optional[torch.Tensor] = None):
-        """weight bf16 [N, K] (CUDA); l1 bf16 [K, r], l2 bf16 [r, N] (the branch adds (x l1) l2)."""
+                 gate: Optional[torch.Tensor] = None, code_format: Optional[int] = None):
+        """weight bf16 [N, K] (CUDA); l1 bf16 [K, r], l2 bf16 [r, N] (the branch adds (x l1) l2).
+        code_format: how the activation codes are stored between the two kernels; by default
+        E4M3 for INT4 with group-64 scales (the FP8 tensor-core GEMM), INT8 otherwise."""
         if weight.dtype != torch.bfloat16 or not weight.is_cuda:
             raise ValueError("weight must be a CUDA bf16 tensor")
         self.N, self.K = weight.shape
         self.bits, self.scale_group, self.rot_group = bits, scale_group, rot_group
+        if code_format is None:
+            code_format = B.CODES_E4M3 if (bits == 4 and scale_group == 64) else B.CODES_INT8
+        self.code_format = code_format
         G = self.K // 64 if scale_group else 1
         dev = weight.device
         self.sw = torch.empty((self.N, G) if scale_group else (self.N,), dtype=torch.float32, device=dev)
@@ -67,16 +72,21 @@ class RotatedLowBitLinear:
 
     def _run(self, x, codes, sx, ld, residual=None, out=None, acc_debug=None) -> torch.Tensor:
         M = x.shape[0]
+        cf = self.code_format
         if self.rank:
-            B.rbd_lowrank_fused(x, codes, sx, self.l1t, ld, self.bits, self.rot_group, self.scale_group)
+            B.rbd_lowrank_fused(x, codes, sx, self.l1t, ld, self.bits, self.rot_group, self.scale_group,
+                                code_format=cf)
         else:
-            B.rbd_rot_quant_act(x, codes, sx, self.bits, self.rot_group, self.scale_group)
+            B.rbd_rot_quant_act(x, codes, sx, self.bits, self.rot_group, self.scale_group, code_format=cf)
         if out is None:
             out = torch.empty((M, self.N), dtype=torch.bfloat16, device=x.device)
         epi = B.make_epilogue(self.bias, ld, self.l2t, self.gate_mode, self.gate_cols, self.gate, residual,
                               acc_debug)
-        fn = B.rbd_w4a4_linear if self.bits == 4 else B.rbd_w8a8_linear
-        fn(codes, sx, self.wq, self.sw, out, self.scale_group, epi, self.rot_group)
+        if self.bits == 4:
+            B.rbd_w4a4_linear(codes, sx, self.wq, self.sw, out, self.scale_group, epi, self.rot_group,
+                              code_format=cf)
+        else:
+            B.rbd_w8a8_linear(codes, sx, self.wq, self.sw, out, self.scale_group, epi, self.rot_group)
         return out
 
     def forward_host(self, xh: torch.Tensor, yh: torch.Tensor, residual_h: Optional[torch.Tensor] = None,

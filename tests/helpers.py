@@ -38,3 +38,10 @@ def check_output(gpu_bits: np.ndarray, ref64: np.ndarray, ref_bf16: np.ndarray, 
     assert rel <= rel_tol, f"rel-L2 vs bf16 reference {rel:.3e} > {rel_tol}"
     assert worst <= 1.0, f"max |err|/bound {worst:.3f} (max err {err.max():.3e})"
     return dict(rel_bf16=rel, rel64=rel64, max_err=float(err.max(initial=0.0)), worst=worst)
+
+
+def e4m3_bytes(codes: np.ndarray) -> np.ndarray:
+    """The E4M3 bytes of integer codes, by torch's float8_e4m3fn conversion (exact for |code| <= 16):
+    what the quantisers write with the E4M3 code format."""
+    t = torch.from_numpy(np.asarray(codes, np.float32)).to(torch.float8_e4m3fn)
+    return t.view(torch.uint8).numpy()

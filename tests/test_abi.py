@@ -38,8 +38,27 @@ FAKE = ctypes.c_void_p(0x10000)          # 16-byte aligned, never dereferenced
 FAKE_MIS = ctypes.c_void_p(0x10001)      # misaligned
 
 
-def q(bits=4, rot=256, sg=0):
-    return B.QCfg(bits, rot, sg)
+def q(bits=4, rot=256, sg=0, cf=0):
+    return B.QCfg(bits, rot, sg, cf)
+
+
+def test_code_format_validation_without_gpu():
+    lib = R.load()
+    e4 = B.CODES_E4M3
+    # an unknown format; E4M3 with 8-bit codes
+    assert lib.rbd_rot_quant_act(FAKE, 4, 256, 256, q(cf=2), FAKE, FAKE, None) == 1
+    assert lib.rbd_rot_quant_act(FAKE, 4, 256, 256, q(bits=8, cf=e4), FAKE, FAKE, None) == 2
+    assert lib.rbd_lowrank_fused(FAKE, 4, 256, 256, q(bits=8, sg=64, cf=e4), FAKE, FAKE, FAKE, 32, FAKE, None) == 2
+    # weight packers store two's-complement codes only
+    assert lib.rbd_pack_weights_int4(FAKE, 4, 256, q(cf=e4), FAKE, FAKE, None) == 2
+    assert lib.rbd_pack_weights_int8(FAKE, 4, 256, q(bits=8, cf=e4), FAKE, FAKE, None) == 2
+    # the E4M3 linear is the W4A4 group-scale path
+    assert _lin(lib.rbd_w4a4_linear, cfg=q(sg=0, cf=e4)) == 2
+    assert _lin(lib.rbd_w8a8_linear, cfg=q(bits=8, sg=64, cf=e4)) == 2
+    assert _lin(lib.rbd_w4a4_linear, cfg=q(sg=64, cf=3)) == 1
+    assert _lin(lib.rbd_w4a4_linear, M=0, cfg=q(sg=64, cf=e4)) == 0
+    # the struct is four int32 fields, as the header declares
+    assert ctypes.sizeof(B.QCfg) == 16
 
 
 @pytest.mark.parametrize("args,expect", [

@@ -14,10 +14,10 @@ from tests.helpers import check_output, dev_bf16, host_u16
 pytestmark = pytest.mark.gpu
 
 
-def build_case(M, N, K, bits, sg, seed=0, rank=0, bias=False, gate_mode=0, gate_cols=(0, 0)):
+def build_case(M, N, K, bits, sg, seed=0, rank=0, bias=False, gate_mode=0, gate_cols=(0, 0), cf=None):
     xb = I.gaussian_bf16(seed + 1, (M, K), 1.0, 0.01, 20.0)
     wb = I.gaussian_bf16(seed + 2, (N, K), 0.02)
-    case = dict(M=M, N=N, K=K, bits=bits, sg=sg, x=xb, w=wb, gate_mode=gate_mode, gate_cols=gate_cols)
+    case = dict(M=M, N=N, K=K, bits=bits, sg=sg, x=xb, w=wb, gate_mode=gate_mode, gate_cols=gate_cols, cf=cf)
     case["bias"] = I.gaussian_bf16(seed + 3, (N,), 0.1) if bias else None
     case["l1"] = I.gaussian_bf16(seed + 4, (K, rank), 0.01) if rank else None
     case["l2"] = I.gaussian_bf16(seed + 5, (rank, N), 0.01) if rank else None
@@ -34,7 +34,7 @@ def run_layer(case, acc_debug=False):
     dv = lambda a: None if a is None else dev_bf16(a)
     layer = R.RotatedLowBitLinear(dv(case["w"]), bits=bits, scale_group=sg, bias=dv(case["bias"]),
                                   l1=dv(case["l1"]), l2=dv(case["l2"]), gate_mode=case["gate_mode"],
-                                  gate_cols=case["gate_cols"], gate=dv(case["gate"]))
+                                  gate_cols=case["gate_cols"], gate=dv(case["gate"]), code_format=case.get("cf"))
     acc = None
     if acc_debug:
         shape = (K // 64, M, N) if sg else (M, N)
@@ -70,11 +70,15 @@ VARIANTS = {
 }
 
 
+# (bits, scale group, activation code format): INT4 with group scales runs both the FP8 (E4M3 codes,
+# the layer's default) and the INT8 tensor-core paths
+PATHS = [(4, 0, None), (4, 64, None), (4, 64, 0), (8, 0, None), (8, 64, None)]
+
+
 @pytest.mark.parametrize("variant", list(VARIANTS))
-@pytest.mark.parametrize("bits", [4, 8])
-@pytest.mark.parametrize("sg", [0, 64])
-def test_tiny_layer_variants(variant, bits, sg):
-    case = build_case(64, 256, 256, bits, sg, seed=10, **VARIANTS[variant])
+@pytest.mark.parametrize("bits,sg,cf", PATHS)
+def test_tiny_layer_variants(variant, bits, sg, cf):
+    case = build_case(64, 256, 256, bits, sg, seed=10, cf=cf, **VARIANTS[variant])
     y, acc, _ = run_layer(case, acc_debug=True)
     ref = reference(case)
     assert np.array_equal(acc.astype(np.int64), exact_acc(case, ref))
@@ -82,10 +86,10 @@ def test_tiny_layer_variants(variant, bits, sg):
 
 
 @pytest.mark.parametrize("M", [1, 7, 128, 200, 333])
-@pytest.mark.parametrize("bits,sg", [(4, 0), (4, 64), (8, 0), (8, 64)])
-def test_ragged_tokens_several_tiles(M, bits, sg):
+@pytest.mark.parametrize("bits,sg,cf", PATHS)
+def test_ragged_tokens_several_tiles(M, bits, sg, cf):
     # N spans 3 feature tiles, K spans 6 stages (wraps the 4-deep ring), M ends ragged
-    case = build_case(M, 384, 768, bits, sg, seed=20 + M, bias=True, rank=16)
+    case = build_case(M, 384, 768, bits, sg, seed=20 + M, bias=True, rank=16, cf=cf)
     y, acc, _ = run_layer(case, acc_debug=True)
     ref = reference(case)
     assert np.array_equal(acc.astype(np.int64), exact_acc(case, ref))
@@ -102,16 +106,17 @@ def test_long_k_group_scales_two_stage_pipeline(bits, rank):
     check_output(y, ref["ref64"], ref["ref_bf16"])
 
 
-@pytest.mark.parametrize("M,N,K,bits,sg,rank", [
-    (2048, 2560, 512, 4, 64, 32),     # group scales: 320 tiles of 128 x 128 over 148 CTAs
-    (4096, 2048, 1024, 8, 0, 0),      # row scales: 256 tiles of 128 x 256
-    (4096, 2048, 512, 4, 0, 16),      # INT4 row scales, 256 tiles
-    (1500, 2304, 256, 8, 64, 0),      # INT8 group scales, 216 tiles, ragged last token tile
+@pytest.mark.parametrize("M,N,K,bits,sg,rank,cf", [
+    (2048, 2560, 512, 4, 64, 32, None),   # group scales, FP8 path: 320 tiles of 128 x 128 over 148 CTAs
+    (2048, 2560, 512, 4, 64, 32, 0),      # the same on the INT8 path
+    (4096, 2048, 1024, 8, 0, 0, None),    # row scales: 256 tiles of 128 x 256
+    (4096, 2048, 512, 4, 0, 16, None),    # INT4 row scales, 256 tiles
+    (1500, 2304, 256, 8, 64, 0, None),    # INT8 group scales, 216 tiles, ragged last token tile
 ])
-def test_persistent_grid_exact_accumulators(M, N, K, bits, sg, rank):
+def test_persistent_grid_exact_accumulators(M, N, K, bits, sg, rank, cf):
     # more tiles than CTAs: every CTA walks several tiles, so the accumulator buffers' phases wrap
     # across tiles and the per-tile scale tables are restaged; every int32 accumulator is checked
-    case = build_case(M, N, K, bits, sg, seed=80 + M % 97, rank=rank, bias=True)
+    case = build_case(M, N, K, bits, sg, seed=80 + M % 97, rank=rank, bias=True, cf=cf)
     y, acc, _ = run_layer(case, acc_debug=True)
     ref = reference(case)
     assert np.array_equal(acc.astype(np.int64), exact_acc(case, ref))

@@ -9,7 +9,7 @@ import torch
 import rotated_bit_dit_b200 as R
 from oracle import rbd_oracle as O
 from rotated_bit_dit_b200 import inputs as I
-from tests.helpers import dev_bf16
+from tests.helpers import dev_bf16, e4m3_bytes
 
 pytestmark = pytest.mark.gpu
 
@@ -86,3 +86,20 @@ def test_norm_full_layer_input():
     xb = I.gaussian_bf16(I.SEED_X, (cfg["M"], cfg["K"]), 1.0, 0.005, 30.0, outlier_seed=0)
     g, sh, sc = vectors(cfg["K"], 45)
     check(xb, g, sh, sc, 1e-6, 4, 256, 64)
+
+
+@pytest.mark.parametrize("sg", [0, 64])
+def test_norm_rot_quant_e4m3_codes(sg):
+    # the normalising prologue writing E4M3 code bytes: the same codes as the oracle, as E4M3 values
+    M, K = 29, 3072
+    xb = I.gaussian_bf16(700, (M, K), 1.0, 0.005, 30.0)
+    g, sh, sc = vectors(K, 701)
+    dv = lambda v: None if v is None else dev_bf16(v)
+    codes = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((M, K // 64) if sg else (M,), dtype=torch.float32, device="cuda")
+    R.rbd_norm_rot_quant_act(dev_bf16(xb), codes, scales, dv(g), dv(sh), dv(sc), 1e-6, 4, 256, sg,
+                             code_format=R.CODES_E4M3)
+    assert R.rbd_check() == 0
+    ref_q, ref_s = O.norm_rot_quant(xb, 4, 256, sg, g, sh, sc, 1e-6)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ref_s.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), e4m3_bytes(ref_q))

@@ -8,7 +8,7 @@ import torch
 import rotated_bit_dit_b200 as R
 from oracle import rbd_oracle as O
 from rotated_bit_dit_b200 import inputs as I
-from tests.helpers import dev_bf16
+from tests.helpers import dev_bf16, e4m3_bytes
 
 pytestmark = pytest.mark.gpu
 
@@ -33,6 +33,22 @@ def test_rot_quant_bit_exact(M, K, bits, rot, sg):
     ref_q, ref_s = O.rot_quant(xb, bits, rot, sg)
     assert np.array_equal(scales.view(np.uint32), ref_s.view(np.uint32))
     assert np.array_equal(codes, ref_q)
+
+
+@pytest.mark.parametrize("M,K", [(64, 256), (37, 768), (5, 3072), (2, 16384)])
+@pytest.mark.parametrize("rot", [256, 0])
+@pytest.mark.parametrize("sg", [0, 64])
+def test_rot_quant_e4m3_codes_bit_exact(M, K, rot, sg):
+    # the E4M3 code format holds the same INT4 codes, each as the E4M3 byte of its value
+    xb = I.gaussian_bf16(150 + K + M, (M, K), 1.0, 0.005, 30.0)
+    x = dev_bf16(xb)
+    codes = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((M, K // 64) if sg else (M,), dtype=torch.float32, device="cuda")
+    R.rbd_rot_quant_act(x, codes, scales, 4, rot, sg, code_format=R.CODES_E4M3)
+    assert R.rbd_check() == 0
+    ref_q, ref_s = O.rot_quant(xb, 4, rot, sg)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ref_s.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), e4m3_bytes(ref_q))
 
 
 def test_rot_quant_degenerate_rows():
@@ -138,6 +154,25 @@ def test_lowrank_fused_shapes(M, K, bits, rot, r):
     assert R.rbd_check() == 0
     ref_q, ref_s = O.rot_quant(xb, bits, rot, 64)
     assert np.array_equal(codes.cpu().numpy(), ref_q)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ref_s.view(np.uint32))
+    ref_ld = O.lowrank_down(xb, l1b)
+    err = np.abs(ld.float().cpu().numpy().astype(np.float64) - ref_ld)
+    assert np.all(err <= np.abs(ref_ld) * 2.0 ** -8 + 1e-4 * np.abs(ref_ld).max())
+
+
+@pytest.mark.parametrize("M,K,rot,r", [(3, 256, 256, 32), (200, 3072, 256, 32), (33, 12288, 0, 64)])
+def test_lowrank_fused_e4m3_codes(M, K, rot, r):
+    # the single-pass group-scale prologue writing E4M3 code bytes (the layout the FP8 GEMM reads)
+    xb = I.gaussian_bf16(26 + M + K, (M, K), 1.0, 0.005, 30.0)
+    l1b = I.gaussian_bf16(27 + r, (K, r), 0.01)
+    x, l1t = dev_bf16(xb), dev_bf16(np.ascontiguousarray(l1b.T))
+    codes = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((M, K // 64), dtype=torch.float32, device="cuda")
+    ld = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    R.rbd_lowrank_fused(x, codes, scales, l1t, ld, 4, rot, 64, code_format=R.CODES_E4M3)
+    assert R.rbd_check() == 0
+    ref_q, ref_s = O.rot_quant(xb, 4, rot, 64)
+    assert np.array_equal(codes.cpu().numpy(), e4m3_bytes(ref_q))
     assert np.array_equal(scales.cpu().numpy().view(np.uint32), ref_s.view(np.uint32))
     ref_ld = O.lowrank_down(xb, l1b)
     err = np.abs(ld.float().cpu().numpy().astype(np.float64) - ref_ld)
