@@ -120,16 +120,24 @@ __device__ __forceinline__ void nibbles_to_e4m3(uint32_t pw, uint32_t& o0, uint3
 }  // namespace
 
 struct SmemLayout {
-  uint32_t x_off, w_off, ld_off, l2_off, sx_off, out_off, bar_off, total, x_stage;
+  uint32_t x_off, w_off, ld_off, l2_off, sx_off, sw_off, out_off, bar_off, total, x_stage;
   int stages, sx_stride;
+  bool sw_table;   // group mode: the tile's weight scales are staged in shared memory
 };
+
+// Group-scale tiles keep the tile's weight scales in shared memory too, one row
+// of 128 features per group; the odd row stride keeps both the staging writes
+// (lanes along groups) and the epilogue's reads (lanes along features) free of
+// bank conflicts.
+constexpr int kSwStride = kTileF + 1;
 
 // Group-scale tiles stage their bf16 output per epilogue warp (32 features x 64
 // tokens, row-major by token) for one bulk tensor store.
 constexpr uint32_t kOutWarpBytes = 32 * 64 * 2;
 
-__host__ __device__ inline SmemLayout smem_layout(int stages, int r, int G, int tt) {
+__host__ __device__ inline SmemLayout smem_layout(int stages, int r, int G, int tt, bool sw_table) {
   SmemLayout L{};
+  L.sw_table = sw_table && tt == tile_tokens(true);
   uint32_t off = 0;
   L.stages = stages;
   L.x_stage = (uint32_t)tt * kBK;
@@ -148,6 +156,9 @@ __host__ __device__ inline SmemLayout smem_layout(int stages, int r, int G, int 
   L.sx_off = off;
   off += (uint32_t)G * L.sx_stride * 4;
   off = (off + 127u) & ~127u;
+  L.sw_off = off;
+  if (L.sw_table) off += (uint32_t)G * kSwStride * 4;
+  off = (off + 127u) & ~127u;
   L.out_off = off;
   if (tt == tile_tokens(true)) off += 8 * kOutWarpBytes;
   off = (off + 15u) & ~15u;
@@ -157,11 +168,16 @@ __host__ __device__ inline SmemLayout smem_layout(int stages, int r, int G, int 
   return L;
 }
 
-// Number of pipeline stages that fit (up to 4, at least 2); 0 if none.
-__host__ __device__ inline int pick_stages(int r, int G, int tt) {
-  for (int s = kMaxStages; s >= 2; --s)
-    if (smem_layout(s, r, G, tt).total <= 227u * 1024u) return s;
-  return 0;
+// The layout with the most pipeline stages (up to 4, at least 2) that fits,
+// with the weight-scale table when it fits; stages == 0 if nothing fits.
+__host__ __device__ inline SmemLayout pick_layout(int r, int G, int tt) {
+  for (int t = 1; t >= 0; --t)
+    for (int s = kMaxStages; s >= 2; --s) {
+      const SmemLayout L = smem_layout(s, r, G, tt, t != 0);
+      if (L.total <= 227u * 1024u) return L;
+    }
+  SmemLayout none{};
+  return none;
 }
 
 // ---------------------------------------------------------------------------
@@ -247,8 +263,9 @@ __device__ __forceinline__ void g64_add_phase(float2 (&y)[32], const uint32_t (&
 // is stored then).
 template <bool W4, bool LR, bool DBG, bool F8>
 __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, uint64_t* pfull, uint64_t* pempty,
-                                         int& pb, uint32_t& pbits, const float* sxc, int sx_stride, int m0, int n,
-                                         int col0, uint32_t lane, const CUtensorMap* tm_y, uint16_t* sout) {
+                                         int& pb, uint32_t& pbits, const float* sxc, int sx_stride,
+                                         const float* sws, int m0, int n, int col0, uint32_t lane,
+                                         const CUtensorMap* tm_y, uint16_t* sout) {
   constexpr int TT = 128;
   const int G = args.G;
   auto release = [&](int b) {
@@ -280,9 +297,10 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
     pb ^= 1;
   }
 
-  // weight scale of this thread's feature, one segment ahead
+  // weight scale of this thread's feature, one segment ahead: from the tile's
+  // table in shared memory, or (when the table did not fit) from global memory
   const float* swp = args.sw + (int64_t)n * G;
-  float swn = __ldg(swp);
+  float swn = sws ? sws[0] : __ldg(swp);
   const int64_t dbg_m0 = (int64_t)m0 + col0;
   int32_t* dbg = DBG ? args.acc_debug + n : nullptr;
   uint32_t vX[32], vY[32];
@@ -296,7 +314,7 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
     // float32 partials (F8): the weight scale itself
     const float a = F8 ? swn * args.acc_scale : __uint_as_float((__float_as_uint(swn * args.acc_scale) + 2u) & ~3u);
     const float c = -kMagicF * a;
-    if (g + 1 < G) swn = __ldg(swp + g + 1);
+    if (g + 1 < G) swn = sws ? sws[(g + 1) * kSwStride] : __ldg(swp + g + 1);
     const float4* b4 = reinterpret_cast<const float4*>(sxc + (int64_t)g * sx_stride);
     int32_t* dg = DBG ? dbg + (int64_t)g * args.M * args.N : nullptr;
     // phase 0 (columns 0-31) while phase 1 is in flight
@@ -350,10 +368,15 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
     if (lane == 0) bulk_wait_read_all();
     __syncwarp();
 #pragma unroll
-    for (int j = 0; j < kG64Half; ++j) {
-      float o = (j & 1) ? y[j >> 1].y : y[j >> 1].x;
-      if (sig) o = __frcp_rn(1.0f + __expf(-o));
-      sout[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+    for (int j2 = 0; j2 < kG64Half / 2; ++j2) {
+      float o0 = y[j2].x, o1 = y[j2].y;
+      if (sig) {
+        o0 = __frcp_rn(1.0f + __expf(-o0));
+        o1 = __frcp_rn(1.0f + __expf(-o1));
+      }
+      const __nv_bfloat162 ob = __floats2bfloat162_rn(o0, o1);   // one conversion per pair
+      sout[(2 * j2) * 32 + lane] = __bfloat16_as_ushort(ob.x);
+      sout[(2 * j2 + 1) * 32 + lane] = __bfloat16_as_ushort(ob.y);
     }
     fence_async_smem();
     __syncwarp();
@@ -377,8 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ unsigned char smem_dyn[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023u) & ~uintptr_t(1023u));
-  const int S = pick_stages(LR ? args.r : 0, args.G, TT);
-  const SmemLayout L = smem_layout(S, LR ? args.r : 0, args.G, TT);
+  const SmemLayout L = pick_layout(LR ? args.r : 0, args.G, TT);
+  const int S = L.stages;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* full = bars;                    // [kMaxStages]
   uint64_t* empty = bars + kMaxStages;      // [kMaxStages]
@@ -672,12 +695,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < kTokPerWarp; ++i) sx_s[g * L.sx_stride + ew + 8 * i] = v[i];
           }
         }
+        if (G64 && L.sw_table) {
+          // the tile's weight scales: warp w stages features w + 8 i, lane l groups g0 + l
+          float* sw_s = reinterpret_cast<float*>(smem + L.sw_off);
+          for (int g0 = 0; g0 < G; g0 += 32) {
+            const int g = g0 + (int)lane;
+            float v[kTileF / 8];
+#pragma unroll
+            for (int i = 0; i < kTileF / 8; ++i)
+              v[i] = g < G ? __ldg(args.sw + (int64_t)(n0 + ew + 8 * i) * G + g) : 0.f;
+            if (g < G) {
+#pragma unroll
+              for (int i = 0; i < kTileF / 8; ++i) sw_s[g * kSwStride + ew + 8 * i] = v[i];
+            }
+          }
+        }
       }
       named_bar_epi();
       if constexpr (G64) {
         if (ok)
           ok = g64_tile<W4, LR, DBG, F8>(args, tmem + lane_base + col0, pfull, pempty, pb, pbits, sx_s + col0,
-                                     L.sx_stride, m0, n0 + fr, (int)col0, lane, &tm_y,
+                                     L.sx_stride,
+                                     L.sw_table ? reinterpret_cast<const float*>(smem + L.sw_off) + fr : nullptr, m0,
+                                     n0 + fr, (int)col0, lane, &tm_y,
                                      reinterpret_cast<uint16_t*>(smem + L.out_off) +
                                          (warp - kWarpEpi0) * (kOutWarpBytes / 2));
         continue;
@@ -823,9 +863,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Host launcher
 // ---------------------------------------------------------------------------
 uint32_t gemm_smem_bytes(bool g64, int r, int G) {
-  const int tt = tile_tokens(g64);
-  const int s = pick_stages(r, G, tt);
-  return s ? smem_layout(s, r, G, tt).total : 0xFFFFFFFFu;
+  const SmemLayout L = pick_layout(r, G, tile_tokens(g64));
+  return L.stages ? L.total : 0xFFFFFFFFu;
 }
 
 int gemm_tile_tokens(bool g64) { return tile_tokens(g64); }
