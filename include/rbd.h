@@ -344,6 +344,47 @@ rbd_status rbd_qk_norm_rope(const void* x, int64_t T, int64_t H, int64_t ldx, co
 rbd_status rbd_rope_tables(const int32_t* pos, int64_t T, double base, float* cos_t, float* sin_t,
                            void* stream);
 
+/* ---- INT8 attention (SageAttention v1 scheme) ------------------------------
+ * "Krea 2 Turbo OrbitQuant W4A4", "Fused transformer": attention takes Q.K^T in
+ * INT8 and P.V in FP16.  Two calls: rbd_attn_quant prepares the operands,
+ * rbd_attn_int8 runs the attention.  Heads are 128 channels wide.
+ *
+ * Bytes of device scratch rbd_attn_quant needs for Tk keys and H heads (the
+ * float64 partial column sums of K and the key mean); -1 for bad sizes.     */
+int64_t rbd_attn_workspace_bytes(int64_t Tk, int64_t H);
+
+/* Operand preparation.
+ *   q bf16 [Tq, ldq], k bf16 [Tk, ldk], v bf16 [Tk, ldv]: head h at columns
+ *     h*128 .. h*128+127 (the layout of the Q|K|V|gate GEMM output after
+ *     rbd_qk_norm_rope); ld* >= H*128, ld* % 8 == 0, 16-byte aligned.
+ *   Keys are smoothed: per head and channel the mean over the Tk tokens is
+ *   taken in float64 (exact sum while a column spans <= 31 binades) and
+ *   subtracted in float64, the result rounded once to float32.  Q and the
+ *   smoothed K are quantised per (token, head) over the 128 channels:
+ *   amax, s = amax/127, inv = 127/amax (IEEE float32 divisions),
+ *   code = clamp(rint_even(x * inv), -128, 127); an all-zero head gets s = 0.
+ *   qc int8 [H, Tq, 128], sq float32 [H, Tq];
+ *   kc int8 [H, Tk, 128], sk float32 [H, tkp] (entries Tk.. unused);
+ *   vt fp16 [H, 128, tkp]: V transposed per head, each value rounded to fp16
+ *     (nearest even), tokens Tk .. tkp-1 written as zeros;
+ *   tkp >= Tk, tkp % 8 == 0 (the row pitch of sk and vt);
+ *   work: rbd_attn_workspace_bytes(Tk, H) bytes of device scratch, 16-byte
+ *     aligned, overwritten (calls sharing it must not overlap).
+ *   Tk == 0 with Tq > 0 is invalid (RBD_ERR_INVALID_ARG); Tq == Tk == 0 is a
+ *   no-op.  All outputs 16-byte aligned (sq 4-byte).                         */
+rbd_status rbd_attn_quant(const void* q, int64_t ldq, const void* k, int64_t ldk, const void* v, int64_t ldv,
+                          int64_t Tq, int64_t Tk, int64_t H, int8_t* qc, float* sq, int8_t* kc, float* sk,
+                          void* vt, int64_t tkp, void* work, void* stream);
+
+/* Attention on the prepared operands: for every head and query,
+ *   S[key] = (qc . kc[key]) * sq * sk[key] / sqrt(128)  (exact int32 dot product),
+ *   P = softmax over the Tk keys, o = P . V with P rounded to fp16 after the
+ *   running row maximum is subtracted and V in fp16, float32 accumulation.
+ * o bf16 [Tq, ldo], head h at columns h*128; ldo >= H*128, ldo % 8 == 0.
+ * Arguments otherwise as rbd_attn_quant produced them (same Tq, Tk, H, tkp).  */
+rbd_status rbd_attn_int8(const int8_t* qc, const float* sq, const int8_t* kc, const float* sk, const void* vt,
+                         int64_t Tq, int64_t Tk, int64_t H, int64_t tkp, void* o, int64_t ldo, void* stream);
+
 /* Synchronises `stream`, then reports the first device-side error recorded
  * since the last rbd_check (RBD_ERR_DEVICE_TIMEOUT) or a CUDA error, and
  * clears the device status word.                                              */

@@ -34,6 +34,10 @@ from ._binding import (  # noqa: F401
     rbd_kv4_decode,
     rbd_qk_norm_rope,
     rbd_rope_tables,
+    rbd_attn_workspace_bytes,
+    rbd_attn_quant,
+    rbd_attn_int8,
 )
+from .attention import attention_operands, int8_attention  # noqa: F401
 from .kvcache import Int4KVCache  # noqa: F401
 from .layer import RotatedLowBitLinear  # noqa: F401

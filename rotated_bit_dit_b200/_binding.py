@@ -21,7 +21,8 @@ STATUS_NAMES = {0: "RBD_OK", 1: "RBD_ERR_INVALID_ARG", 2: "RBD_ERR_UNSUPPORTED",
 
 EXPORTED = ("rbd_rot_quant_act", "rbd_norm_rot_quant_act", "rbd_lowrank_fused", "rbd_lowrank_down", "rbd_pack_weights_int4", "rbd_pack_weights_int8",
             "rbd_w4a4_linear", "rbd_w8a8_linear", "rbd_nvfp4_scale_bytes", "rbd_nvfp4_quant",
-            "rbd_nvfp4_quant_noalloc", "rbd_nvfp4_linear", "rbd_kv4_encode", "rbd_kv4_decode", "rbd_qk_norm_rope", "rbd_rope_tables", "rbd_check", "rbd_debug_timeout_probe", "rbd_status_string", "rbd_version")
+            "rbd_nvfp4_quant_noalloc", "rbd_nvfp4_linear", "rbd_kv4_encode", "rbd_kv4_decode", "rbd_qk_norm_rope", "rbd_rope_tables", "rbd_attn_workspace_bytes", "rbd_attn_quant", "rbd_attn_int8",
+            "rbd_check", "rbd_debug_timeout_probe", "rbd_status_string", "rbd_version")
 
 
 class RbdError(RuntimeError):
@@ -81,6 +82,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "rbd_kv4_decode": [vp, vp, i64, i64, i64, i64, i32, vp, i64, vp],
         "rbd_qk_norm_rope": [vp, i64, i64, i64, vp, vp, vp, ctypes.c_float, vp, i64, vp],
         "rbd_rope_tables": [vp, i64, ctypes.c_double, vp, vp, vp],
+        "rbd_attn_quant": [vp, i64, vp, i64, vp, i64, i64, i64, i64, vp, vp, vp, vp, vp, i64, vp, vp],
+        "rbd_attn_int8": [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i64, vp],
         "rbd_check": [vp],
         "rbd_debug_timeout_probe": [i64, vp],
     }
@@ -90,6 +93,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         f.restype = ctypes.c_int
     lib.rbd_nvfp4_scale_bytes.argtypes = [i64, i64]
     lib.rbd_nvfp4_scale_bytes.restype = i64
+    lib.rbd_attn_workspace_bytes.argtypes = [i64, i64]
+    lib.rbd_attn_workspace_bytes.restype = i64
     lib.rbd_status_string.argtypes = [ctypes.c_int]
     lib.rbd_status_string.restype = ctypes.c_char_p
     lib.rbd_version.argtypes = []
@@ -331,3 +336,31 @@ def rbd_rope_tables(pos: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor, bas
     if cos.shape != (T, 64) or sin.shape != (T, 64) or not (cos.is_contiguous() and sin.is_contiguous()):
         raise ValueError("cos and sin must be contiguous [T, 64]")
     _ok(load().rbd_rope_tables(_ptr(pos), T, base, _ptr(cos), _ptr(sin), _stream(stream)), "rbd_rope_tables")
+
+
+def rbd_attn_workspace_bytes(Tk: int, H: int) -> int:
+    """Bytes of device scratch rbd_attn_quant needs for Tk keys and H heads."""
+    return int(load().rbd_attn_workspace_bytes(Tk, H))
+
+
+def rbd_attn_quant(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, H: int, qc: torch.Tensor, sq: torch.Tensor,
+                   kc: torch.Tensor, sk: torch.Tensor, vt: torch.Tensor, work: torch.Tensor, stream=None) -> None:
+    """q bf16 [Tq, >=H*128], k / v bf16 [Tk, >=H*128] -> qc int8 [H, Tq, 128], sq float32 [H, Tq],
+    kc int8 [H, Tk, 128], sk float32 [H, tkp], vt fp16 [H, 128, tkp] (tkp = sk.shape[1]);
+    work: rbd_attn_workspace_bytes(Tk, H) bytes of device scratch."""
+    Tq, Tk = q.shape[0], k.shape[0]
+    tkp = sk.shape[1]
+    if vt.shape[-1] != tkp:
+        raise ValueError("sk and vt must share the padded key count")
+    _ok(load().rbd_attn_quant(_ptr(q), _rowstride(q), _ptr(k), _rowstride(k), _ptr(v), _rowstride(v), Tq, Tk, H,
+                              _ptr(qc), _ptr(sq), _ptr(kc), _ptr(sk), _ptr(vt), tkp, _ptr(work), _stream(stream)),
+        "rbd_attn_quant")
+
+
+def rbd_attn_int8(qc: torch.Tensor, sq: torch.Tensor, kc: torch.Tensor, sk: torch.Tensor, vt: torch.Tensor,
+                  o: torch.Tensor, stream=None) -> None:
+    """Attention on rbd_attn_quant's operands -> o bf16 [Tq, >=H*128]."""
+    H, Tq = sq.shape
+    Tk = kc.shape[1]
+    _ok(load().rbd_attn_int8(_ptr(qc), _ptr(sq), _ptr(kc), _ptr(sk), _ptr(vt), Tq, Tk, H, sk.shape[1], _ptr(o),
+                             _rowstride(o), _stream(stream)), "rbd_attn_int8")

@@ -73,6 +73,24 @@ bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uin
   return r == CUDA_SUCCESS;
 }
 
+// Row-major tensor of rank 2 or 3 (dims innermost first, strides in bytes for
+// dims 1..rank-1) with an explicit swizzle; used by the attention maps.
+bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint32_t rank, const uint64_t* dims,
+              const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[3], st[2];
+  cuuint32_t b[3], es[3] = {1, 1, 1};
+  for (uint32_t i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    if (i + 1 < rank) st[i] = strides[i];
+  }
+  CUresult r = fn(map, dt, rank, const_cast<void*>(base), d, st, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------
 // Library-owned scratch for rbd_nvfp4_quant_noalloc.  Some callers cannot hand
 // the library a scratch buffer: plain C hosts with no device allocator of their
@@ -352,6 +370,79 @@ rbd_status rbd_rope_tables(const int32_t* pos, int64_t T, double base, float* co
   if (!pos || !cos_t || !sin_t) return RBD_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(pos) & 3u) || !aligned16(cos_t) || !aligned16(sin_t)) return RBD_ERR_ALIGNMENT;
   return cuda_status(rbd::launch_rope_tables(pos, static_cast<int>(T), base, cos_t, sin_t, as_stream(stream)));
+}
+
+int64_t rbd_attn_workspace_bytes(int64_t Tk, int64_t H) {
+  if (Tk <= 0 || H <= 0) return -1;
+  return rbd::attn_workspace_bytes(Tk, H);
+}
+
+namespace {
+rbd_status attn_sizes_ok(int64_t Tq, int64_t Tk, int64_t H, int64_t tkp) {
+  if (Tq < 0 || Tk < 0 || H <= 0) return RBD_ERR_INVALID_ARG;
+  if (tkp < Tk || tkp % 8 != 0) return RBD_ERR_INVALID_ARG;
+  if (H > 256 || Tq > (1 << 24) || tkp > (1 << 24)) return RBD_ERR_UNSUPPORTED;
+  return RBD_OK;
+}
+}  // namespace
+
+rbd_status rbd_attn_quant(const void* q, int64_t ldq, const void* k, int64_t ldk, const void* v, int64_t ldv,
+                          int64_t Tq, int64_t Tk, int64_t H, int8_t* qc, float* sq, int8_t* kc, float* sk, void* vt,
+                          int64_t tkp, void* work, void* stream) {
+  rbd_status s = attn_sizes_ok(Tq, Tk, H, tkp);
+  if (s != RBD_OK) return s;
+  if (Tq == 0 && Tk == 0) return RBD_OK;
+  if (Tk == 0) return RBD_ERR_INVALID_ARG;   // queries with no keys have no softmax
+  if (!q || !k || !v || !qc || !sq || !kc || !sk || !vt || !work) return RBD_ERR_INVALID_ARG;
+  if (ldq < H * 128 || ldk < H * 128 || ldv < H * 128) return RBD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(qc) || !aligned16(kc) || !aligned16(vt) ||
+      !aligned16(sk) || !aligned16(work) || (ldq % 8) || (ldk % 8) || (ldv % 8) ||
+      (reinterpret_cast<uintptr_t>(sq) & 3u))
+    return RBD_ERR_ALIGNMENT;
+  return cuda_status(rbd::launch_attn_quant(static_cast<const uint16_t*>(q), ldq, static_cast<const uint16_t*>(k),
+                                            ldk, static_cast<const uint16_t*>(v), ldv, static_cast<int>(Tq),
+                                            static_cast<int>(Tk), static_cast<int>(H), qc, sq, kc, sk, vt, tkp, work,
+                                            as_stream(stream)));
+}
+
+rbd_status rbd_attn_int8(const int8_t* qc, const float* sq, const int8_t* kc, const float* sk, const void* vt,
+                         int64_t Tq, int64_t Tk, int64_t H, int64_t tkp, void* o, int64_t ldo, void* stream) {
+  rbd_status s = attn_sizes_ok(Tq, Tk, H, tkp);
+  if (s != RBD_OK) return s;
+  if (Tq == 0) return RBD_OK;
+  if (Tk == 0) return RBD_ERR_INVALID_ARG;
+  if (!qc || !sq || !kc || !sk || !vt || !o) return RBD_ERR_INVALID_ARG;
+  if (ldo < H * 128) return RBD_ERR_INVALID_ARG;
+  if (!aligned16(qc) || !aligned16(kc) || !aligned16(vt) || !aligned16(sk) || !aligned16(o) || (ldo % 8) ||
+      (reinterpret_cast<uintptr_t>(sq) & 3u))
+    return RBD_ERR_ALIGNMENT;
+  CUtensorMap tm_q{}, tm_k{}, tm_v{}, tm_sk{};
+  {
+    const uint64_t d[3] = {128, (uint64_t)Tq, (uint64_t)H}, st[2] = {128, (uint64_t)Tq * 128};
+    const uint32_t b[3] = {128, 128, 1};
+    if (!make_map(&tm_q, qc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B))
+      return RBD_ERR_CUDA;
+  }
+  {
+    const uint64_t d[3] = {128, (uint64_t)Tk, (uint64_t)H}, st[2] = {128, (uint64_t)Tk * 128};
+    const uint32_t b[3] = {128, 128, 1};
+    if (!make_map(&tm_k, kc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B))
+      return RBD_ERR_CUDA;
+  }
+  {
+    const uint64_t d[3] = {(uint64_t)tkp, 128, (uint64_t)H}, st[2] = {(uint64_t)tkp * 2, (uint64_t)tkp * 256};
+    const uint32_t b[3] = {64, 128, 1};
+    if (!make_map(&tm_v, vt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B))
+      return RBD_ERR_CUDA;
+  }
+  {
+    const uint64_t d[2] = {(uint64_t)tkp, (uint64_t)H}, st[1] = {(uint64_t)tkp * 4};
+    const uint32_t b[2] = {128, 1};
+    if (!make_map(&tm_sk, sk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, d, st, b, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return RBD_ERR_CUDA;
+  }
+  return cuda_status(rbd::launch_attn_int8(tm_q, tm_k, tm_v, tm_sk, sq, static_cast<int>(Tq), static_cast<int>(Tk),
+                                           static_cast<int>(H), static_cast<uint16_t*>(o), ldo, as_stream(stream)));
 }
 
 rbd_status rbd_pack_weights_int4(const void* w, int64_t N, int64_t K, rbd_qcfg cfg, uint8_t* packed, float* scales,

@@ -78,6 +78,15 @@ cudaError_t launch_kv4_encode(const uint16_t* x, int T, int H, int64_t ldt, int 
 cudaError_t launch_kv4_decode(const uint8_t* codes, const float* scales, int64_t capacity, int64_t slot0, int T,
                               int H, int n, uint16_t* y, int64_t ldt, cudaStream_t st);
 
+// INT8 attention (SageAttention v1 scheme): preparation and the attention kernel.
+int64_t attn_workspace_bytes(int64_t Tk, int64_t H);
+cudaError_t launch_attn_quant(const uint16_t* q, int64_t ldq, const uint16_t* k, int64_t ldk, const uint16_t* v,
+                              int64_t ldv, int Tq, int Tk, int H, int8_t* qc, float* sq, int8_t* kc, float* sk,
+                              void* vt, int64_t tkp, void* work, cudaStream_t st);
+cudaError_t launch_attn_int8(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                             const CUtensorMap& tm_sk, const float* sq, int Tq, int Tk, int H, uint16_t* o,
+                             int64_t ldo, cudaStream_t st);
+
 uint32_t gemm_smem_bytes(bool g64, int r, int G);   // dynamic shared memory of one GEMM CTA
 int gemm_tile_tokens(bool g64);                     // tokens per GEMM tile
 

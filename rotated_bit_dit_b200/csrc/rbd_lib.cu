@@ -7,3 +7,4 @@
 #include "rbd_nvfp4.cu"
 #include "rbd_kv4.cu"
 #include "rbd_rope.cu"
+#include "rbd_attn.cu"

@@ -243,3 +243,28 @@ def test_qk_norm_rope_validation_without_gpu():
     assert t(ctypes.c_void_p(0x10002), 4, 10000.0, FAKE, FAKE, null) == 3
     assert t(FAKE, 4, 10000.0, FAKE_MIS, FAKE, null) == 3
     assert t(FAKE, 1 << 26, 10000.0, FAKE, FAKE, null) == 2
+
+
+def test_attention_validation_without_gpu():
+    lib = R.load()
+    null = ctypes.c_void_p(0)
+    assert lib.rbd_attn_workspace_bytes(1000, 2) == (4 + 1) * 2 * 128 * 8     # 4 chunks of 256 keys + the mean
+    assert lib.rbd_attn_workspace_bytes(0, 2) == -1
+    aq, ai = lib.rbd_attn_quant, lib.rbd_attn_int8
+    args = lambda **kw: [kw.get(n, d) for n, d in (
+        ("q", FAKE), ("ldq", 256), ("k", FAKE), ("ldk", 256), ("v", FAKE), ("ldv", 256), ("Tq", 4), ("Tk", 8),
+        ("H", 2), ("qc", FAKE), ("sq", FAKE), ("kc", FAKE), ("sk", FAKE), ("vt", FAKE), ("tkp", 8), ("work", FAKE),
+        ("stream", null))]
+    assert aq(*args(tkp=4)) == 1                 # padded key count below Tk
+    assert aq(*args(tkp=12)) == 1                # padded key count not a multiple of 8
+    assert aq(*args(Tk=0)) == 1                  # queries without keys
+    assert aq(*args(Tq=0, Tk=0)) == 0            # nothing to do
+    assert aq(*args(ldk=200)) == 1               # row shorter than the heads
+    assert aq(*args(work=null)) == 1
+    assert aq(*args(v=FAKE_MIS)) == 3
+    assert aq(*args(ldq=260)) == 3
+    assert aq(*args(H=300)) == 2
+    assert ai(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 2, 8, FAKE, 200, null) == 1   # ldo < H * 128
+    assert ai(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0, 2, 8, FAKE, 256, null) == 1   # no keys
+    assert ai(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 2, 8, FAKE, 256, null) == 0   # no queries
+    assert ai(FAKE, FAKE, FAKE, FAKE_MIS, FAKE, 4, 8, 2, 8, FAKE, 256, null) == 3
