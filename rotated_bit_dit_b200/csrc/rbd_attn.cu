@@ -356,11 +356,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t lane_addr = (32u * qtr) << 16;
     const int qrow = q0 + row;
     const float cq = qrow < args.Tq ? __ldg(args.sq + (int64_t)h * args.Tq + qrow) * kLog2eRsqrtD : 0.f;
+    // waits whose outcome the whole warp shares: the warp's TMEM accesses are
+    // .sync.aligned, so its lanes must never part ways on a timeout
+    auto wait_warp = [](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity)) != 0;
+    };
     float m_use = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int s = j & 1;
-      if (!mbar_wait(&s_full[s], (j >> 1) & 1)) { ok = false; break; }
+      if (!wait_warp(&s_full[s], (j >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
       uint32_t sreg[kAttnTile];
 #pragma unroll
@@ -388,27 +393,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       // the P buffer of this tile is free once PV_{j-2} has completed
-      if (j >= 2 && !mbar_wait(&pv_done[s], ((j - 2) >> 1) & 1)) { ok = false; break; }
-      if (mt > m_use + kLazyRescale) {
-        if (j >= 1) {
-          // O holds PV_0 .. PV_{j-1}: wait for the last of them, then scale O in TMEM
-          if (!mbar_wait(&pv_done[s ^ 1], ((j - 1) >> 1) & 1)) { ok = false; break; }
-          tc_fence_after();
-          const float f = ex2(m_use - mt);
+      if (j >= 2 && !wait_warp(&pv_done[s], ((j - 2) >> 1) & 1)) { ok = false; break; }
+      // Each row decides for itself whether its maximum moves, but the TMEM loads and
+      // stores of a rescale are warp-wide (.sync.aligned): the warp rescales when any
+      // of its rows needs it, the other rows with factor 1.
+      const bool move = mt > m_use + kLazyRescale;
+      if (j >= 1 && __any_sync(0xffffffffu, move)) {
+        // O holds PV_0 .. PV_{j-1}: wait for the last of them, then scale O in TMEM
+        if (!wait_warp(&pv_done[s ^ 1], ((j - 1) >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const float f = move ? ex2(m_use - mt) : 1.0f;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(t_o + lane_addr + 32 * c, ov);
-            tmem_wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(t_o + lane_addr + 32 * c, ov);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-            tmem_st32(t_o + lane_addr + 32 * c, ov);
-          }
-          tmem_wait_st();
-          l *= f;
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+          tmem_st32(t_o + lane_addr + 32 * c, ov);
         }
-        m_use = mt;
+        tmem_wait_st();
+        l *= f;
       }
+      if (move) m_use = mt;
       // P = 2^(z - m) as fp16, written to this tile's P buffer (two 64-key halves,
       // row = query, 128-byte swizzle); the row sum stays in float32
       unsigned char* prow = smem + kPOff + s * 32768 + row * 128;
@@ -434,7 +441,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (lane == 0) mbar_arrive(&p_full[s]);
     }
     // O / l -> bf16, this thread's query row
-    if (ok && mbar_wait(o_done, 0)) {
+    if (ok && wait_warp(o_done, 0)) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
       uint16_t* orow = args.o + (int64_t)qrow * args.ldo + h * kAttnDim;

@@ -59,13 +59,15 @@ def test_attention_matches_oracle(Tq, Tk, H):
 
 def test_attention_running_maximum_moves_across_tiles():
     # keys grow in magnitude along the sequence and queries point along them, so later key tiles hold
-    # far larger scores than the first: the running maximum moves several times and O is rescaled
+    # far larger scores than the first: the running maximum moves several times and O is rescaled.
+    # (Much sharper inputs, a few keys carrying the weight, reach rel-L2 ~1e-3 from the fp16 rounding
+    # of P alone, the scheme's own P.V precision; these keys keep about a hundred in play.)
     Tq, Tk, H = 128, 1024, 1
     rng = np.random.default_rng(5)
     d = rng.standard_normal(128)
     d /= np.linalg.norm(d)
     ramp = np.linspace(0.0, 6.0, Tk)[:, None]
-    k = rng.standard_normal((Tk, 128)) * 0.3 + ramp * d[None, :] * 10
+    k = rng.standard_normal((Tk, 128)) * 1.0 + ramp * d[None, :] * 10
     q = rng.standard_normal((Tq, 128)) * 0.3 + d[None, :] * 3
     qb = I.f32_to_bf16_bits(q.astype(np.float32)).reshape(Tq, 1, 128)
     kb = I.f32_to_bf16_bits(k.astype(np.float32)).reshape(Tk, 1, 128)
