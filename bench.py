@@ -684,6 +684,78 @@ def run_qknorm_sweep(args):
             flush=True)
 
 
+# ----------------------------------------------------------------------------- INT8 attention
+def run_attn_sweep(args):
+    """INT8 attention (SageAttention v1 scheme) at 16384 tokens x 24 heads x 128 channels (a 2048 x 2048
+    image's latent with the 3072-wide model), self-attention on Q and K after the library's Q/K
+    RMSNorm + RoPE step (as attention receives them in the block): the preparation call (key smoothing,
+    INT8 codes and scales, fp16 V^T) and the attention call timed separately.  Work = Q.K^T
+    2 T^2 128 INT8 ops + P.V 2 T^2 128 fp16 FLOPs per head; the tensor floor is the INT8 part at the
+    measured INT8 ceiling plus the fp16 part at the measured bf16 dense peak (the same rate)."""
+    import torch
+
+    import rotated_bit_dit_b200 as R
+    from rotated_bit_dit_b200 import _binding as B
+    from rotated_bit_dit_b200 import inputs as I
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    R.load()
+    peaks, src = load_peaks()
+    int8_peak, int8_src = int8_peak_tops(peaks, src)
+    T, H = 16384, 24
+
+    def up(seed):
+        a = I.gaussian_bf16(seed, (T, H * 128), 1.0, 0.02, 20.0)
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v = up(20), up(21), up(22)
+    # Q and K as attention receives them: after the Q/K RMSNorm + RoPE step (one 128 x 128 frame)
+    pos = torch.from_numpy(I.video_positions(1, 128, 128)).to(dev)
+    cos = torch.empty((T, 64), dtype=torch.float32, device=dev)
+    sin = torch.empty((T, 64), dtype=torch.float32, device=dev)
+    B.rbd_rope_tables(pos, cos, sin)
+    B.rbd_qk_norm_rope(q, cos, sin, q, None, 1e-6)
+    B.rbd_qk_norm_rope(k, cos, sin, k, None, 1e-6)
+    qc, sq, kc, sk, vt = R.attention_operands(q, k, v, H)
+    work = torch.empty((B.rbd_attn_workspace_bytes(T, H),), dtype=torch.uint8, device=dev)
+    o = torch.empty((T, H * 128), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    ops_qk = 2.0 * T * T * 128 * H
+    floor_s = ops_qk / (int8_peak * 1e12) + ops_qk / (peaks["bf16_tflops"] * 1e12)
+    prep_bytes = T * H * 128 * 2 * 3 + 2 * T * H * 128 + 2 * T * H * 4 + T * H * 128 * 2
+    for case, fn in (("prepare", lambda: B.rbd_attn_quant(q, k, v, H, qc, sq, kc, sk, vt, work)),
+                     ("attention", lambda: B.rbd_attn_int8(qc, sq, kc, sk, vt, o))):
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        assert R.rbd_check() == 0
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) / 1e3)
+        assert R.rbd_check() == 0
+        t = statistics.median(ts)
+        line = {"sweep": "attn", "case": case, "tokens": T, "heads": H, "us": t * 1e6,
+                "timing": f"median of {args.steps} calls, each after a 256 MB L2 flush"}
+        if case == "attention":
+            line.update({"tops": 2 * ops_qk / t / 1e12, "tensor_floor_us": floor_s * 1e6,
+                         "frac_of_tensor_floor": floor_s / t,
+                         "peaks": f"INT8 {int8_peak:.0f} TOPS ({int8_src}); fp16 = {src} bf16 dense "
+                                  f"{peaks['bf16_tflops']} TFLOP/s"})
+        else:
+            gbs = prep_bytes / t / 1e9
+            line.update({"hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes": prep_bytes})
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- NVFP4 at the layer shape
 def run_nvfp4_sweep(args):
     """The NVFP4 variant at the grouped Q|K|V|gate shape (K = 3072, N = 12288, rank-32 branch, sigmoid
@@ -861,11 +933,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--print-gemm-hash", action="store_true", help="print the GEMM source hash and exit")
-    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4", "nvfp4", "qknorm", "peaks"], default=None,
+    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4", "nvfp4", "qknorm", "peaks", "attn"], default=None,
                     help="instead of the headline line, print the small-token-count sweep (one line per case)")
     args = ap.parse_args()
     if args.print_gemm_hash:
         print(gemm_source_hash())
+        return
+    if args.sweep == "attn":
+        run_attn_sweep(args)
         return
     if args.sweep == "peaks":
         run_peaks(args)

@@ -24,22 +24,27 @@
 //   attn_vt_kernel          V -> fp16, transposed to [head][channel][token];
 //   attn_int8_kernel        the attention itself, one CTA per (head, 128 queries).
 //
-// attn_int8_kernel, per CTA (6 warps):
-//   warp 0: TMA producer (Q once; K codes, key scales and V^T tiles of 128 keys
-//           into a 2-stage ring);
+// attn_int8_kernel, per CTA (11 warps):
+//   warps 0 and 10: TMA producers (Q once; K codes and key scales of 128-key
+//           tiles into a 2-stage ring freed by Q.K^T; V^T tiles into a 2-stage
+//           ring freed by P.V);
 //   warp 1: TMEM owner and MMA issuer: S_j = Q K_j^T (kind::i8, int32) into one
 //           of two 128-column S buffers, O += P_j V_j (kind::f16, fp32) into a
 //           third 128-column buffer;
-//   warps 2-5: softmax, thread = query row (TMEM lane): the row of S_j (128
-//           int32) is loaded once into registers, turned into base-2 logits,
-//           masked past Tk, and exponentiated against the row's running maximum
-//           m.  m only moves when a tile's maximum exceeds it by more than 8
-//           (so P <= 256 stays well inside fp16); O and the running sum are then
-//           rescaled in TMEM first.  P goes to shared memory as fp16 in the
-//           128-byte-swizzled K-major layout the P.V MMA reads.
+//   warps 2-9: softmax, two threads per query row (TMEM lane), each with 64 of
+//           the tile's keys: its part of the row of S_j (int32) is loaded once
+//           into registers, scaled, the pair's row maximum exchanged through
+//           shared memory, keys past Tk masked, and 2^(logit - m) taken against
+//           the row's running maximum m.  m only moves when a tile's maximum exceeds it by more than 8
+//           (so P <= 256 stays well inside fp16); O is then rescaled in TMEM
+//           first.  P goes to shared memory as fp16 in the 128-byte-swizzled
+//           K-major layout the P.V MMA reads.  The P.V MMA is N = 144 wide: 16
+//           rows of ones below V^T make its column 128 the row sum of P.
 // The tensor core runs QK_{j+1} while the softmax works on tile j, and PV_j
 // while it works on tile j + 1.
 #include <cuda_fp16.h>
+
+#include <type_traits>
 
 #include "rbd_common.cuh"
 #include "rbd_internal.cuh"
@@ -50,19 +55,31 @@ namespace {
 
 constexpr int kAttnDim = 128;           // channels per head
 constexpr int kAttnTile = 128;          // queries per CTA, keys per tile
-constexpr int kAttnThreads = 192;       // 6 warps
+constexpr int kAttnThreads = 352;       // 11 warps
+constexpr int kAttnVWarp = 10;          // the V producer
 constexpr int kAttnSoftmax0 = 2;        // first softmax warp
 constexpr int kColsumChunk = 256;       // tokens per partial column sum
 constexpr float kLog2eRsqrtD = 0.12751743082459868f;   // log2(e) / sqrt(128)
 constexpr float kLazyRescale = 8.0f;    // base-2 headroom before the running maximum moves
 
+// The P.V MMA runs with N = 144: rows 128..143 of every V^T half hold fp16 ones,
+// so O's column 128 accumulates the row sum of exactly the fp16 P that P.V
+// multiplies (the softmax denominator), rescaled together with O.
+constexpr int kPvN = kAttnDim + 16;
+constexpr uint32_t kVHalf = kPvN * 128;                // 144 rows x 128 B (64 keys)
+
 // shared-memory layout of attn_int8_kernel (offsets from a 1024-byte aligned base)
 constexpr uint32_t kQOff = 0;                          // Q codes, 128 x 128 B
 constexpr uint32_t kKOff = kQOff + 16384;              // K codes, 2 stages x 16 KB
-constexpr uint32_t kVOff = kKOff + 2 * 16384;          // V^T, 2 stages x 2 halves x 16 KB
-constexpr uint32_t kPOff = kVOff + 2 * 32768;          // P, 2 buffers x 2 halves x 16 KB
-constexpr uint32_t kSkOff = kPOff + 2 * 32768;         // key scales, 2 stages x 512 B
-constexpr uint32_t kBarOff = kSkOff + 2 * 512;
+constexpr uint32_t kVOff = kKOff + 2 * 16384;          // V^T (+ ones), 2 stages x 2 halves x 18 KB
+constexpr uint32_t kPOff = kVOff + 4 * kVHalf;         // P, 2 buffers x 2 halves x 16 KB
+// Key scales ride with the K codes but are read by the softmax, after Q.K^T: they
+// get a 4-deep ring.  Slot j % 4 is rewritten for tile j + 4 only after Q.K^T of
+// tile j + 2, which waits for the softmax of tile j to release its S buffer, which
+// it does after reading the slot.
+constexpr uint32_t kSkOff = kPOff + 2 * 32768;         // key scales, 4 slots x 512 B
+constexpr uint32_t kRedOff = kSkOff + 4 * 512;         // row-maximum exchange, 2 x 2 x 128 floats
+constexpr uint32_t kBarOff = kRedOff + 2048;
 constexpr uint32_t kAttnSmem = kBarOff + 256 + 1024;   // + alignment slack
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
@@ -109,6 +126,16 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// 32 lanes x 16 columns register -> TMEM store.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 
@@ -244,15 +271,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023u) & ~uintptr_t(1023u));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;    // [2]
-  uint64_t* kv_empty = bars + 3;   // [2]
+  uint64_t* k_full = bars + 1;     // [2] K codes and key scales of a stage landed
+  uint64_t* k_empty = bars + 3;    // [2] Q.K^T of the stage's tile done
+  uint64_t* v_full = bars + 21;    // [2] V^T of a stage landed
+  uint64_t* v_empty = bars + 23;   // [2] P.V of the stage's tile done
   uint64_t* s_full = bars + 5;     // [2]
   uint64_t* s_empty = bars + 7;    // [2]
   uint64_t* p_full = bars + 9;     // [2]
   uint64_t* pv_done = bars + 11;   // [2]
   uint64_t* o_done = bars + 13;
   uint64_t* drain = bars + 14;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* red_bar = bars + 15;   // [2] the pair's row maxima are in shared memory
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 26);
 
   const uint32_t warp = warp_id(), lane = lane_id();
   const int h = blockIdx.y;
@@ -262,15 +292,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 0 && lane == 0) {
     mbar_init(q_full, 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&kv_full[b], 1);
-      mbar_init(&kv_empty[b], 1);
+      mbar_init(&k_full[b], 1);
+      mbar_init(&k_empty[b], 1);
+      mbar_init(&v_full[b], 1);
+      mbar_init(&v_empty[b], 1);
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 4);
-      mbar_init(&p_full[b], 4);
+      mbar_init(&s_empty[b], 8);
+      mbar_init(&p_full[b], 8);
       mbar_init(&pv_done[b], 1);
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
+    mbar_init(&red_bar[0], 8);
+    mbar_init(&red_bar[1], 8);
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -282,25 +316,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_relinquish();
     tc_fence_before();
   }
+  // the ones rows (128..143) of the four V^T halves: 4 x 2 KB of fp16 1.0
+  for (int i = threadIdx.x; i < 4 * 128; i += kAttnThreads) {
+    const int hv = i >> 7, w = i & 127;
+    reinterpret_cast<uint4*>(smem + kVOff + hv * kVHalf + 16384)[w] =
+        make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+  }
+  fence_async_shared();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t t_o = tmem + 2 * kAttnTile;   // O accumulator columns 256..383
+  const uint32_t t_o = tmem + 2 * kAttnTile;   // O accumulator columns 256..399 (column 384: the row sum)
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == kAttnVWarp) {
+    // ------------------------------------------------------------ TMA producers
+    // warp 0: Q once, then K codes and key scales (a stage is free once its Q.K^T is
+    // done); warp 10: V^T (a stage is free once its P.V is done)
     if (lane == 0) {
+      const bool kprod = warp == 0;
       bool ok = true;
-      mbar_arrive_expect_tx(q_full, 16384);
-      tma_load_3d(smem + kQOff, &tm_q, q_full, 0, q0, h);
+      if (kprod) {
+        mbar_arrive_expect_tx(q_full, 16384);
+        tma_load_3d(smem + kQOff, &tm_q, q_full, 0, q0, h);
+      }
       for (int j = 0; j < ntiles && ok; ++j) {
         const int s = j & 1;
-        if (!mbar_wait(&kv_empty[s], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(&kv_full[s], 16384 + 32768 + 512);
-        tma_load_3d(smem + kKOff + s * 16384, &tm_k, &kv_full[s], 0, j * kAttnTile, h);
-        tma_load_3d(smem + kVOff + s * 32768, &tm_v, &kv_full[s], j * kAttnTile, 0, h);
-        tma_load_3d(smem + kVOff + s * 32768 + 16384, &tm_v, &kv_full[s], j * kAttnTile + 64, 0, h);
-        tma_load_2d(smem + kSkOff + s * 512, &tm_sk, &kv_full[s], j * kAttnTile, h);
+        if (kprod) {
+          if (!mbar_wait(&k_empty[s], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[s], 16384 + 512);
+          tma_load_3d(smem + kKOff + s * 16384, &tm_k, &k_full[s], 0, j * kAttnTile, h);
+          tma_load_2d(smem + kSkOff + (j & 3) * 512, &tm_sk, &k_full[s], j * kAttnTile, h);
+        } else {
+          if (!mbar_wait(&v_empty[s], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&v_full[s], 32768);
+          tma_load_3d(smem + kVOff + (2 * s) * kVHalf, &tm_v, &v_full[s], j * kAttnTile, 0, h);
+          tma_load_3d(smem + kVOff + (2 * s + 1) * kVHalf, &tm_v, &v_full[s], j * kAttnTile + 64, 0, h);
+        }
       }
       if (!ok) {
         const uint64_t t0 = globaltimer_ns();
@@ -311,37 +362,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
       const uint32_t id_qk = idesc_i8(kAttnTile, kAttnTile);
-      const uint32_t id_pv = idesc_f16(kAttnTile, kAttnDim);
+      const uint32_t id_pv = idesc_f16(kAttnTile, kPvN);
       const uint64_t qdesc = smem_desc_kmajor(smem_u32(smem + kQOff), 128);
       bool ok = mbar_wait(q_full, 0);
       tc_fence_after();
       auto issue_qk = [&](int j) {
         const int s = j & 1;
-        if (!mbar_wait(&kv_full[s], (j >> 1) & 1)) return false;
+        if (!mbar_wait(&k_full[s], (j >> 1) & 1)) return false;
         if (j >= 2 && !mbar_wait(&s_empty[s], ((j - 2) >> 1) & 1)) return false;
         tc_fence_after();
         const uint64_t kdesc = smem_desc_kmajor(smem_u32(smem + kKOff + s * 16384), 128);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) mma_i8_ss(tmem + s * kAttnTile, qdesc + 2 * kk, kdesc + 2 * kk, id_qk, kk > 0);
         tc_commit(&s_full[s]);
+        tc_commit(&k_empty[s]);
         return true;
       };
       if (ok) ok = issue_qk(0);
       if (ok && ntiles > 1) ok = issue_qk(1);
       for (int j = 0; j < ntiles && ok; ++j) {
         const int s = j & 1;
-        if (!mbar_wait(&p_full[s], (j >> 1) & 1)) { ok = false; break; }
+        if (!mbar_wait(&p_full[s], (j >> 1) & 1) || !mbar_wait(&v_full[s], (j >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t pbase = smem_u32(smem + kPOff + s * 32768);
-        const uint32_t vbase = smem_u32(smem + kVOff + s * 32768);
+        const uint32_t vbase = smem_u32(smem + kVOff + 2 * s * kVHalf);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t half = (uint32_t)(kk >> 2) * 16384u, off = (uint32_t)(kk & 3) * 32u;
-          mma_bf16_ss(t_o, smem_desc_kmajor(pbase + half + off, 128), smem_desc_kmajor(vbase + half + off, 128),
+          const uint32_t ph = (uint32_t)(kk >> 2) * 16384u, vh = (uint32_t)(kk >> 2) * kVHalf;
+          const uint32_t off = (uint32_t)(kk & 3) * 32u;
+          mma_bf16_ss(t_o, smem_desc_kmajor(pbase + ph + off, 128), smem_desc_kmajor(vbase + vh + off, 128),
                       id_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(&pv_done[s]);
-        tc_commit(&kv_empty[s]);
+        tc_commit(&v_empty[s]);
         if (j + 2 < ntiles && !issue_qk(j + 2)) { ok = false; break; }
       }
       tc_commit(o_done);
@@ -349,54 +402,77 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(drain, 0, 100000000ull);
     }
     __syncwarp();
-  } else {
+  } else if (warp < kAttnVWarp) {
     // ------------------------------------------------------------ softmax warps
+    // Warp w (2..9) covers query rows 32 (w & 3) .. +31 (its TMEM lane quarter) and
+    // keys 64 half .. +63 of every tile (half = (w - 2) >> 2): two warps per row.
+    // The pair exchanges its two row maxima through shared memory once per tile.
     const uint32_t qtr = warp & 3u;
+    const int half = ((int)warp - kAttnSoftmax0) >> 2;
     const int row = 32 * (int)qtr + (int)lane;                  // query row inside the tile (TMEM lane)
     const uint32_t lane_addr = (32u * qtr) << 16;
     const int qrow = q0 + row;
     const float cq = qrow < args.Tq ? __ldg(args.sq + (int64_t)h * args.Tq + qrow) * kLog2eRsqrtD : 0.f;
+    float* red = reinterpret_cast<float*>(smem + kRedOff);     // [2 tiles][2 halves][128 rows]
     // waits whose outcome the whole warp shares: the warp's TMEM accesses are
     // .sync.aligned, so its lanes must never part ways on a timeout
     auto wait_warp = [](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity)) != 0;
     };
-    float m_use = -INFINITY, l = 0.f;
+    float m_use = -INFINITY;   // running maximum, base-2 logits
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int s = j & 1;
       if (!wait_warp(&s_full[s], (j >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sreg[kAttnTile];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_addr + s * kAttnTile + 32 * c, sreg + 32 * c);
+      uint32_t sreg[64];
+      tmem_ld32(tmem + lane_addr + s * kAttnTile + 64 * half, sreg);
+      tmem_ld32(tmem + lane_addr + s * kAttnTile + 64 * half + 32, sreg + 32);
       tmem_wait_ld();
+      // u = acc * s_k (the logit is u * cq, cq = s_q log2(e) / sqrt(128) >= 0, so the row
+      // maximum of u gives that of the logits); keys past Tk are left out (last tile only)
+      const float4* sk4 = reinterpret_cast<const float4*>(smem + kSkOff + (j & 3) * 512) + 16 * half;
+      const int nvalid = args.Tk - j * kAttnTile - 64 * half;   // valid keys of this half
+      const bool full = nvalid >= 64;
+      float mx[8];   // eight independent max chains
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+      auto logits = [&](auto full_tile) {
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 kq = sk4[c4];
+          const float ks[4] = {kq.x, kq.y, kq.z, kq.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = 4 * c4 + e;
+            const float a = __uint_as_float(sreg[col] + 0x4B400000u) - 12582912.0f;   // exact: |acc| < 2^22
+            const float u = a * ks[e];
+            if (decltype(full_tile)::value || col < nvalid) mx[col & 7] = fmaxf(mx[col & 7], u);
+            sreg[col] = __float_as_uint(u);
+          }
+        }
+      };
+      if (full) logits(std::true_type{});
+      else logits(std::false_type{});
+      float mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      // S buffer read and key-scale slot read: release the S buffer
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[s]);
-      // base-2 logits z = acc * s_q * s_k * log2(e) / sqrt(128); keys past Tk masked
-      const float4* sk4 = reinterpret_cast<const float4*>(smem + kSkOff + s * 512);
-      const int nvalid = args.Tk - j * kAttnTile;
-      float mt = -INFINITY;
-#pragma unroll
-      for (int c4 = 0; c4 < kAttnTile / 4; ++c4) {
-        const float4 kq = sk4[c4];
-        const float ks[4] = {kq.x, kq.y, kq.z, kq.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int col = 4 * c4 + e;
-          const float a = __uint_as_float(sreg[col] + 0x4B400000u) - 12582912.0f;   // exact: |acc| < 2^22
-          float z = a * (cq * ks[e]);
-          if (col >= nvalid) z = -INFINITY;
-          mt = fmaxf(mt, z);
-          sreg[col] = __float_as_uint(z);
-        }
-      }
+      red[(s * 2 + half) * kAttnTile + row] = mh;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&red_bar[s]);
+      if (!wait_warp(&red_bar[s], (j >> 1) & 1)) { ok = false; break; }
+      mh = fmaxf(mh, red[(s * 2 + (half ^ 1)) * kAttnTile + row]);
+      const float mt = mh * cq;                                  // the tile's row maximum, base 2
       // the P buffer of this tile is free once PV_{j-2} has completed
       if (j >= 2 && !wait_warp(&pv_done[s], ((j - 2) >> 1) & 1)) { ok = false; break; }
-      // Each row decides for itself whether its maximum moves, but the TMEM loads and
-      // stores of a rescale are warp-wide (.sync.aligned): the warp rescales when any
-      // of its rows needs it, the other rows with factor 1.
+      // Each row decides for itself whether its maximum moves (both warps of the pair
+      // decide alike), but the TMEM loads and stores of a rescale are warp-wide
+      // (.sync.aligned): the warp rescales when any of its rows needs it, the other
+      // rows with factor 1.  Half 0 rescales O columns 0..63 and the row-sum block
+      // 128..143, half 1 columns 64..127.
       const bool move = mt > m_use + kLazyRescale;
       if (j >= 1 && __any_sync(0xffffffffu, move)) {
         // O holds PV_0 .. PV_{j-1}: wait for the last of them, then scale O in TMEM
@@ -404,51 +480,67 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
         const float f = move ? ex2(m_use - mt) : 1.0f;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t ov[32];
-          tmem_ld32(t_o + lane_addr + 32 * c, ov);
+          tmem_ld32(t_o + lane_addr + 64 * half + 32 * c, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-          tmem_st32(t_o + lane_addr + 32 * c, ov);
+          tmem_st32(t_o + lane_addr + 64 * half + 32 * c, ov);
+        }
+        if (half == 0) {
+          uint32_t ov[16];   // columns 128..143: the row sum and the unused rest
+          tmem_ld16(t_o + lane_addr + kAttnDim, ov);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+          tmem_st16(t_o + lane_addr + kAttnDim, ov);
         }
         tmem_wait_st();
-        l *= f;
       }
       if (move) m_use = mt;
-      // P = 2^(z - m) as fp16, written to this tile's P buffer (two 64-key halves,
-      // row = query, 128-byte swizzle); the row sum stays in float32
-      unsigned char* prow = smem + kPOff + s * 32768 + row * 128;
+      // P = 2^(u cq - m) as fp16 into this half of the tile's P buffer (row = query,
+      // 128-byte swizzle); masked keys get P = 0; the P.V MMA's ones column sums it
+      unsigned char* prow = smem + kPOff + s * 32768 + half * 16384 + row * 128;
+      const float nm = -m_use;
+      auto probs = [&](auto full_tile) {
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        uint32_t packed[4];
+        for (int c8 = 0; c8 < 8; ++c8) {
+          uint32_t packed[4];
 #pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const int col = 8 * ch + 2 * e2;
-          const float p0 = ex2(__uint_as_float(sreg[col]) - m_use);
-          const float p1 = ex2(__uint_as_float(sreg[col + 1]) - m_use);
-          const __half2 hp = __floats2half2_rn(p0, p1);
-          l += __low2float(hp) + __high2float(hp);   // the sum of what P.V multiplies
-          packed[e2] = *reinterpret_cast<const uint32_t*>(&hp);
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const int col = 8 * c8 + 2 * e2;
+            float p0 = ex2(fmaf(__uint_as_float(sreg[col]), cq, nm));
+            float p1 = ex2(fmaf(__uint_as_float(sreg[col + 1]), cq, nm));
+            if (!decltype(full_tile)::value) {
+              p0 = col < nvalid ? p0 : 0.f;
+              p1 = col + 1 < nvalid ? p1 : 0.f;
+            }
+            const __half2 hp = __floats2half2_rn(p0, p1);
+            packed[e2] = *reinterpret_cast<const uint32_t*>(&hp);
+          }
+          *reinterpret_cast<uint4*>(prow + ((c8 ^ (row & 7)) << 4)) =
+              make_uint4(packed[0], packed[1], packed[2], packed[3]);
         }
-        const int half = ch >> 3, c8 = ch & 7;
-        *reinterpret_cast<uint4*>(prow + half * 16384 + ((c8 ^ (row & 7)) << 4)) =
-            make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      }
+      };
+      if (full) probs(std::true_type{});
+      else probs(std::false_type{});
       fence_async_shared();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[s]);
     }
-    // O / l -> bf16, this thread's query row
+    // O / l -> bf16: this warp's 64 output channels of its query rows
     if (ok && wait_warp(o_done, 0)) {
       tc_fence_after();
+      uint32_t lv[16];
+      tmem_ld16(t_o + lane_addr + kAttnDim, lv);
+      const float l = __uint_as_float(lv[0]);
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-      uint16_t* orow = args.o + (int64_t)qrow * args.ldo + h * kAttnDim;
+      uint16_t* orow = args.o + (int64_t)qrow * args.ldo + h * kAttnDim + 64 * half;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t ov[32];
-        tmem_ld32(t_o + lane_addr + 32 * c, ov);
+        tmem_ld32(t_o + lane_addr + 64 * half + 32 * c, ov);
         tmem_wait_ld();
         if (qrow < args.Tq) {
 #pragma unroll
