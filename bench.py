@@ -756,6 +756,34 @@ def run_attn_sweep(args):
         print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- offline SVDQuant fit
+def run_svdquant_sweep(args):
+    """The offline SVDQuant fit (rbd_svdquant_fit) of the Q|K|V|gate weight (N = 12288, K = 3072),
+    INT4 group-64, rank 32, oversampling 8, three iterates; wall time of the synchronous call (the
+    fit is offline: float64 products on the device, QR / SVD on the host)."""
+    import torch
+
+    import rotated_bit_dit_b200 as R
+    from rotated_bit_dit_b200 import inputs as I
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    R.load()
+    N, K, rank, iters = 12288, 3072, 32, 3
+    w = torch.from_numpy(np.ascontiguousarray(I.gaussian_bf16(30, (N, K), 0.02)).view(np.int16))
+    w = w.view(torch.bfloat16).to(dev)
+    om = np.random.default_rng(31).standard_normal((iters, K, rank + 8))
+    R.rbd_svdquant_fit(w, rank, om[:1], 4, 256, 64)        # warm-up (one iterate)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    out = R.rbd_svdquant_fit(w, rank, om, 4, 256, 64)
+    dt = time.perf_counter() - t0
+    assert R.rbd_check() == 0
+    print(json.dumps({"sweep": "svdquant", "N": N, "K": K, "rank": rank, "oversample": 8, "iters": iters,
+                      "seconds": dt, "errs": out["errs"].tolist(), "best": out["best"],
+                      "timing": "wall time of one synchronous call after a one-iterate warm-up"}), flush=True)
+
+
 # ----------------------------------------------------------------------------- NVFP4 at the layer shape
 def run_nvfp4_sweep(args):
     """The NVFP4 variant at the grouped Q|K|V|gate shape (K = 3072, N = 12288, rank-32 branch, sigmoid
@@ -933,11 +961,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--print-gemm-hash", action="store_true", help="print the GEMM source hash and exit")
-    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4", "nvfp4", "qknorm", "peaks", "attn"], default=None,
+    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4", "nvfp4", "qknorm", "peaks", "attn", "svdquant"], default=None,
                     help="instead of the headline line, print the small-token-count sweep (one line per case)")
     args = ap.parse_args()
     if args.print_gemm_hash:
         print(gemm_source_hash())
+        return
+    if args.sweep == "svdquant":
+        run_svdquant_sweep(args)
         return
     if args.sweep == "attn":
         run_attn_sweep(args)

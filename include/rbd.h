@@ -385,6 +385,44 @@ rbd_status rbd_attn_quant(const void* q, int64_t ldq, const void* k, int64_t ldk
 rbd_status rbd_attn_int8(const int8_t* qc, const float* sq, const int8_t* kc, const float* sk, const void* vt,
                          int64_t Tq, int64_t Tk, int64_t H, int64_t tkp, void* o, int64_t ldo, void* stream);
 
+/* ---- Offline SVDQuant fit of the low-rank branch --------------------------
+ * "Krea-2-SVDQuant-ComfyUI", "Low-rank refinement, and what the objective
+ * actually is" and "Activation-aware branch".  Minimises
+ * ||(W - (deq(Q) + L)) diag(d)||_F over a rank-r branch L and codes Q in the
+ * layer's own rotated format (cfg: bits 4 or 8, rot_group, scale_group;
+ * code_format RBD_CODES_INT8): iterate 1 splits W by a randomized SVD of
+ * W diag(d) (test matrix omega_1, one power iteration, QR after every
+ * product); each later iterate re-fits the branch to (W - deq(Q)) diag(d) with
+ * its own test matrix and quantises bf16(W - L) again; the iterate with the
+ * smallest error is kept.  d = act_rms / mean(act_rms), floored at 0.05, or
+ * all ones when act_rms is NULL.
+ *
+ * Bytes of device scratch for an N x K weight, rank r and oversampling p
+ * (-1 for an unsupported configuration).                                    */
+int64_t rbd_svdquant_workspace_bytes(int64_t N, int64_t K, int32_t rank, int32_t oversample, rbd_qcfg cfg);
+
+/* The fit.  SYNCHRONOUS: it waits for the device between steps (the thin QR
+ * factorisations and the (r+p) x K SVD run on the host in float64; the
+ * products with W, the requantisation, dequantisation and error run on the
+ * device in float64).
+ *   w        bf16 [N, K] device, 16-byte aligned; K a multiple of 256 with
+ *            rotation (of 64 without), K <= 16384.
+ *   omegas   HOST float64 [iters][K][rank + oversample]: the Gaussian test
+ *            matrices (inputs, one per iterate).
+ *   act_rms  HOST float64 [K] or NULL.
+ *   q, scales  device: the kept iterate's codes (packed INT4 [N, K/2] or INT8
+ *            [N, K], as rbd_pack_weights_*) and scales.
+ *   l1       HOST float64 [K][rank] = (V / d) sqrt(S); l2 HOST float64
+ *            [rank][N] = sqrt(S) U^T, so that the branch adds (x l1) l2.
+ *   errs     HOST float64 [iters]: the objective after every iterate;
+ *   best     HOST int32 (may be NULL): index of the kept iterate.
+ *   work     rbd_svdquant_workspace_bytes(...) bytes of device scratch,
+ *            16-byte aligned.
+ * rank + oversample <= min(N, K, 256).                                       */
+rbd_status rbd_svdquant_fit(const void* w, int64_t N, int64_t K, rbd_qcfg cfg, int32_t rank, int32_t oversample,
+                            int32_t iters, const double* omegas, const double* act_rms, void* q, float* scales,
+                            double* l1, double* l2, double* errs, int32_t* best, void* work, void* stream);
+
 /* Synchronises `stream`, then reports the first device-side error recorded
  * since the last rbd_check (RBD_ERR_DEVICE_TIMEOUT) or a CUDA error, and
  * clears the device status word.                                              */

@@ -37,6 +37,7 @@ from ._binding import (  # noqa: F401
     rbd_attn_workspace_bytes,
     rbd_attn_quant,
     rbd_attn_int8,
+    rbd_svdquant_fit,
 )
 from .attention import attention_operands, int8_attention  # noqa: F401
 from .kvcache import Int4KVCache  # noqa: F401

@@ -22,6 +22,7 @@ STATUS_NAMES = {0: "RBD_OK", 1: "RBD_ERR_INVALID_ARG", 2: "RBD_ERR_UNSUPPORTED",
 EXPORTED = ("rbd_rot_quant_act", "rbd_norm_rot_quant_act", "rbd_lowrank_fused", "rbd_lowrank_down", "rbd_pack_weights_int4", "rbd_pack_weights_int8",
             "rbd_w4a4_linear", "rbd_w8a8_linear", "rbd_nvfp4_scale_bytes", "rbd_nvfp4_quant",
             "rbd_nvfp4_quant_noalloc", "rbd_nvfp4_linear", "rbd_kv4_encode", "rbd_kv4_decode", "rbd_qk_norm_rope", "rbd_rope_tables", "rbd_attn_workspace_bytes", "rbd_attn_quant", "rbd_attn_int8",
+            "rbd_svdquant_workspace_bytes", "rbd_svdquant_fit",
             "rbd_check", "rbd_debug_timeout_probe", "rbd_status_string", "rbd_version")
 
 
@@ -84,6 +85,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         "rbd_rope_tables": [vp, i64, ctypes.c_double, vp, vp, vp],
         "rbd_attn_quant": [vp, i64, vp, i64, vp, i64, i64, i64, i64, vp, vp, vp, vp, vp, i64, vp, vp],
         "rbd_attn_int8": [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i64, vp],
+        "rbd_svdquant_fit": [vp, i64, i64, QCfg, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "rbd_check": [vp],
         "rbd_debug_timeout_probe": [i64, vp],
     }
@@ -95,6 +97,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.rbd_nvfp4_scale_bytes.restype = i64
     lib.rbd_attn_workspace_bytes.argtypes = [i64, i64]
     lib.rbd_attn_workspace_bytes.restype = i64
+    lib.rbd_svdquant_workspace_bytes.argtypes = [i64, i64, i32, i32, QCfg]
+    lib.rbd_svdquant_workspace_bytes.restype = i64
     lib.rbd_status_string.argtypes = [ctypes.c_int]
     lib.rbd_status_string.restype = ctypes.c_char_p
     lib.rbd_version.argtypes = []
@@ -364,3 +368,35 @@ def rbd_attn_int8(qc: torch.Tensor, sq: torch.Tensor, kc: torch.Tensor, sk: torc
     Tk = kc.shape[1]
     _ok(load().rbd_attn_int8(_ptr(qc), _ptr(sq), _ptr(kc), _ptr(sk), _ptr(vt), Tq, Tk, H, sk.shape[1], _ptr(o),
                              _rowstride(o), _stream(stream)), "rbd_attn_int8")
+
+
+def rbd_svdquant_fit(w: torch.Tensor, rank: int, omegas, bits: int = 4, rot_group: int = 256, scale_group: int = 0,
+                     act_rms=None, stream=None):
+    """The offline SVDQuant fit of a bf16 [N, K] CUDA weight.  omegas: float64 array-like
+    [iters, K, rank + oversample] (the test matrices); act_rms: float64 [K] or None.
+    Returns dict(q, scales (CUDA tensors of the kept iterate), l1 [K, rank], l2 [rank, N] (float64
+    numpy), errs [iters] (float64 numpy), best).  Synchronous."""
+    import numpy as np
+    N, K = w.shape
+    om = np.ascontiguousarray(omegas, dtype=np.float64)
+    iters, k_, p = om.shape
+    if k_ != K or p < rank:
+        raise ValueError("omegas must be [iters, K, rank + oversample]")
+    cfg = _qcfg(bits, rot_group, scale_group)
+    nbytes = int(load().rbd_svdquant_workspace_bytes(N, K, rank, p - rank, cfg))
+    if nbytes < 0:
+        raise RbdError(2, "rbd_svdquant_workspace_bytes")
+    dev = w.device
+    work = torch.empty((nbytes,), dtype=torch.uint8, device=dev)
+    q = torch.empty((N, K // 2) if bits == 4 else (N, K), dtype=torch.uint8 if bits == 4 else torch.int8, device=dev)
+    scales = torch.empty((N, K // 64) if scale_group else (N,), dtype=torch.float32, device=dev)
+    l1 = np.zeros((K, rank), np.float64)
+    l2 = np.zeros((rank, N), np.float64)
+    errs = np.zeros(iters, np.float64)
+    best = ctypes.c_int32(-1)
+    ar = None if act_rms is None else np.ascontiguousarray(act_rms, dtype=np.float64)
+    dp = lambda a: None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+    _ok(load().rbd_svdquant_fit(_ptr(w), N, K, cfg, rank, p - rank, iters, dp(om), dp(ar), _ptr(q), _ptr(scales),
+                                dp(l1), dp(l2), dp(errs), ctypes.byref(best), _ptr(work), _stream(stream)),
+        "rbd_svdquant_fit")
+    return dict(q=q, scales=scales, l1=l1, l2=l2, errs=errs, best=int(best.value))

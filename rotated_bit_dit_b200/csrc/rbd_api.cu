@@ -445,6 +445,40 @@ rbd_status rbd_attn_int8(const int8_t* qc, const float* sq, const int8_t* kc, co
                                            static_cast<int>(H), static_cast<uint16_t*>(o), ldo, as_stream(stream)));
 }
 
+namespace {
+rbd_status svdquant_cfg_ok(int64_t N, int64_t K, rbd_qcfg cfg, int32_t rank, int32_t oversample) {
+  rbd_status s = check_qcfg(cfg, K);
+  if (s != RBD_OK) return s;
+  if (cfg.code_format != RBD_CODES_INT8) return RBD_ERR_UNSUPPORTED;
+  if (N <= 0 || rank <= 0 || oversample < 0) return RBD_ERR_INVALID_ARG;
+  const int64_t p = (int64_t)rank + oversample;
+  if (p > N || p > K || p > 256 || N > (1 << 20)) return RBD_ERR_UNSUPPORTED;
+  return RBD_OK;
+}
+}  // namespace
+
+int64_t rbd_svdquant_workspace_bytes(int64_t N, int64_t K, int32_t rank, int32_t oversample, rbd_qcfg cfg) {
+  if (svdquant_cfg_ok(N, K, cfg, rank, oversample) != RBD_OK) return -1;
+  return rbd::svdquant_workspace_bytes(N, K, rank, oversample, cfg.bits, cfg.scale_group);
+}
+
+rbd_status rbd_svdquant_fit(const void* w, int64_t N, int64_t K, rbd_qcfg cfg, int32_t rank, int32_t oversample,
+                            int32_t iters, const double* omegas, const double* act_rms, void* q, float* scales,
+                            double* l1, double* l2, double* errs, int32_t* best, void* work, void* stream) {
+  rbd_status s = svdquant_cfg_ok(N, K, cfg, rank, oversample);
+  if (s != RBD_OK) return s;
+  if (iters <= 0) return RBD_ERR_INVALID_ARG;
+  if (!w || !omegas || !q || !scales || !l1 || !l2 || !errs || !work) return RBD_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(q) || !aligned16(work) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return RBD_ERR_ALIGNMENT;
+  int b = -1;
+  const cudaError_t e = rbd::svdquant_fit(static_cast<const uint16_t*>(w), N, K, cfg.bits, cfg.rot_group != 0,
+                                          cfg.scale_group, rank, oversample, iters, omegas, act_rms, q, scales,
+                                          l1, l2, errs, &b, work, as_stream(stream));
+  if (best) *best = b;
+  return cuda_status(e);
+}
+
 rbd_status rbd_pack_weights_int4(const void* w, int64_t N, int64_t K, rbd_qcfg cfg, uint8_t* packed, float* scales,
                                  void* stream) {
   if (cfg.bits != 4) return RBD_ERR_INVALID_ARG;

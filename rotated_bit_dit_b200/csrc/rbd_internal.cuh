@@ -87,6 +87,13 @@ cudaError_t launch_attn_int8(const CUtensorMap& tm_q, const CUtensorMap& tm_k, c
                              const CUtensorMap& tm_sk, const float* sq, int Tq, int Tk, int H, uint16_t* o,
                              int64_t ldo, cudaStream_t st);
 
+// Offline SVDQuant fit (synchronous; host linear algebra between device steps).
+int64_t svdquant_workspace_bytes(int64_t n, int64_t k, int rank, int oversample, int bits, int scale_group);
+cudaError_t svdquant_fit(const uint16_t* w, int64_t n, int64_t k, int bits, bool rot, int scale_group, int rank,
+                         int oversample, int iters, const double* omegas, const double* act_rms, void* q_out,
+                         float* scales_out, double* l1, double* l2, double* errs, int* best_out, void* work,
+                         cudaStream_t st);
+
 uint32_t gemm_smem_bytes(bool g64, int r, int G);   // dynamic shared memory of one GEMM CTA
 int gemm_tile_tokens(bool g64);                     // tokens per GEMM tile
 

@@ -8,3 +8,4 @@
 #include "rbd_kv4.cu"
 #include "rbd_rope.cu"
 #include "rbd_attn.cu"
+#include "rbd_svdquant.cu"

@@ -268,3 +268,22 @@ def test_attention_validation_without_gpu():
     assert ai(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0, 2, 8, FAKE, 256, null) == 1   # no keys
     assert ai(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 2, 8, FAKE, 256, null) == 0   # no queries
     assert ai(FAKE, FAKE, FAKE, FAKE_MIS, FAKE, 4, 8, 2, 8, FAKE, 256, null) == 3
+
+
+def test_svdquant_validation_without_gpu():
+    lib = R.load()
+    null = ctypes.c_void_p(0)
+    assert lib.rbd_svdquant_workspace_bytes(384, 3072, 32, 8, q()) > 384 * 3072 * 24
+    assert lib.rbd_svdquant_workspace_bytes(384, 3072, 300, 8, q()) == -1          # rank + oversample > 256
+    assert lib.rbd_svdquant_workspace_bytes(384, 3000, 32, 8, q()) == -1           # K not a multiple of 256
+    assert lib.rbd_svdquant_workspace_bytes(384, 3072, 32, 8, q(cf=1)) == -1       # codes of weights are int8
+    f = lib.rbd_svdquant_fit
+    ok = lambda **kw: [kw.get(n, dflt) for n, dflt in (
+        ("w", FAKE), ("N", 384), ("K", 3072), ("cfg", q()), ("rank", 32), ("os", 8), ("iters", 3), ("om", FAKE),
+        ("ar", null), ("q", FAKE), ("sc", FAKE), ("l1", FAKE), ("l2", FAKE), ("errs", FAKE), ("best", null),
+        ("work", FAKE), ("stream", null))]
+    assert f(*ok(iters=0)) == 1
+    assert f(*ok(om=null)) == 1
+    assert f(*ok(rank=0)) == 1
+    assert f(*ok(N=16)) == 2                     # rank + oversample > N
+    assert f(*ok(w=FAKE_MIS)) == 3
