@@ -448,63 +448,96 @@ def run_small_m_sweep(args):
     wqfs = [wqf.clone() for _ in range(copies)]
     wbfs = [wbf.clone() for _ in range(copies)]
     torch.cuda.synchronize()
-    for fmt in ("w4a4", "nvfp4"):
-        for M in (1, 16, 64, 256, 1024):
+    # group-64 weights (the Q|K|V|gate layer's scale layout) for the E4M3-code path
+    wq4g = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    sw4g = torch.empty((N, K // 64), dtype=torch.float32, device=dev)
+    B.rbd_pack_weights_int4(w, wq4g, sw4g, 256, 64)
+    wq4gs = [wq4g.clone() for _ in range(copies)]
+    sw4gs = [sw4g.clone() for _ in range(copies)]
+    torch.cuda.synchronize()
+
+    def graph_time(fn):
+        """Median device time per call of a CUDA graph of `copies` calls fn(i)."""
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        assert R.rbd_check() == 0
+        stream = torch.cuda.Stream(device=dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(copies):
+                    fn(i)
+        for _ in range(max(args.warmup, 3)):
+            g.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) / 1e3 / copies)
+        assert R.rbd_check() == 0
+        del g
+        return statistics.median(ts)
+
+    fmts = args.formats.split(",") if args.formats else ["w4a4", "w4a4_g64", "nvfp4"]
+    mlist = [int(v) for v in args.m_list.split(",")] if args.m_list else [1, 16, 64, 256, 1024]
+    for fmt in fmts:
+        for M in mlist:
             xb = I.gaussian_bf16(2 + M, (M, K), 1.0, 0.005, 30.0)
             x = torch.from_numpy(np.ascontiguousarray(xb).view(np.int16)).view(torch.bfloat16).to(dev)
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-            if fmt == "w4a4":
+            if fmt in ("w4a4", "w4a4_g64"):
+                g64 = fmt == "w4a4_g64"
+                sg = 64 if g64 else 0
+                cf = B.CODES_E4M3 if g64 else B.CODES_INT8
                 codes = torch.empty((M, K), dtype=torch.int8, device=dev)
-                sx = torch.empty((M,), dtype=torch.float32, device=dev)
+                sx = torch.empty((M, K // 64) if g64 else (M,), dtype=torch.float32, device=dev)
+                wl, sl = (wq4gs, sw4gs) if g64 else (wq4s, sw4s)
 
-                def call(i):
-                    B.rbd_rot_quant_act(x, codes, sx, 4, 256, 0)
-                    B.rbd_w4a4_linear(codes, sx, wq4s[i], sw4s[i], y, 0, None)
-                wbytes = N * K // 2 + N * 4
-                abytes = M * (2 * K + K + 4 + 2 * N)
+                def prologue(i):
+                    B.rbd_rot_quant_act(x, codes, sx, 4, 256, sg, code_format=cf)
+
+                def gemm(i):
+                    B.rbd_w4a4_linear(codes, sx, wl[i], sl[i], y, sg, None, code_format=cf)
+                wbytes = N * K // 2 + N * 4 * (K // 64 if g64 else 1)
+                gbytes = wbytes + M * (K + 4 * (K // 64 if g64 else 1) + 2 * N)   # GEMM alone
+                abytes = M * (2 * K + K + 4 * (K // 64 if g64 else 1) + 2 * N)
             else:
                 xq = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
                 xbs = torch.empty((B.rbd_nvfp4_scale_bytes(M, K),), dtype=torch.uint8, device=dev)
                 xgs = torch.empty((1,), dtype=torch.float32, device=dev)
 
-                def call(i):
+                def prologue(i):
                     B.rbd_nvfp4_quant(x, xq, xbs, xgs, work, 256)
+
+                def gemm(i):
                     B.rbd_nvfp4_linear(xq, xbs, xgs, wqfs[i], wbfs[i], wgf, y, None)
                 wbytes = N * K // 2 + N * K // 16
+                gbytes = wbytes + M * (K // 2 + K // 16 + 2 * N)
                 abytes = M * (2 * K + 2 * K + K // 2 + K // 16 + 2 * N)   # X read twice (two passes)
-            for i in range(3):
-                call(i)
-            torch.cuda.synchronize()
-            assert R.rbd_check() == 0
-            stream = torch.cuda.Stream(device=dev)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.stream(stream):
-                with torch.cuda.graph(g, stream=stream):
-                    for i in range(copies):
-                        call(i)
-            for _ in range(max(args.warmup, 3)):
-                g.replay()
-            torch.cuda.synchronize()
-            ts = []
-            for _ in range(args.steps):
-                a = torch.cuda.Event(enable_timing=True)
-                b = torch.cuda.Event(enable_timing=True)
-                a.record()
-                g.replay()
-                b.record()
-                torch.cuda.synchronize()
-                ts.append(a.elapsed_time(b) / 1e3 / copies)
-            assert R.rbd_check() == 0
-            t = statistics.median(ts)
+
+            def layer(i):
+                prologue(i)
+                gemm(i)
+            t = graph_time(layer)
+            tg = graph_time(gemm)
+            tp = graph_time(prologue)
             gbs = (wbytes + abytes) / t / 1e9
             print(json.dumps({
                 "sweep": "small-m", "format": fmt, "M": M, "K": K, "N": N, "us_per_layer": t * 1e6,
                 "tokens_per_s": M / t, "tops": 2.0 * M * N * K / t / 1e12, "hbm_gbs": gbs,
                 "hbm_frac": gbs / peaks["hbm_gbs"], "peak_source": f"{src} copy {peaks['hbm_gbs']} GB/s",
                 "algorithmic_bytes": wbytes + abytes,
-                "timing": f"median of {args.steps} replays of a graph of {copies} layer calls on distinct weight copies"}),
+                "gemm_us": tg * 1e6, "gemm_hbm_frac": gbytes / tg / 1e9 / peaks["hbm_gbs"],
+                "prologue_us": tp * 1e6,
+                "timing": f"median of {args.steps} replays of a graph of {copies} calls on distinct weight "
+                          "copies (layer = prologue + GEMM; GEMM and prologue also timed alone)"}),
                 flush=True)
-            del g
 
 
 # ----------------------------------------------------------------------------- prologue sweep
@@ -961,6 +994,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--print-gemm-hash", action="store_true", help="print the GEMM source hash and exit")
+    ap.add_argument("--m-list", default=None,
+                    help="small-m sweep: comma-separated token counts (default 1,16,64,256,1024)")
+    ap.add_argument("--formats", default=None,
+                    help="small-m sweep: comma-separated subset of w4a4,w4a4_g64,nvfp4")
     ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4", "nvfp4", "qknorm", "peaks", "attn", "svdquant"], default=None,
                     help="instead of the headline line, print the small-token-count sweep (one line per case)")
     args = ap.parse_args()

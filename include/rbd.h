@@ -208,13 +208,21 @@ typedef struct rbd_epilogue {
  *   per-tile scale table does not fit in shared memory (group scales with a
  *   very large K) returns RBD_ERR_UNSUPPORTED.
  *   epi     may be NULL (no bias, branch or gate).
- *   y       bf16 [M, ldy], ldy >= N, ldy % 8 == 0.                           */
+ *   y       bf16 [M, ldy], ldy >= N, ldy % 8 == 0.
+ * Up to 64 tokens run on a weight-streaming kernel (16 output features per
+ * block, K split across its warps, warp-level MMAs) instead of the tiled
+ * one; results follow the same contract.  That kernel is launched with
+ * programmatic stream serialisation: it may start while the preceding
+ * kernel on the stream is still running, but before that kernel has
+ * completed it only prefetches w_packed into L2 (never stale: L2 is the
+ * point of coherence) and reads nothing else.                               */
 rbd_status rbd_w4a4_linear(const int8_t* codes, const float* sx, const uint8_t* w_packed,
                            const float* sw, int64_t M, int64_t N, int64_t K, rbd_qcfg cfg,
                            const rbd_epilogue* epi, void* y, int64_t ldy, void* stream);
 
 /* W8A8 linear (per-row INT8 ff.down): INT8 codes times INT8 weights.
- * Same contract as rbd_w4a4_linear with w8 int8 [N, K] and cfg.bits == 8.   */
+ * Same contract as rbd_w4a4_linear with w8 int8 [N, K] and cfg.bits == 8,
+ * including the weight-streaming kernel for up to 64 tokens.               */
 rbd_status rbd_w8a8_linear(const int8_t* codes, const float* sx, const int8_t* w8,
                            const float* sw, int64_t M, int64_t N, int64_t K, rbd_qcfg cfg,
                            const rbd_epilogue* epi, void* y, int64_t ldy, void* stream);

@@ -198,21 +198,6 @@ rbd_status linear_common(const int8_t* codes, const float* sx, const void* w, co
   if (e.acc_debug && (reinterpret_cast<uintptr_t>(e.acc_debug) & 3u)) return RBD_ERR_ALIGNMENT;
 
   const bool g64 = cfg.scale_group == 64;
-  if (rbd::gemm_smem_bytes(g64, e.r, G) > 227u * 1024u) return RBD_ERR_UNSUPPORTED;
-  const int tt = rbd::gemm_tile_tokens(g64);
-
-  CUtensorMap tm_x{}, tm_w{}, tm_ld{}, tm_l2{};
-  if (!make_map_2d(&tm_x, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, K, 128, tt)) return RBD_ERR_CUDA;
-  if (!W4 && !make_map_2d(&tm_w, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, K, 128, 128)) return RBD_ERR_CUDA;
-  if (e.r) {
-    if (!make_map_2d(&tm_ld, e.ld, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, e.r, M, 2 * e.r, e.r, tt))
-      return RBD_ERR_CUDA;
-    if (!make_map_2d(&tm_l2, e.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, e.r, N, 2 * e.r, e.r, 128))
-      return RBD_ERR_CUDA;
-  }
-  CUtensorMap tm_y{};
-  if (g64 && !make_map_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 2 * ldy, 32, 64, true))
-    return RBD_ERR_CUDA;
   GemmArgs a{};
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
@@ -234,6 +219,28 @@ rbd_status linear_common(const int8_t* codes, const float* sx, const void* w, co
   a.ldy = ldy;
   a.acc_debug = e.acc_debug;
   a.acc_scale = (W4 && !f8) ? 1.0f / 16.0f : 1.0f;   // the INT8 path widens a nibble q to the byte 16 q
+  a.x = reinterpret_cast<const uint8_t*>(codes);
+  a.w8 = W4 ? nullptr : static_cast<const int8_t*>(w);
+  a.ld = static_cast<const uint16_t*>(e.ld);
+  a.l2t = static_cast<const uint16_t*>(e.l2t);
+  // a few tokens: the weight-streaming kernel
+  if (M <= rbd::kSkinnyMaxM) return cuda_status(rbd::launch_skinny_gemm(W4, g64, f8, a, as_stream(stream)));
+
+  if (rbd::gemm_smem_bytes(g64, e.r, G) > 227u * 1024u) return RBD_ERR_UNSUPPORTED;
+  const int tt = rbd::gemm_tile_tokens(g64);
+
+  CUtensorMap tm_x{}, tm_w{}, tm_ld{}, tm_l2{};
+  if (!make_map_2d(&tm_x, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, K, 128, tt)) return RBD_ERR_CUDA;
+  if (!W4 && !make_map_2d(&tm_w, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, K, 128, 128)) return RBD_ERR_CUDA;
+  if (e.r) {
+    if (!make_map_2d(&tm_ld, e.ld, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, e.r, M, 2 * e.r, e.r, tt))
+      return RBD_ERR_CUDA;
+    if (!make_map_2d(&tm_l2, e.l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, e.r, N, 2 * e.r, e.r, 128))
+      return RBD_ERR_CUDA;
+  }
+  CUtensorMap tm_y{};
+  if (g64 && !make_map_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 2 * ldy, 32, 64, true))
+    return RBD_ERR_CUDA;
   a.num_m_tiles = static_cast<int>((M + tt - 1) / tt);
   a.num_tiles = a.num_m_tiles * static_cast<int>(N / 128);
   const int sms = num_sms_current();

@@ -92,31 +92,6 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-
-// Eight packed two's-complement nibbles (code k in bits 4k..4k+3) -> their eight
-// E4M3 bytes, codes 0-3 in o0 and 4-7 in o1, in order.  Two byte-permute
-// tables give the E4M3 byte of every non-negative nibble value (0..7) and of
-// every negative one (-8..-1) from the nibble's low three bits; a third permute
-// replicates each nibble's sign bit into a byte mask that selects between them.
-constexpr uint32_t kE4Pos0 = 0x44403800u;   // E4M3 of 0, 1, 2, 3
-constexpr uint32_t kE4Pos1 = 0x4E4C4A48u;   // E4M3 of 4, 5, 6, 7
-constexpr uint32_t kE4Neg0 = 0xCACCCED0u;   // E4M3 of -8, -7, -6, -5
-constexpr uint32_t kE4Neg1 = 0xB8C0C4C8u;   // E4M3 of -4, -3, -2, -1
-__device__ __forceinline__ void nibbles_to_e4m3(uint32_t pw, uint32_t& o0, uint32_t& o1) {
-  const uint32_t sel = pw & 0x77777777u;   // low three bits of every nibble
-  const uint32_t sh4 = pw << 4;            // sign bits of the even nibbles at byte msbs
-  const uint32_t selh = sel >> 16;
-  const uint32_t m0 = prmt(sh4, pw, 0xD9C8u);   // 0xFF where codes 0..3 are negative
-  const uint32_t m1 = prmt(sh4, pw, 0xFBEAu);   // likewise codes 4..7
-  o0 = (prmt(kE4Pos0, kE4Pos1, sel) & ~m0) | (prmt(kE4Neg0, kE4Neg1, sel) & m0);
-  o1 = (prmt(kE4Pos0, kE4Pos1, selh) & ~m1) | (prmt(kE4Neg0, kE4Neg1, selh) & m1);
-}
-
 }  // namespace
 
 struct SmemLayout {

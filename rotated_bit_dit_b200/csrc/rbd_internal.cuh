@@ -27,6 +27,12 @@ struct GemmArgs {
   int32_t* acc_debug;   // optional exact accumulators
   float acc_scale;      // 1/16 for widened INT4 weights, 1 for INT8
   int num_m_tiles, num_tiles;
+  // plain pointers of the operands the tiled kernel reads through tensor maps
+  // (the small-token kernel reads them directly)
+  const uint8_t* x;     // activation codes [M, K]
+  const int8_t* w8;     // INT8 weights [N, K] (W8A8 only)
+  const uint16_t* ld;   // bf16 [M, r]
+  const uint16_t* l2t;  // bf16 [N, r]
 };
 
 // e4m3: write each (4-bit) code as the E4M3 byte of equal value instead of an int8.
@@ -47,6 +53,12 @@ cudaError_t launch_lowrank_down(const uint16_t* x, int64_t M, int64_t K, int64_t
 cudaError_t launch_lowbit_gemm(bool w4, bool g64, bool f8, const CUtensorMap& tm_x, const CUtensorMap& tm_w8,
                                const CUtensorMap& tm_ld, const CUtensorMap& tm_l2, const CUtensorMap& tm_y,
                                const GemmArgs& a, int num_sms, cudaStream_t st);
+
+// Token counts up to this run on the small-token kernel (warp mma.sync with K
+// split across the warps of a 16-feature block), larger ones on the tiled one.
+constexpr int kSkinnyMaxM = 64;
+// f8: E4M3 activation codes (W4A4 with group scales only).
+cudaError_t launch_skinny_gemm(bool w4, bool g64, bool f8, const GemmArgs& a, cudaStream_t st);
 
 // Arguments of the block-scaled FP4 GEMM.
 struct NvArgs {

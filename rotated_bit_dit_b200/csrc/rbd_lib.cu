@@ -4,6 +4,7 @@
 #include "rbd_api.cu"
 #include "rbd_prologue.cu"
 #include "rbd_gemm.cu"
+#include "rbd_skinny.cu"
 #include "rbd_nvfp4.cu"
 #include "rbd_kv4.cu"
 #include "rbd_rope.cu"

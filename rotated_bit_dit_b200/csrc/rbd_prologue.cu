@@ -74,6 +74,8 @@ __global__ void __launch_bounds__(256) rot_quant_kernel(const uint16_t* __restri
                                                         int64_t ldx, float qmax, int teams, int rows,
                                                         int8_t* __restrict__ codes, float* __restrict__ scales,
                                                         NormArgs norm) {
+  // a linear launched after this kernel may start streaming its weights now
+  pdl_launch_dependents();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* xbuf = reinterpret_cast<double*>(smem_raw);        // [teams*rows][256]
   float* red = reinterpret_cast<float*>(smem_raw + (size_t)blockDim.x / kTeam * 256 * sizeof(double));
@@ -407,6 +409,7 @@ __global__ void __launch_bounds__(kLrWarps * 32, R <= 32 ? 3 : 2)
     rot_quant_lowrank_kernel(const uint16_t* __restrict__ x, int64_t M, int K, int64_t ldx, float qmax,
                              const uint16_t* __restrict__ l1t, int8_t* __restrict__ codes,
                              float* __restrict__ scales, uint16_t* __restrict__ ld) {
+  pdl_launch_dependents();   // as in rot_quant_kernel
   constexpr int NT = R / 8;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* xbuf = reinterpret_cast<double*>(smem_raw);

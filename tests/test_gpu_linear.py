@@ -75,21 +75,41 @@ VARIANTS = {
 PATHS = [(4, 0, None), (4, 64, None), (4, 64, 0), (8, 0, None), (8, 64, None)]
 
 
+# 64 tokens run on the small-token kernel, 96 on the tiled tcgen05 kernel
+@pytest.mark.parametrize("M", [64, 96])
 @pytest.mark.parametrize("variant", list(VARIANTS))
 @pytest.mark.parametrize("bits,sg,cf", PATHS)
-def test_tiny_layer_variants(variant, bits, sg, cf):
-    case = build_case(64, 256, 256, bits, sg, seed=10, cf=cf, **VARIANTS[variant])
+def test_tiny_layer_variants(variant, bits, sg, cf, M):
+    case = build_case(M, 256, 256, bits, sg, seed=10, cf=cf, **VARIANTS[variant])
     y, acc, _ = run_layer(case, acc_debug=True)
     ref = reference(case)
     assert np.array_equal(acc.astype(np.int64), exact_acc(case, ref))
     check_output(y, ref["ref64"], ref["ref_bf16"])
 
 
-@pytest.mark.parametrize("M", [1, 7, 128, 200, 333])
+@pytest.mark.parametrize("M", [1, 7, 13, 33, 64, 65, 128, 200, 333])
 @pytest.mark.parametrize("bits,sg,cf", PATHS)
 def test_ragged_tokens_several_tiles(M, bits, sg, cf):
+    # M <= 64: the small-token kernel (one to eight 8-token MMA columns, ragged);
+    # M > 64: the tiled kernel
     # N spans 3 feature tiles, K spans 6 stages (wraps the 4-deep ring), M ends ragged
     case = build_case(M, 384, 768, bits, sg, seed=20 + M, bias=True, rank=16, cf=cf)
+    y, acc, _ = run_layer(case, acc_debug=True)
+    ref = reference(case)
+    assert np.array_equal(acc.astype(np.int64), exact_acc(case, ref))
+    check_output(y, ref["ref64"], ref["ref_bf16"])
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (1, 12288, 3072),    # the Q|K|V|gate shape at one token: 768 blocks of 16 features
+    (16, 3072, 12288),   # ff.down shape: 24 groups per warp, rings wrap many times
+    (40, 128, 1280),     # 20 groups over 8 warps (uneven split), 5 token columns
+    (3, 256, 256),       # 4 groups: four of the eight warps have no work
+])
+@pytest.mark.parametrize("bits,sg,cf", PATHS)
+def test_small_token_kernel_shapes(M, N, K, bits, sg, cf):
+    case = build_case(M, N, K, bits, sg, seed=50 + M, bias=True, rank=32 if N <= 4096 else 0,
+                      gate_mode=2 if bits == 8 else 1, gate_cols=(N // 2, N), cf=cf)
     y, acc, _ = run_layer(case, acc_debug=True)
     ref = reference(case)
     assert np.array_equal(acc.astype(np.int64), exact_acc(case, ref))
