@@ -24,16 +24,16 @@
 //   attn_vt_kernel          V -> fp16, transposed to [head][channel][token];
 //   attn_int8_kernel        the attention itself, one CTA per (head, 128 queries).
 //
-// attn_int8_kernel, per CTA (11 warps):
-//   warps 0 and 10: TMA producers (Q once; K codes and key scales of 128-key
+// attn_int8_kernel, per CTA (19 warps):
+//   warps 0 and 18: TMA producers (Q once; K codes and key scales of 128-key
 //           tiles into a 2-stage ring freed by Q.K^T; V^T tiles into a 2-stage
 //           ring freed by P.V);
 //   warp 1: TMEM owner and MMA issuer: S_j = Q K_j^T (kind::i8, int32) into one
 //           of two 128-column S buffers, O += P_j V_j (kind::f16, fp32) into a
 //           third 128-column buffer;
-//   warps 2-9: softmax, two threads per query row (TMEM lane), each with 64 of
-//           the tile's keys: its part of the row of S_j (int32) is loaded once
-//           into registers, scaled, the pair's row maximum exchanged through
+//   warps 2-17: softmax, four threads per query row (TMEM lane), each with 32
+//           of the tile's keys: its part of the row of S_j (int32) is loaded once
+//           into registers, scaled, the four parts' row maxima exchanged through
 //           shared memory, keys past Tk masked, and 2^(logit - m) taken against
 //           the row's running maximum m.  m only moves when a tile's maximum exceeds it by more than 8
 //           (so P <= 256 stays well inside fp16); O is then rescaled in TMEM
@@ -55,9 +55,11 @@ namespace {
 
 constexpr int kAttnDim = 128;           // channels per head
 constexpr int kAttnTile = 128;          // queries per CTA, keys per tile
-constexpr int kAttnThreads = 352;       // 11 warps
-constexpr int kAttnVWarp = 10;          // the V producer
+constexpr int kAttnParts = 4;           // softmax threads per query row
+constexpr int kAttnPartKeys = 128 / kAttnParts;   // keys of a tile per softmax thread
 constexpr int kAttnSoftmax0 = 2;        // first softmax warp
+constexpr int kAttnVWarp = kAttnSoftmax0 + 4 * kAttnParts;   // the V producer (warp 18)
+constexpr int kAttnThreads = 32 * (kAttnVWarp + 1);          // 19 warps
 constexpr int kColsumChunk = 256;       // tokens per partial column sum
 constexpr float kLog2eRsqrtD = 0.12751743082459868f;   // log2(e) / sqrt(128)
 constexpr float kLazyRescale = 8.0f;    // base-2 headroom before the running maximum moves
@@ -78,9 +80,9 @@ constexpr uint32_t kPOff = kVOff + 4 * kVHalf;         // P, 2 buffers x 2 halve
 // tile j + 2, which waits for the softmax of tile j to release its S buffer, which
 // it does after reading the slot.
 constexpr uint32_t kSkOff = kPOff + 2 * 32768;         // key scales, 4 slots x 512 B
-constexpr uint32_t kRedOff = kSkOff + 4 * 512;         // row-maximum exchange, 2 x 2 x 128 floats
-constexpr uint32_t kBarOff = kRedOff + 2048;
-constexpr uint32_t kAttnSmem = kBarOff + 256 + 1024;   // + alignment slack
+constexpr uint32_t kRedOff = kSkOff + 4 * 512;         // row-maximum exchange, 2 x kAttnParts x 128 floats
+constexpr uint32_t kBarOff = kRedOff + 2 * kAttnParts * 128 * 4;
+constexpr uint32_t kAttnSmem = kBarOff + 512 + 1024;   // + alignment slack
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
   asm volatile(
@@ -281,7 +283,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* pv_done = bars + 11;   // [2]
   uint64_t* o_done = bars + 13;
   uint64_t* drain = bars + 14;
-  uint64_t* red_bar = bars + 15;   // [2] the pair's row maxima are in shared memory
+  uint64_t* red_bar = bars + 32;   // [2][4] the row maxima of a lane quarter's four parts are in shared memory
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 26);
 
   const uint32_t warp = warp_id(), lane = lane_id();
@@ -297,14 +299,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&v_full[b], 1);
       mbar_init(&v_empty[b], 1);
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 8);
-      mbar_init(&p_full[b], 8);
+      mbar_init(&s_empty[b], 4 * kAttnParts);
+      mbar_init(&p_full[b], 4 * kAttnParts);
       mbar_init(&pv_done[b], 1);
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
-    mbar_init(&red_bar[0], 8);
-    mbar_init(&red_bar[1], 8);
+    for (int b = 0; b < 8; ++b) mbar_init(&red_bar[b], kAttnParts);
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -331,7 +332,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 0 || warp == kAttnVWarp) {
     // ------------------------------------------------------------ TMA producers
     // warp 0: Q once, then K codes and key scales (a stage is free once its Q.K^T is
-    // done); warp 10: V^T (a stage is free once its P.V is done)
+    // done); warp 18: V^T (a stage is free once its P.V is done)
     if (lane == 0) {
       const bool kprod = warp == 0;
       bool ok = true;
@@ -404,16 +405,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
   } else if (warp < kAttnVWarp) {
     // ------------------------------------------------------------ softmax warps
-    // Warp w (2..9) covers query rows 32 (w & 3) .. +31 (its TMEM lane quarter) and
-    // keys 64 half .. +63 of every tile (half = (w - 2) >> 2): two warps per row.
-    // The pair exchanges its two row maxima through shared memory once per tile.
+    // Warp w (2..17) covers query rows 32 (w & 3) .. +31 (its TMEM lane quarter) and
+    // keys 32 part .. +31 of every tile (part = (w - 2) >> 2): four warps per row.
+    // The four exchange their row maxima through shared memory once per tile.
     const uint32_t qtr = warp & 3u;
-    const int half = ((int)warp - kAttnSoftmax0) >> 2;
+    const int part = ((int)warp - kAttnSoftmax0) >> 2;
     const int row = 32 * (int)qtr + (int)lane;                  // query row inside the tile (TMEM lane)
     const uint32_t lane_addr = (32u * qtr) << 16;
     const int qrow = q0 + row;
     const float cq = qrow < args.Tq ? __ldg(args.sq + (int64_t)h * args.Tq + qrow) * kLog2eRsqrtD : 0.f;
-    float* red = reinterpret_cast<float*>(smem + kRedOff);     // [2 tiles][2 halves][128 rows]
+    float* red = reinterpret_cast<float*>(smem + kRedOff);     // [2 tiles][kAttnParts][128 rows]
     // waits whose outcome the whole warp shares: the warp's TMEM accesses are
     // .sync.aligned, so its lanes must never part ways on a timeout
     auto wait_warp = [](uint64_t* bar, uint32_t parity) {
@@ -425,21 +426,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int s = j & 1;
       if (!wait_warp(&s_full[s], (j >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sreg[64];
-      tmem_ld32(tmem + lane_addr + s * kAttnTile + 64 * half, sreg);
-      tmem_ld32(tmem + lane_addr + s * kAttnTile + 64 * half + 32, sreg + 32);
+      uint32_t sreg[kAttnPartKeys];
+      tmem_ld32(tmem + lane_addr + s * kAttnTile + kAttnPartKeys * part, sreg);
       tmem_wait_ld();
       // u = acc * s_k (the logit is u * cq, cq = s_q log2(e) / sqrt(128) >= 0, so the row
       // maximum of u gives that of the logits); keys past Tk are left out (last tile only)
-      const float4* sk4 = reinterpret_cast<const float4*>(smem + kSkOff + (j & 3) * 512) + 16 * half;
-      const int nvalid = args.Tk - j * kAttnTile - 64 * half;   // valid keys of this half
-      const bool full = nvalid >= 64;
+      const float4* sk4 = reinterpret_cast<const float4*>(smem + kSkOff + (j & 3) * 512) + (kAttnPartKeys / 4) * part;
+      const int nvalid = args.Tk - j * kAttnTile - kAttnPartKeys * part;   // valid keys of this part
+      const bool full = nvalid >= kAttnPartKeys;
       float mx[8];   // eight independent max chains
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
       auto logits = [&](auto full_tile) {
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
+        for (int c4 = 0; c4 < kAttnPartKeys / 4; ++c4) {
           const float4 kq = sk4[c4];
           const float ks[4] = {kq.x, kq.y, kq.z, kq.w};
 #pragma unroll
@@ -460,35 +460,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[s]);
-      red[(s * 2 + half) * kAttnTile + row] = mh;
+      red[(s * kAttnParts + part) * kAttnTile + row] = mh;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&red_bar[s]);
-      if (!wait_warp(&red_bar[s], (j >> 1) & 1)) { ok = false; break; }
-      mh = fmaxf(mh, red[(s * 2 + (half ^ 1)) * kAttnTile + row]);
+      if (lane == 0) mbar_arrive(&red_bar[4 * s + qtr]);   // only the warps of these rows wait on it
+      if (!wait_warp(&red_bar[4 * s + qtr], (j >> 1) & 1)) { ok = false; break; }
+#pragma unroll
+      for (int o = 1; o < kAttnParts; ++o)
+        mh = fmaxf(mh, red[(s * kAttnParts + ((part + o) % kAttnParts)) * kAttnTile + row]);
       const float mt = mh * cq;                                  // the tile's row maximum, base 2
       // the P buffer of this tile is free once PV_{j-2} has completed
       if (j >= 2 && !wait_warp(&pv_done[s], ((j - 2) >> 1) & 1)) { ok = false; break; }
       // Each row decides for itself whether its maximum moves (both warps of the pair
       // decide alike), but the TMEM loads and stores of a rescale are warp-wide
       // (.sync.aligned): the warp rescales when any of its rows needs it, the other
-      // rows with factor 1.  Half 0 rescales O columns 0..63 and the row-sum block
-      // 128..143, half 1 columns 64..127.
+      // rows with factor 1.  Part p rescales O columns 32 p .. 32 p + 31, part 0
+      // also the row-sum block 128..143.
       const bool move = mt > m_use + kLazyRescale;
       if (j >= 1 && __any_sync(0xffffffffu, move)) {
         // O holds PV_0 .. PV_{j-1}: wait for the last of them, then scale O in TMEM
         if (!wait_warp(&pv_done[s ^ 1], ((j - 1) >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const float f = move ? ex2(m_use - mt) : 1.0f;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        {
           uint32_t ov[32];
-          tmem_ld32(t_o + lane_addr + 64 * half + 32 * c, ov);
+          tmem_ld32(t_o + lane_addr + 32 * part, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-          tmem_st32(t_o + lane_addr + 64 * half + 32 * c, ov);
+          tmem_st32(t_o + lane_addr + 32 * part, ov);
         }
-        if (half == 0) {
+        if (part == 0) {
           uint32_t ov[16];   // columns 128..143: the row sum and the unused rest
           tmem_ld16(t_o + lane_addr + kAttnDim, ov);
 #pragma unroll
@@ -498,13 +499,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_wait_st();
       }
       if (move) m_use = mt;
-      // P = 2^(u cq - m) as fp16 into this half of the tile's P buffer (row = query,
-      // 128-byte swizzle); masked keys get P = 0; the P.V MMA's ones column sums it
-      unsigned char* prow = smem + kPOff + s * 32768 + half * 16384 + row * 128;
+      // P = 2^(u cq - m) as fp16 into this part of the tile's P buffer (row = query;
+      // keys 0..63 in the first 16 KB half, 64..127 in the second, 128-byte swizzle);
+      // masked keys get P = 0; the P.V MMA's ones column sums it
+      unsigned char* prow = smem + kPOff + s * 32768 + (part >> 1) * 16384 + row * 128;
+      const int c8_0 = (part & 1) * 4;   // first 16-byte chunk of this part in the row
       const float nm = -m_use;
       auto probs = [&](auto full_tile) {
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
+        for (int c8 = 0; c8 < kAttnPartKeys / 8; ++c8) {
           uint32_t packed[4];
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
@@ -518,7 +521,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const __half2 hp = __floats2half2_rn(p0, p1);
             packed[e2] = *reinterpret_cast<const uint32_t*>(&hp);
           }
-          *reinterpret_cast<uint4*>(prow + ((c8 ^ (row & 7)) << 4)) =
+          *reinterpret_cast<uint4*>(prow + (((c8_0 + c8) ^ (row & 7)) << 4)) =
               make_uint4(packed[0], packed[1], packed[2], packed[3]);
         }
       };
@@ -529,18 +532,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[s]);
     }
-    // O / l -> bf16: this warp's 64 output channels of its query rows
+    // O / l -> bf16: this warp's 32 output channels of its query rows
     if (ok && wait_warp(o_done, 0)) {
       tc_fence_after();
       uint32_t lv[16];
       tmem_ld16(t_o + lane_addr + kAttnDim, lv);
       const float l = __uint_as_float(lv[0]);
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-      uint16_t* orow = args.o + (int64_t)qrow * args.ldo + h * kAttnDim + 64 * half;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      uint16_t* orow = args.o + (int64_t)qrow * args.ldo + h * kAttnDim + 32 * part;
+      {
+        const int c = 0;
         uint32_t ov[32];
-        tmem_ld32(t_o + lane_addr + 64 * half + 32 * c, ov);
+        tmem_ld32(t_o + lane_addr + 32 * part, ov);
         tmem_wait_ld();
         if (qrow < args.Tq) {
 #pragma unroll

@@ -19,7 +19,8 @@
 //
 // Thread mapping: a half-warp per (token, head) unit; lane i of the half owns
 // channels 8i .. 8i+7 (four pairs): one 16-byte load of x, 16 bytes each of
-// cos and sin, one 16-byte store.  In-place use (y == x) is safe: every element
+// cos and sin, one 16-byte store; the loads of a warp's units are all issued
+// before its first reduction.  In-place use (y == x) is safe: every element
 // is read and written by the same thread.
 #include <cuda_bf16.h>
 
@@ -34,7 +35,7 @@ namespace {
 constexpr int kRopeDim = 128;
 constexpr int kRopePairs = kRopeDim / 2;
 constexpr int kRopeWarps = 8;
-constexpr int kRopeSteps = 4;   // units per half-warp
+constexpr int kRopeSteps = 2;   // units per half-warp
 
 __device__ __forceinline__ void bf16x8_to_float(const uint4 v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -64,7 +65,10 @@ __global__ void __launch_bounds__(kRopeWarps * 32) qk_norm_rope_kernel(const uin
 #pragma unroll
     for (int j = 0; j < 8; ++j) g[j] = 1.f;
   }
+  // every load of the warp's units (x and the token's cos / sin) is issued
+  // before the first reduction, so a unit costs one memory latency
   uint4 xv[kRopeSteps];
+  float4 cv[kRopeSteps], sv[kRopeSteps];
   int tok[kRopeSteps];
 #pragma unroll
   for (int k = 0; k < kRopeSteps; ++k) {
@@ -73,9 +77,12 @@ __global__ void __launch_bounds__(kRopeWarps * 32) qk_norm_rope_kernel(const uin
       const int t = unit / H, h = unit - t * H;
       tok[k] = t;
       xv[k] = *reinterpret_cast<const uint4*>(x + (int64_t)t * ldx + (int64_t)h * kRopeDim + 8 * li);
+      cv[k] = __ldg(reinterpret_cast<const float4*>(cos_t + (int64_t)t * kRopePairs) + li);
+      sv[k] = __ldg(reinterpret_cast<const float4*>(sin_t + (int64_t)t * kRopePairs) + li);
     } else {
       tok[k] = -1;
       xv[k] = make_uint4(0u, 0u, 0u, 0u);
+      cv[k] = sv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
 #pragma unroll
@@ -95,9 +102,7 @@ __global__ void __launch_bounds__(kRopeWarps * 32) qk_norm_rope_kernel(const uin
     const float r = rad > 0.0 ? (float)(1.0 / sqrt(rad)) : 0.f;   // an all-zero head with eps 0 stays 0
     const int unit = unit0 + 2 * k + half;
     const int h = unit - t * H;
-    const float4 c4 = __ldg(reinterpret_cast<const float4*>(cos_t + (int64_t)t * kRopePairs) + li);
-    const float4 s4 = __ldg(reinterpret_cast<const float4*>(sin_t + (int64_t)t * kRopePairs) + li);
-    const float c[4] = {c4.x, c4.y, c4.z, c4.w}, s[4] = {s4.x, s4.y, s4.z, s4.w};
+    const float c[4] = {cv[k].x, cv[k].y, cv[k].z, cv[k].w}, s[4] = {sv[k].x, sv[k].y, sv[k].z, sv[k].w};
     uint32_t out[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
