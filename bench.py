@@ -278,6 +278,25 @@ def run_ours(args, cfg, t):
     torch.cuda.synchronize()
     e2e_t = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / 1e3, dev)
     e2e_value = whole_job_rate(world, args.steps, ops_step, e2e_t) / 1e12
+    # the end-to-end bound: the pinned-memory copy rates of this machine, one direction at a time
+    # (a step needs X in and Y out; with the copies overlapped the slower direction bounds it)
+    def copy_rate(dst, src):
+        for _ in range(2):
+            dst.copy_(src, non_blocking=True)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(5):
+            dst.copy_(src, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        return 5 * src.numel() * src.element_size() / (a.elapsed_time(b) / 1e3) / 1e9
+    yd_probe = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    xd_probe = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    d2h_gbs = copy_rate(yh, yd_probe)
+    h2d_gbs = copy_rate(xd_probe, xh)
+    del yd_probe, xd_probe
+    e2e_bound_s = max(yh.numel() * 2 / (d2h_gbs * 1e9), xh.numel() * 2 / (h2d_gbs * 1e9), t_rank / args.steps)
 
     if rank == 0:
         peaks, src = load_peaks()
@@ -308,7 +327,12 @@ def run_ours(args, cfg, t):
             "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": int(xh.numel() * 2),
                     "d2h_bytes_per_step": int(yh.numel() * 2),
                     "call": "RotatedLowBitLinear.forward_host: pinned host X in, Y out, 1024-token slices on "
-                            "two streams (copies overlap the kernels)"},
+                            "two streams (copies overlap the kernels)",
+                    "bound": {"d2h_gbs": d2h_gbs, "h2d_gbs": h2d_gbs,
+                              "value": ops_step / e2e_bound_s / 1e12,
+                              "frac": e2e_value / world / (ops_step / e2e_bound_s / 1e12),
+                              "what": "slowest of: Y device->host at the measured pinned copy rate, X "
+                                      "host->device likewise, the device step; all perfectly overlapped"}},
             "gpu_launches": 2 * args.steps,   # fused prologue + GEMM per step
             "clocks": clk.summary(),
         }
