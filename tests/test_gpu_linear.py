@@ -210,3 +210,35 @@ def test_intermediates_are_kept_per_stream():
         b1b = layer.buffers(64, torch.device("cuda"))
     assert b1[0].data_ptr() != b2[0].data_ptr() and b1[1].data_ptr() != b2[1].data_ptr()
     assert b1[0].data_ptr() == b1b[0].data_ptr()
+
+
+# The small-M sweep's layer (K = N = 3072) at every token count it times, on both kernels
+# (M <= 64 the small-token kernel, above it the tiled one): every output and accumulator.
+@pytest.mark.parametrize("M", [1, 16, 64, 256, 1024])
+@pytest.mark.parametrize("sg,cf", [(0, None), (64, None)])
+def test_small_m_sweep_layer_shapes(M, sg, cf):
+    case = dict(M=M, N=3072, K=3072, bits=4, sg=sg, cf=cf, x=I.gaussian_bf16(2 + M, (M, 3072), 1.0, 0.005, 30.0),
+                w=I.gaussian_bf16(1, (3072, 3072), 0.02), bias=None, l1=None, l2=None, gate_mode=0,
+                gate_cols=(0, 0), gate=None, residual=None)
+    y, acc, _ = run_layer(case, acc_debug=True)
+    ref = reference(case)
+    assert np.array_equal(acc.astype(np.int64), exact_acc(case, ref))
+    check_output(y, ref["ref64"], ref["ref_bf16"])
+
+
+# The 28-block stack's layer shapes at its token count (M = 16384, per-row scales, the INT4
+# and the protected INT8 layers), in the launch configuration the stack sweep times: sampled
+# rows against the oracle.
+STACK_SHAPES = [(4, 3072, 3072), (8, 3072, 3072), (4, 3072, 12288), (4, 12288, 3072), (8, 12288, 3072)]
+
+
+@pytest.mark.parametrize("bits,K,N", STACK_SHAPES)
+def test_stack_layer_shapes_sampled_rows(bits, K, N):
+    M = 16384
+    case = dict(M=M, N=N, K=K, bits=bits, sg=0, x=I.gaussian_bf16(K, (M, K), 1.0, 0.005, 30.0),
+                w=I.gaussian_bf16(7 + N, (N, K), 0.02), bias=None, l1=None, l2=None, gate_mode=0,
+                gate_cols=(0, 0), gate=None, residual=None)
+    y, _, _ = run_layer(case)
+    rows = _sample_rows(M, n=32, seed=K + N + bits)
+    ref = reference(case, rows=rows)
+    check_output(y[rows], ref["ref64"], ref["ref_bf16"])
