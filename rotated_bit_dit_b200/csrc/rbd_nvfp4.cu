@@ -208,11 +208,13 @@ constexpr int kNvTile = 128;                  // features and tokens per tile
 constexpr int kNvBK = 256;                    // K elements per stage
 constexpr uint32_t kNvOpBytes = 128 * 128;    // one operand stage
 constexpr uint32_t kNvSfBytes = 4 * 512;      // one scale stage (4 K steps)
-constexpr int kNvStages = 4;
+// pipeline stages: 4 with the low-rank branch (its tiles take the rest of
+// shared memory and its accumulator TMEM columns 384..511), 6 without
+__host__ __device__ constexpr int nv_stages(bool lr) { return lr ? 4 : 6; }
 constexpr uint32_t kNvStageBytes = 2 * kNvOpBytes + 2 * kNvSfBytes;
 constexpr uint32_t kNvLrBytes = 2 * 128 * 128;  // low-rank tiles: l2t [128 x r] and ld [128 x r], r <= 64
 __host__ __device__ constexpr uint32_t nv_smem_bytes(bool lr) {
-  return kNvStages * kNvStageBytes + (lr ? kNvLrBytes : 0u) + 1024 + 256;
+  return nv_stages(lr) * kNvStageBytes + (lr ? kNvLrBytes : 0u) + 1024 + 256;
 }
 constexpr uint32_t kNvAccCols = 2 * kNvTile;  // two accumulator buffers
 constexpr uint32_t kNvLrCol = 384;            // low-rank accumulator (after the scale regions)
@@ -228,6 +230,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023u) & ~uintptr_t(1023u));
   // stage s: A (weights) | B (tokens) | SFA | SFB
   // low-rank tiles after the stages: l2t rows (A side) then ld rows (B side)
+  constexpr int kNvStages = nv_stages(LR);
   unsigned char* lr_a = smem + kNvStages * kNvStageBytes;
   unsigned char* lr_b = lr_a + kNvLrBytes / 2;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kNvStages * kNvStageBytes + (LR ? kNvLrBytes : 0u));
