@@ -6,13 +6,17 @@ W4A4 GEMM with group-64 dequant, rank-32 branch and sigmoid gate epilogue
 (the grouped Q|K|V|gate projection, M=4096 tokens, K=3072, N=4*3072).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-    python bench.py --sweep small-m|stack|prologue|kv4|nvfp4|qknorm   (one JSON line per case)
+    python bench.py --sweep small-m|stack|prologue|ffdown|kv4|nvfp4|qknorm|attn|svdquant|peaks
+                                                            (one JSON line per case)
 
-Sweeps: small-m (K = N = 3072 layer at 1..1024 tokens, W4A4 and NVFP4, HBM
-roofline), stack (the 28-block stack of 224 linears), prologue (the
-activation prologues at the layer shapes, HBM roofline), kv4 (the INT4
-KV-cache codec, HBM roofline), nvfp4 (the NVFP4 variant at the Q|K|V|gate
-shape against the FP4 dense peak), qknorm (Q/K RMSNorm + RoPE, HBM roofline).
+Sweeps: small-m (K = N = 3072 layer at 1..1024 tokens, W4A4 row / group-64 and
+NVFP4, HBM roofline; --m-list and --formats restrict it), stack (the 28-block
+stack of 224 linears), prologue (the activation prologues at the layer shapes,
+HBM roofline), ffdown (the W8A8 ff.down layer with its gated residual), kv4
+(the INT4 KV-cache codec, HBM roofline), nvfp4 (the NVFP4 variant at the
+Q|K|V|gate shape against the FP4 dense peak), qknorm (Q/K RMSNorm + RoPE, HBM
+roofline), attn (the INT8 attention and its operand preparation), svdquant
+(the offline SVDQuant fit), peaks (measured INT8 / FP8 library GEMM ceilings).
 
 Under torchrun each rank runs its own replica on its own batch (tokens are
 independent; no collective on the data path), scaling is weak and the value
@@ -564,6 +568,74 @@ def run_small_m_sweep(args):
                 flush=True)
 
 
+# ----------------------------------------------------------------------------- ff.down layer
+def run_ffdown_sweep(args):
+    """The W8A8 ff.down layer (cfg2: M = 4096, K = 12288, N = 3072, per-row INT8, group-256
+    rotation, gated residual): the rotate/quantise prologue and the GEMM (with the gated-residual
+    epilogue) timed apart and together, each after a 256 MB L2 flush, CUDA events on the stream.
+    The GEMM against the measured INT8 ceiling; the prologue against HBM."""
+    import torch
+
+    import rotated_bit_dit_b200 as R
+    from rotated_bit_dit_b200 import _binding as B
+    from rotated_bit_dit_b200 import inputs as I
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    R.load()
+    cfg = I.CONFIGS["w8a8_ffdown"]
+    t = I.make_layer_inputs(cfg, seed=0)
+    M, K, N = cfg["M"], cfg["K"], cfg["N"]
+    up = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    x, w, res, gate = up(t["x"]), up(t["w"]), up(t["residual"]), up(t["gate"])
+    w8 = torch.empty((N, K), dtype=torch.int8, device=dev)
+    sw = torch.empty((N,), dtype=torch.float32, device=dev)
+    B.rbd_pack_weights_int8(w, w8, sw, 256, 0)
+    codes = torch.empty((M, K), dtype=torch.int8, device=dev)
+    sx = torch.empty((M,), dtype=torch.float32, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    epi = B.Epilogue(gate_mode=2, gate=gate.data_ptr(), residual=res.data_ptr(), ldr=N)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    peaks, src = load_peaks()
+    int8_peak, int8_src = int8_peak_tops(peaks, src)
+    pro = lambda: B.rbd_rot_quant_act(x, codes, sx, 8, 256, 0)
+    gemm = lambda: B.rbd_w8a8_linear(codes, sx, w8, sw, y, 0, epi)
+
+    def layer():
+        pro()
+        gemm()
+
+    def timed(fn):
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        assert R.rbd_check() == 0
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) / 1e3)
+        assert R.rbd_check() == 0
+        return statistics.median(ts)
+
+    with ClockSampler(dev.index) as clk:
+        tp, tg, tl = timed(pro), timed(gemm), timed(layer)
+    ops = 2.0 * M * N * K
+    pro_bytes = M * K * 2 + M * K + M * 4
+    print(json.dumps({
+        "sweep": "ffdown", "M": M, "K": K, "N": N, "prologue_us": tp * 1e6, "gemm_us": tg * 1e6,
+        "layer_us": tl * 1e6, "gemm_tops": ops / tg / 1e12, "gemm_frac_int8": ops / tg / 1e12 / int8_peak,
+        "layer_tops": ops / tl / 1e12, "prologue_hbm_frac": pro_bytes / tp / 1e9 / peaks["hbm_gbs"],
+        "int8_peak_source": int8_src, "clocks": clk.summary(),
+        "timing": f"median of {args.steps} calls each, every call after a 256 MB L2 flush"}), flush=True)
+
+
 # ----------------------------------------------------------------------------- prologue sweep
 def run_prologue_sweep(args):
     """The memory-bound activation prologues at the layer shapes: rotate/quantise, the normalising
@@ -1022,7 +1094,7 @@ def main():
                     help="small-m sweep: comma-separated token counts (default 1,16,64,256,1024)")
     ap.add_argument("--formats", default=None,
                     help="small-m sweep: comma-separated subset of w4a4,w4a4_g64,nvfp4")
-    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4", "nvfp4", "qknorm", "peaks", "attn", "svdquant"], default=None,
+    ap.add_argument("--sweep", choices=["small-m", "stack", "prologue", "kv4", "nvfp4", "qknorm", "peaks", "attn", "svdquant", "ffdown"], default=None,
                     help="instead of the headline line, print the small-token-count sweep (one line per case)")
     args = ap.parse_args()
     if args.print_gemm_hash:
@@ -1045,6 +1117,9 @@ def main():
         return
     if args.sweep == "prologue":
         run_prologue_sweep(args)
+        return
+    if args.sweep == "ffdown":
+        run_ffdown_sweep(args)
         return
     if args.sweep == "kv4":
         run_kv4_sweep(args)
