@@ -328,7 +328,7 @@ __device__ __forceinline__ bool g64_tile(const GemmArgs& args, uint32_t tcol, ui
     for (int j = 0; j < kG64Half; ++j) {
       if (j < jmax) {
         const float o = (j & 1) ? y[j >> 1].y : y[j >> 1].x;
-        const float rres = __uint_as_float((uint32_t)*rp << 16);
+        const float rres = __uint_as_float((uint32_t)__ldg(rp) << 16);   // read-only path, as in row mode
         *yp = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(gv, o, rres)));
       }
       yp += args.ldy;
@@ -790,13 +790,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint16_t* yp = args.y + mbase * args.ldy + n;
       const int64_t ystep = args.ldy;
       if (args.gate_mode == 2) {
+        // the residual through the read-only path: each element is read once, by the
+        // thread that then writes the output there (so even y == residual is safe),
+        // and the loads may move ahead of the stores instead of waiting behind them
         const uint16_t* rp = args.residual + mbase * args.ldr + n;
         const int64_t rstep = args.ldr;
 #pragma unroll
         for (int j = 0; j < EC; ++j) {
           if (j < jmax) {
             const float o = (j & 1) ? y[j >> 1].y : y[j >> 1].x;
-            const float rres = __uint_as_float((uint32_t)*rp << 16);
+            const float rres = __uint_as_float((uint32_t)__ldg(rp) << 16);
             *yp = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(gv, o, rres)));
           }
           yp += ystep;
