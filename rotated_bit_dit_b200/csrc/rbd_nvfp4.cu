@@ -413,7 +413,9 @@ __global__ void __launch_bounds__(kNvThreads, 1)
           float o = fmaf(__uint_as_float(v[j >> 4][j & 15]), gsc, bias);
           if (R) o += __uint_as_float(vl[j >> 4][j & 15]);
           if (args.gate_mode == 2) {
-            o = fmaf(gv, o, __uint_as_float((uint32_t)args.residual[m * args.ldr + n] << 16));
+            // read-only path: each residual element is read once, by the thread that then
+            // writes the output there, so the loads may run ahead of the stores
+            o = fmaf(gv, o, __uint_as_float((uint32_t)__ldg(args.residual + m * args.ldr + n) << 16));
           } else if (sig) {
             o = __frcp_rn(1.0f + __expf(-o));
           }

@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(kSkThreads) skinny_gemm_kernel(const GemmArgs 
     }
     if (sig) o = __frcp_rn(1.0f + __expf(-o));
     if (args.gate_mode == 2) {
-      const float rres = __uint_as_float((uint32_t)args.residual[(int64_t)m * args.ldr + n] << 16);
+      const float rres = __uint_as_float((uint32_t)__ldg(args.residual + (int64_t)m * args.ldr + n) << 16);
       o = fmaf(e_gv, o, rres);
     }
     args.y[(int64_t)m * args.ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
