@@ -775,3 +775,21 @@ def test_attention_tiled_fp16_p_stays_within_the_output_tolerance():
         out[:, h] = acc / l[:, None]
     got = O.f64_to_bf16(out)
     check_output(got.reshape(Tq, -1), ref64.reshape(Tq, -1), O.f64_to_bf16(ref64).reshape(Tq, -1))
+
+
+def test_exact_to_f32_matches_an_independent_rounding():
+    """exact_to_f32 (exact rational -> float32, nearest, ties to even) against numpy's own
+    float64 -> float32 conversion, which rounds the same way, on values a float64 holds exactly:
+    random magnitudes over the normal and subnormal range, exact halfway points between
+    neighbouring float32 values (both parities of the lower neighbour), and signs."""
+    rng = np.random.default_rng(7)
+    vals = list(rng.standard_normal(2000) * np.exp2(rng.integers(-140, 100, 2000)))
+    # exact ties: midpoint of f and its upper neighbour, for f with even and odd significands
+    for f in np.float32([1.0, 1.0 + 2.0 ** -23, 3.0, 1.5 + 2.0 ** -22, 1e-40, 7.0e-39, 123.456]):
+        up = np.nextafter(f, np.float32(np.inf))
+        vals.append((float(f) + float(up)) / 2.0)
+        vals.append(-(float(f) + float(up)) / 2.0)
+    for v in vals:
+        want = np.float32(np.float64(v))
+        got = O.exact_to_f32(Fraction(float(v)))
+        assert got == want and np.signbit(got) == np.signbit(want), (v, got, want)
